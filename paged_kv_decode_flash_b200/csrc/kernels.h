@@ -1,0 +1,20 @@
+// kernels.h -- launchers of the libpagedattn kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace pa {
+
+// Plain split-KV decode on CUDA cores (any block_size % 16 == 0, fp16/q8_0).
+size_t decode_simt_smem_bytes(int rows);
+cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
+
+// Log-sum-exp merge of split partials into fp16 rows.
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+
+// Per-row key-resolution record (debug / tests).
+cudaError_t launch_trace(const DecodeParams& p, int32_t* trace, cudaStream_t stream);
+
+}  // namespace pa

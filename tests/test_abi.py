@@ -1,0 +1,114 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol
+include/pagedattn.h declares, and its host-side logic (argument checks,
+workspace sizing) behaves.  No call here reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from paged_kv_decode_flash_b200 import build
+    build.build()
+    from paged_kv_decode_flash_b200 import binding
+    return binding.lib()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(paged_attn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("paged_attn_decode", "paged_attn_merge", "paged_attn_workspace_size",
+                 "paged_attn_get_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared but not exported"
+
+
+def dims(**kw):
+    from paged_kv_decode_flash_b200.binding import Dims
+    d = dict(num_seqs=1, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+             max_blocks_per_seq=3841, num_blocks=3841, workspace=None, workspace_bytes=0)
+    d.update(kw)
+    return Dims(**d)
+
+
+def test_workspace_size_host_only(L):
+    d = dims()
+    n = L.paged_attn_workspace_size(ctypes.byref(d), 8)
+    assert n > 256 and n % 256 == 0
+    # more query tokens need at least as much
+    assert L.paged_attn_workspace_size(ctypes.byref(d), 8) >= L.paged_attn_workspace_size(ctypes.byref(d), 1)
+    # invalid shapes -> 0
+    for bad in (dims(num_q_heads=30), dims(block_size=8), dims(head_dim=64), dims(num_seqs=0)):
+        assert L.paged_attn_workspace_size(ctypes.byref(bad), 8) == 0
+    assert L.paged_attn_workspace_size(ctypes.byref(d), 0) == 0
+    assert L.paged_attn_workspace_size(ctypes.byref(d), 9) == 0
+    assert L.paged_attn_workspace_size(None, 1) == 0
+
+
+def test_decode_rejects_bad_arguments_on_host(L):
+    from paged_kv_decode_flash_b200 import binding as b
+    d = dims(workspace=4096, workspace_bytes=1 << 30)
+    p = ctypes.c_void_p(1 << 20)  # never dereferenced: checks fail first
+    args = lambda **kw: dict(dict(q=p, k=p, v=p, bt=p, cl=p, nq=8, causal=1, window=0,
+                                  scale=0.088, dt=0, out=p), **kw)
+
+    def call(dd, a):
+        return L.paged_attn_decode(ctypes.byref(dd) if dd is not None else None, a["q"], a["k"],
+                                   a["v"], a["bt"], a["cl"], a["nq"], a["causal"], a["window"],
+                                   a["scale"], a["dt"], a["out"], None)
+
+    assert call(None, args()) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(q=None)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(nq=0)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(nq=9)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(causal=2)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(window=-1)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(dt=7)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(scale=float("nan"))) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(q=ctypes.c_void_p((1 << 20) + 2))) == b.PA_ERR_INVALID_ARG  # misaligned
+    assert call(dims(head_dim=64, workspace=4096, workspace_bytes=1 << 30), args()) == b.PA_ERR_UNSUPPORTED
+    assert call(dims(num_q_heads=128, num_kv_heads=8, workspace=4096, workspace_bytes=1 << 30),
+                args()) == b.PA_ERR_UNSUPPORTED  # 8 tokens x 16 heads per KV head > 64 rows
+    assert call(dims(workspace=None), args()) == b.PA_ERR_WORKSPACE
+    assert call(dims(workspace=4100, workspace_bytes=1 << 30), args()) == b.PA_ERR_WORKSPACE
+
+
+def test_merge_rejects_bad_arguments_on_host(L):
+    from paged_kv_decode_flash_b200 import binding as b
+    p = ctypes.c_void_p(1 << 20)
+    assert L.paged_attn_merge(None, p, 2, 4, 128, p, None, None) == b.PA_ERR_INVALID_ARG
+    assert L.paged_attn_merge(p, p, 0, 4, 128, p, None, None) == b.PA_ERR_INVALID_ARG
+    assert L.paged_attn_merge(p, p, 2, -1, 128, p, None, None) == b.PA_ERR_INVALID_ARG
+    assert L.paged_attn_merge(p, p, 2, 4, 96, p, None, None) == b.PA_ERR_UNSUPPORTED
+
+
+def test_status_strings(L):
+    from paged_kv_decode_flash_b200 import binding as b
+    for code in range(-6, 1):
+        assert L.paged_attn_status_string(code)
+    assert b.status_string(b.PA_ERR_BAD_BLOCK_INDEX) == "block_table entry out of range"
+
+
+def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
+    from paged_kv_decode_flash_b200 import binding as b
+    monkeypatch.setattr(b, "_LIB", None)
+    monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        b.lib()

@@ -1,0 +1,271 @@
+"""GPU parity: libpagedattn (through its C ABI) against the fp64 oracle on the
+same seeded inputs, plus bit-exact invariants of the GPU path itself.
+
+Tolerance (tests/parity.py): max-abs 2e-3 and max-rel 1e-2 against
+max(|oracle|, 1e-3), on the fp16 output.  Block-index resolution and masking
+are checked bit-exactly through the trace entry point, through NaN poisoning
+of every never-visible key and through closed forms.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+from parity import assert_parity
+from paged_kv_decode_flash_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.load()
+
+
+@pytest.fixture(scope="module")
+def B():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_decode_flash_b200 import binding
+    binding.lib()
+    return binding
+
+
+def run(B, case):
+    out, dec = B.decode_case(case)
+    torch.cuda.synchronize()
+    assert dec.get_error() == 0
+    return out.cpu().numpy(), dec
+
+
+def sampled_rows(case, n, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(case.rows, size=min(n, case.rows), replace=False).tolist())
+    rows |= {0, case.rows - 1}
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
+# small problems, every row against the oracle
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", range(3))
+def test_tiny_config(B, orc, seed):
+    case = gen.tiny(seed)
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, f"tiny seed {seed}")
+
+
+def _sweep_cases():
+    rng = np.random.default_rng(2024)
+    for t in range(40):
+        nq = int(rng.integers(1, 9))
+        G = int(rng.choice([1, 2, 4, 6, 8]))
+        while nq * G > 64:
+            G //= 2
+        Hkv = int(rng.choice([1, 2, 3]))
+        bs = int(rng.choice([16, 32, 64]))
+        causal = int(rng.integers(0, 2))
+        window = int(rng.choice([0, 0, 1, 7, 100, 513]))
+        dt = gen.KV_Q8_0 if t % 3 == 2 else gen.KV_FP16
+        nseq = int(rng.integers(1, 4))
+        lens = [int(x) for x in rng.integers(nq, 1500, size=nseq)]
+        if t % 7 == 0:
+            lens[0] = nq  # the shortest legal context
+        extra = int(rng.integers(0, 3))
+        mbps = max((l + bs - 1) // bs for l in lens) + extra
+        yield gen.make_case(seed=5000 + t, context_lens=tuple(lens), n_query=nq,
+                            num_q_heads=Hkv * G, num_kv_heads=Hkv, block_size=bs,
+                            causal=causal, window=window, kv_dtype=dt, spare_blocks=3,
+                            max_blocks_per_seq=mbps)
+
+
+@pytest.mark.parametrize("case", list(_sweep_cases()),
+                         ids=lambda c: f"B{c.num_seqs}_nq{c.n_query}_G{c.group}_Hkv{c.num_kv_heads}"
+                         f"_bs{c.block_size}_c{c.causal}_w{c.window}_dt{c.kv_dtype}")
+def test_random_sweep(B, orc, case):
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, "sweep")
+
+
+def test_sliding_window_config_and_nan_invariance(B, orc):
+    case = gen.sliding_window(0)
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, "sliding window")
+    # the 1408 out-of-window blocks hold NaN; zeroing them changes no bit
+    clean = gen.Case(**case.__dict__)
+    clean.k_cache = np.nan_to_num(case.k_cache, nan=0.0)
+    clean.v_cache = np.nan_to_num(case.v_cache, nan=0.0)
+    out2, _ = run(B, clean)
+    assert np.array_equal(out.view(np.uint16), out2.view(np.uint16))
+
+
+def test_single_key_is_bit_exact(B):
+    for dt in (gen.KV_FP16, gen.KV_Q8_0):
+        case = gen.make_case(seed=7, context_lens=(1, 1), n_query=1, num_q_heads=8,
+                             num_kv_heads=2, kv_dtype=dt, spare_blocks=4)
+        out, _ = run(B, case)
+        import pins
+        for s in range(2):
+            V = pins.dense_kv(case, s, "v")
+            for h in range(8):
+                want = V[h // 4, 0].astype(np.float16)  # fp16 values (exact for fp16 cache)
+                if dt == gen.KV_FP16:
+                    assert np.array_equal(out[s, 0, h].view(np.uint16), want.view(np.uint16))
+                else:  # q8_0 value q*d rounded once to fp16
+                    assert np.array_equal(out[s, 0, h], want)
+
+
+def test_window_one_returns_own_value(B):
+    case = gen.make_case(seed=8, context_lens=(300,), n_query=4, num_q_heads=4,
+                         num_kv_heads=1, causal=1, window=1)
+    out, _ = run(B, case)
+    import pins
+    V = pins.dense_kv(case, 0, "v")[0]
+    for i in range(4):
+        for h in range(4):
+            assert np.array_equal(out[0, i, h].view(np.uint16),
+                                  V[300 - 4 + i].astype(np.float16).view(np.uint16))
+
+
+def test_block_permutation_bit_identical(B):
+    case = gen.make_case(seed=9, context_lens=(2000, 777), n_query=4, num_q_heads=16,
+                         num_kv_heads=4, causal=1, window=900, spare_blocks=10)
+    out, _ = run(B, case)
+    perm = np.random.default_rng(1).permutation(case.num_blocks)
+    k2 = np.empty_like(case.k_cache); k2[perm] = case.k_cache
+    v2 = np.empty_like(case.v_cache); v2[perm] = case.v_cache
+    c2 = gen.Case(**{**case.__dict__, "k_cache": k2, "v_cache": v2,
+                     "block_table": perm[case.block_table].astype(np.int32)})
+    out2, _ = run(B, c2)
+    assert np.array_equal(out.view(np.uint16), out2.view(np.uint16))
+
+
+def test_sequence_independent_of_neighbours(B):
+    """Each sequence's output depends only on its own data (the varlen
+    indexing bug in 'Flash-Next (vLLM)' on the gfx1030 wiki reused a global
+    chunk index): change the other sequences' lengths and values, keep the
+    shapes, and sequence 1 must not change by a bit."""
+    a = gen.make_case(seed=10, context_lens=(500, 1200, 64), n_query=3, num_q_heads=8,
+                      num_kv_heads=2, causal=1, max_blocks_per_seq=80)
+    out_a, _ = run(B, a)
+    b = gen.Case(**a.__dict__)
+    b.context_lens = a.context_lens.copy()
+    b.context_lens[0], b.context_lens[2] = 3, 1279
+    b.q = a.q.copy(); b.q[0] = -a.q[0]; b.q[2] = a.q[2] * 2
+    rows_other = [bb for s in (0, 2) for bb in a.block_table[s] if bb != a.num_blocks - 1]
+    b.k_cache = a.k_cache.copy(); b.v_cache = a.v_cache.copy()
+    b.k_cache[rows_other] = 0.5; b.v_cache[rows_other] = -0.25
+    b.block_table = a.block_table.copy()
+    # sequence 2 grows into blocks that were padding: point them at fresh data
+    out_b, _ = run(B, b)
+    assert np.array_equal(out_a[1].view(np.uint16), out_b[1].view(np.uint16))
+
+
+def test_batch_matches_each_sequence_alone(B, orc):
+    case = gen.make_case(seed=11, context_lens=(900, 33, 2500, 8), n_query=2,
+                         num_q_heads=8, num_kv_heads=2, causal=1)
+    out, _ = run(B, case)
+    for s in range(4):
+        c1 = gen.Case(**{**case.__dict__, "num_seqs": 1, "q": case.q[s:s + 1].copy(),
+                         "block_table": case.block_table[s:s + 1].copy(),
+                         "context_lens": case.context_lens[s:s + 1].copy()})
+        o1, _ = run(B, c1)
+        ref, _ = orc.attend(c1)
+        assert_parity(out[s:s + 1], ref, f"batch seq {s}")
+        assert_parity(o1, ref, f"alone seq {s}")
+
+
+def test_trace_is_bit_exact(B, orc):
+    cases = [gen.tiny(0), gen.sliding_window(0)] + list(_sweep_cases())[:12]
+    for case in cases:
+        dev = B.case_to_device(case)
+        dec = B.PagedDecode.for_case(case)
+        t = dec.trace(dev["block_table"], dev["context_lens"], causal=case.causal,
+                      window=case.window)
+        got = t.cpu().numpy().reshape(-1, 5)
+        assert np.array_equal(got, orc.trace(case)), case.name
+
+
+def test_merge_entry_point(B, orc):
+    rng = np.random.default_rng(12)
+    for S, rows in ((1, 5), (7, 33), (148, 64)):
+        po = rng.standard_normal((S, rows, 128)).astype(np.float32)
+        pl = (rng.standard_normal((S, rows)) * 20).astype(np.float32)
+        pl[rng.random((S, rows)) < 0.2] = -np.inf  # empty splits
+        if rows > 1:
+            pl[:, 1] = -np.inf  # a row no split saw
+        po[pl == -np.inf] = np.nan  # an empty split's output is never read
+        out, lse = B.merge(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda())
+        ref, ref_lse = orc.merge(np.nan_to_num(po, nan=0.0).astype(np.float64), pl.astype(np.float64))
+        assert_parity(out.cpu().numpy(), ref, f"merge S={S}")
+        l = lse.cpu().numpy()
+        fin = np.isfinite(ref_lse)
+        assert np.array_equal(np.isfinite(l), fin)
+        assert np.max(np.abs(l[fin] - ref_lse[fin])) < 1e-4
+
+
+def test_bad_block_index_is_flagged(B):
+    case = gen.make_case(seed=13, context_lens=(200,), n_query=1, num_q_heads=4,
+                         num_kv_heads=1)
+    case.block_table[0, 3] = case.num_blocks + 5
+    out, dec = B.decode_case(case)
+    assert dec.get_error() == B.PA_ERR_BAD_BLOCK_INDEX
+    assert dec.get_error() == 0  # cleared by the read
+    assert np.all(np.isfinite(out.cpu().numpy()))
+
+
+def test_bad_context_len_is_flagged_and_rows_zeroed(B):
+    case = gen.make_case(seed=14, context_lens=(100, 50), n_query=4, num_q_heads=4,
+                         num_kv_heads=1, max_blocks_per_seq=7)
+    case.context_lens[1] = 7 * 16 + 1  # beyond the table's capacity
+    out, dec = B.decode_case(case)
+    assert dec.get_error() == B.PA_ERR_BAD_CONTEXT_LEN
+    o = out.cpu().numpy()
+    assert np.all(o[1] == 0)
+    case.context_lens[1] = 3  # fewer keys than query tokens
+    out, dec = B.decode_case(case)
+    assert dec.get_error() == B.PA_ERR_BAD_CONTEXT_LEN
+
+
+def test_cuda_graph_replay_matches_eager(B):
+    case = gen.make_case(seed=15, context_lens=(3000,), n_query=8, num_q_heads=32,
+                         num_kv_heads=8, causal=1)
+    dev = B.case_to_device(case)
+    dec = B.PagedDecode.for_case(case)
+    kw = dict(causal=1, window=0, scale=case.scale, kv_dtype=case.kv_dtype)
+    eager = dec(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["context_lens"], **kw)
+    out = torch.empty_like(eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        dec(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["context_lens"],
+            out=out, stream=s, **kw)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dec(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["context_lens"],
+            out=out, stream=torch.cuda.current_stream(), **kw)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads: sampled rows against the oracle
+# ---------------------------------------------------------------------------
+@pytest.mark.slow
+@pytest.mark.parametrize("name,nrows", [("spec_verify_61k", 24), ("decode_200k", 12),
+                                        ("mixed_q8_0", 24), ("sliding_window", 256)])
+def test_full_size_sampled(B, orc, name, nrows):
+    case = gen.CONFIGS[name](0)
+    out, _ = run(B, case)
+    o = out.reshape(case.rows, case.head_dim)
+    assert np.all(np.isfinite(o)), "non-finite output at full size"
+    rows = sampled_rows(case, nrows)
+    ref, _ = orc.attend_rows(case, rows)
+    assert_parity(o[rows], ref, name)
