@@ -153,6 +153,29 @@ int paged_attn_trace(const pa_dims* dims, const int32_t* block_table,
  * current device (host only). */
 int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query);
 
+/* Allocation-free variant of paged_attn_decode.  The paper has no
+ * counterpart: it exists for callers that cannot give the library device
+ * memory of its own -- programs whose host owns every byte of device memory
+ * (a serving engine with one fixed pool planned at start-up, a plug-in host
+ * without an allocator) or hot paths that must not call cudaMalloc, which can
+ * implicitly synchronise the device.  Same arguments, layouts and results as
+ * paged_attn_decode; the workspace fields of *dims are ignored.  The split
+ * partials live in one array of PA_NOALLOC_SCRATCH_BYTES inside the
+ * library's device image, held by every GPU that loads the library until
+ * exit; shapes that need more return PA_ERR_WORKSPACE before anything is
+ * enqueued.  All calls on a device share that array: calls whose work
+ * overlaps on the GPU race and corrupt each other, so order them (one
+ * stream, or events).  The first call on a device looks up the array's
+ * device address and caches it; make it before any stream capture begins.
+ * Device-side data errors are handled as in paged_attn_decode (masked keys,
+ * zeroed rows) but are not reported: the status word is cleared per call. */
+#define PA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* block_table,
+                              const int32_t* context_lens, int32_t n_query,
+                              int32_t causal, int32_t window, float scale,
+                              int32_t kv_dtype, void* out, void* stream);
+
 /* Static string for a pa_status. */
 const char* paged_attn_status_string(int32_t status);
 
