@@ -205,7 +205,7 @@ def bench_ours(args, rank, world, dist):
             "ms_per_step": total_ms / steps,
             "us_median": per_call[len(per_call) // 2], "us_min": per_call[0],
             "us_p90": per_call[min(len(per_call) - 1, int(0.9 * len(per_call)))],
-            "clocks": clk.summary(), "splits": dec.num_splits,
+            "clocks": clk.summary(), "splits": dec.num_splits(case.kv_dtype),
         }
         if with_e2e:
             res["e2e"] = e2e(case, dec, base, pools[0], steps=min(steps, 500))

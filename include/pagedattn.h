@@ -79,7 +79,8 @@ typedef enum {
   PA_ERR_WORKSPACE = -3,      /* workspace missing, misaligned or too small */
   PA_ERR_CUDA = -4,           /* a CUDA runtime call or launch failed */
   PA_ERR_BAD_BLOCK_INDEX = -5,/* device saw block_table entry out of range */
-  PA_ERR_BAD_CONTEXT_LEN = -6 /* device saw context_lens out of range */
+  PA_ERR_BAD_CONTEXT_LEN = -6,/* device saw context_lens out of range */
+  PA_ERR_TIMEOUT = -7         /* a device-side wait gave up (kernel left early) */
 } pa_status;
 
 /* Static shapes of one call.  Host memory, read during the call only. */
@@ -132,9 +133,11 @@ int paged_attn_merge(const float* partial_out, const float* partial_lse,
                      void* out, float* out_lse, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device-side data-error
- * flag of the workspace: PA_OK, PA_ERR_BAD_BLOCK_INDEX or
- * PA_ERR_BAD_CONTEXT_LEN (the first of these if both were raised), or
- * PA_ERR_CUDA if the stream reports an error. */
+ * flag of the workspace: PA_OK, PA_ERR_TIMEOUT, PA_ERR_BAD_BLOCK_INDEX or
+ * PA_ERR_BAD_CONTEXT_LEN (the first of these that was raised, in that order),
+ * or PA_ERR_CUDA if the stream reports an error.  PA_ERR_TIMEOUT means a
+ * pipeline wait inside a kernel passed its time limit (about a second): the
+ * kernel released its resources and returned, and its output is not valid. */
 int paged_attn_get_error(const pa_dims* dims, void* stream);
 
 /* Debug: the key-resolution record of every row, computed on the device
@@ -149,9 +152,9 @@ int paged_attn_trace(const pa_dims* dims, const int32_t* block_table,
                      int32_t causal, int32_t window, int32_t* trace,
                      void* stream);
 
-/* Number of key splits paged_attn_decode uses for these shapes on the
- * current device (host only). */
-int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query);
+/* Number of key splits paged_attn_decode uses for these shapes and cache
+ * type on the current device (host only; negative pa_status on error). */
+int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
 
 /* Allocation-free variant of paged_attn_decode.  The paper has no
  * counterpart: it exists for callers that cannot give the library device

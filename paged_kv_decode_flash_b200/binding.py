@@ -24,6 +24,7 @@ PA_ERR_WORKSPACE = -3
 PA_ERR_CUDA = -4
 PA_ERR_BAD_BLOCK_INDEX = -5
 PA_ERR_BAD_CONTEXT_LEN = -6
+PA_ERR_TIMEOUT = -7
 
 KV_FP16 = _inputs.KV_FP16
 KV_Q8_0 = _inputs.KV_Q8_0
@@ -73,7 +74,7 @@ def lib() -> ctypes.CDLL:
             L.paged_attn_get_error.restype = ctypes.c_int
             L.paged_attn_trace.argtypes = [P, vp, vp, i32, i32, i32, vp, vp]
             L.paged_attn_trace.restype = ctypes.c_int
-            L.paged_attn_num_splits.argtypes = [P, i32]
+            L.paged_attn_num_splits.argtypes = [P, i32, i32]
             L.paged_attn_num_splits.restype = ctypes.c_int32
             L.paged_attn_status_string.argtypes = [i32]
             L.paged_attn_status_string.restype = ctypes.c_char_p
@@ -151,9 +152,8 @@ class PagedDecode:
                    block_size=case.block_size, max_blocks_per_seq=case.max_blocks_per_seq,
                    num_blocks=case.num_blocks, n_query=case.n_query, device=device)
 
-    @property
-    def num_splits(self) -> int:
-        n = lib().paged_attn_num_splits(ctypes.byref(self.dims), self.n_query)
+    def num_splits(self, kv_dtype: int = KV_FP16) -> int:
+        n = lib().paged_attn_num_splits(ctypes.byref(self.dims), self.n_query, int(kv_dtype))
         if n < 0:
             raise PagedAttnError(n, "num_splits")
         return n

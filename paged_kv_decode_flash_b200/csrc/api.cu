@@ -45,15 +45,36 @@ int check_dims(const pa_dims* d, int n_query) {
   return PA_OK;
 }
 
-int plan_splits(const pa_dims* d, long long target_ctas, int* blocks_per_split) {
+// splits = target CTAs / (sequences x KV heads), at least 128 keys per
+// split.  `fill` rounds up (the CUDA-core kernel, several CTAs per SM) or
+// down (the tensor-core kernel, one CTA per SM: a second wave would double
+// the time).
+int plan_splits(const pa_dims* d, long long target_ctas, bool round_up, int* blocks_per_split) {
   const long long min_blocks = ceil_div(kMinKeysPerSplit, d->block_size);
   const long long max_splits = std::max(1LL, ceil_div(d->max_blocks_per_seq, min_blocks));
   const long long per_split = (long long)d->num_seqs * d->num_kv_heads;
-  long long splits = std::max(1LL, ceil_div(target_ctas, per_split));
-  splits = std::min(splits, max_splits);
+  long long splits = round_up ? ceil_div(target_ctas, per_split) : target_ctas / per_split;
+  splits = std::max(1LL, std::min(splits, max_splits));
   const long long bps = ceil_div(d->max_blocks_per_seq, splits);
   *blocks_per_split = (int)bps;
   return (int)ceil_div(d->max_blocks_per_seq, bps);
+}
+
+// Which kernel a call uses, and its split plan.
+struct Plan {
+  bool tensor_cores;
+  int splits, blocks_per_split;
+};
+
+Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
+  Plan pl{};
+  const int rows = n_query * (d->num_q_heads / d->num_kv_heads);
+  pl.tensor_cores = decode_tc_supported(kv_dtype, rows, d->num_blocks, d->num_kv_heads,
+                                        d->block_size);
+  pl.splits = pl.tensor_cores ? plan_splits(d, sms, false, &pl.blocks_per_split)
+                              : plan_splits(d, (long long)sms * kCtasPerSm, true,
+                                            &pl.blocks_per_split);
+  return pl;
 }
 
 struct WsLayout {
@@ -89,17 +110,17 @@ extern "C" {
 size_t paged_attn_workspace_size(const pa_dims* dims, int32_t n_query) {
   if (check_dims(dims, n_query) != PA_OK) return 0;
   int bps = 0;
-  const int splits = plan_splits(dims, kMaxTargetCtas, &bps);
+  const int splits = plan_splits(dims, kMaxTargetCtas, true, &bps);
   return ws_layout(dims, n_query, splits).total;
 }
 
-int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query) {
+int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_dtype) {
   const int rc = check_dims(dims, n_query);
   if (rc != PA_OK) return rc;
+  if (kv_dtype != PA_KV_FP16 && kv_dtype != PA_KV_Q8_0) return PA_ERR_INVALID_ARG;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  int bps = 0;
-  return plan_splits(dims, (long long)sms * kCtasPerSm, &bps);
+  return make_plan(dims, n_query, kv_dtype, sms).splits;
 }
 
 int paged_attn_workspace_init(const pa_dims* dims, void* stream) {
@@ -129,8 +150,8 @@ int paged_attn_decode(const pa_dims* dims, const void* q, const void* k_cache,
 
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  int bps = 0;
-  const int splits = plan_splits(dims, (long long)sms * kCtasPerSm, &bps);
+  const Plan plan = make_plan(dims, n_query, kv_dtype, sms);
+  const int splits = plan.splits, bps = plan.blocks_per_split;
   const WsLayout w = ws_layout(dims, n_query, splits);
   if (dims->workspace_bytes < w.total) return PA_ERR_WORKSPACE;
 
@@ -161,7 +182,8 @@ int paged_attn_decode(const pa_dims* dims, const void* q, const void* k_cache,
   p.flags = reinterpret_cast<unsigned*>(ws);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (launch_decode_simt(p, st) != cudaSuccess) return PA_ERR_CUDA;
+  const cudaError_t e = plan.tensor_cores ? launch_decode_tc(p, st) : launch_decode_simt(p, st);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
 
   MergeParams m{};
   m.part_out = p.part_out;
@@ -208,6 +230,7 @@ int paged_attn_get_error(const pa_dims* dims, void* stream) {
     return PA_ERR_CUDA;
   if (cudaMemsetAsync(dims->workspace, 0, sizeof(flags), st) != cudaSuccess) return PA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return PA_ERR_CUDA;
+  if (flags & kFlagTimeout) return PA_ERR_TIMEOUT;
   if (flags & kFlagBadBlock) return PA_ERR_BAD_BLOCK_INDEX;
   if (flags & kFlagBadLen) return PA_ERR_BAD_CONTEXT_LEN;
   return PA_OK;
@@ -249,6 +272,7 @@ const char* paged_attn_status_string(int32_t status) {
     case PA_ERR_CUDA: return "CUDA runtime error";
     case PA_ERR_BAD_BLOCK_INDEX: return "block_table entry out of range";
     case PA_ERR_BAD_CONTEXT_LEN: return "context length out of range";
+    case PA_ERR_TIMEOUT: return "a device-side wait timed out; output invalid";
     default: return "unknown status";
   }
 }

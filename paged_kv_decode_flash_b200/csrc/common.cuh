@@ -20,7 +20,7 @@ constexpr size_t kWsHeader = 256;      // status header at the start of the work
 constexpr int kChunk = 16;             // keys per gather unit (block_size % 16 == 0)
 
 // Device-side data-error flags (bits of the first uint32 of the workspace).
-enum : unsigned { kFlagBadBlock = 1u, kFlagBadLen = 2u };
+enum : unsigned { kFlagBadBlock = 1u, kFlagBadLen = 2u, kFlagTimeout = 4u };
 
 enum KvDtype : int { kKvFp16 = 0, kKvQ8_0 = 1 };
 

@@ -101,7 +101,7 @@ def test_merge_rejects_bad_arguments_on_host(L):
 
 def test_status_strings(L):
     from paged_kv_decode_flash_b200 import binding as b
-    for code in range(-6, 1):
+    for code in range(-7, 1):
         assert L.paged_attn_status_string(code)
     assert b.status_string(b.PA_ERR_BAD_BLOCK_INDEX) == "block_table entry out of range"
 
