@@ -10,16 +10,18 @@
 // left for the log-sum-exp merge.  Masks and block-table resolution follow
 // section "Bug 2: the drafter read freed memory".
 //
-// Hardware mapping (one CTA per SM, 6 warps):
-//   warp 0      TMA producer: resolves the block table, loads whole 16-key
-//               chunks of K and V (two 64-column halves each, 128-byte
-//               swizzle) into a 3-stage ring of 128-key tiles.
+// Hardware mapping (one CTA per SM, 11 warps):
+//   warps 0, 10 TMA producers for K and for V: resolve the block table and
+//               load whole 16-key chunks (two 64-column halves each, 128-byte
+//               swizzle) into separate 3-slot rings of 128-key tiles; K slots
+//               are released as soon as QK^T has read them, so K runs ahead.
 //   warp 1      MMA issuer (one thread): S^T = K Q^T with M = 128 keys and
-//               N = the query rows (16 or 32), then O^T = V^T P^T with
+//               N = the query rows, then O^T = V^T [P_hi | P_lo]^T with
 //               M = 128 head_dim lanes; accumulators live in TMEM.
-//   warps 2-5   softmax and correction: thread = key for S (row max by a
-//               warp transpose-reduction plus one named barrier), thread =
-//               head_dim element for O (running accumulators in registers).
+//   warps 2-9   two softmax warpgroups, each owning half of the query rows:
+//               thread = key for S (row max by a warp transpose-reduction
+//               plus one named barrier per group), thread = head_dim element
+//               for O (running accumulators in registers).
 // Putting keys and head_dim on the MMA's M side keeps the tensor core free of
 // padding even at 4-32 query rows.
 //
@@ -52,49 +54,60 @@ using namespace sm100;
 
 constexpr int kTileKeys = 128;                 // keys per pipeline tile (M of S^T)
 constexpr int kChunksPerTile = kTileKeys / kChunk;
-constexpr int kStages = 3;
+constexpr int kStages = 3;                     // slots per K ring and per V ring
 constexpr uint32_t kHalfBytes = kTileKeys * 128;   // 64 fp16 columns of 128 keys
 constexpr uint32_t kKVBytes = 2 * kHalfBytes;      // one K (or V) tile
-constexpr uint32_t kStageBytes = 2 * kKVBytes;     // K then V
 constexpr uint32_t kChunkBytes = kChunk * 128;     // one 16-key half-chunk (TMA box)
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kGroups = 2;                     // softmax warpgroups (split the rows)
+constexpr int kSoftmaxThreads = 128;           // per warpgroup
+constexpr int kVWarp = 2 + kGroups * 4;        // the V producer's warp
+constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr int kPShift = 14;                    // weights scaled by 2^14 before fp16
 
 enum : int {
-  BAR_FULL = 0,     // [3] TMA tile landed
-  BAR_EMPTY = 3,    // [3] stage consumed (PV done)
-  BAR_SFULL = 6,    // [2] S^T in TMEM
-  BAR_SEMPTY = 8,   // [2] S^T read by the softmax warps
-  BAR_PFULL = 10,   // P written to shared memory
-  BAR_PEMPTY = 11,  // P consumed by the PV product
-  BAR_OFULL = 12,   // [2] O^T of one tile in TMEM
-  BAR_OEMPTY = 14,  // [2] O^T read by the correction
-  BAR_DONE = 16,    // every MMA finished
-  BAR_COUNT = 17
+  BAR_KFULL = 0,    // [3] K tile landed
+  BAR_KEMPTY = 3,   // [3] K tile read by QK^T
+  BAR_VFULL = 6,    // [3] V tile landed
+  BAR_VEMPTY = 9,   // [3] V tile read by PV
+  BAR_SFULL = 12,   // [2] S^T in TMEM
+  BAR_SEMPTY = 14,  // [2] S^T read by the softmax warps
+  BAR_PFULL = 16,   // P written to shared memory
+  BAR_PEMPTY = 17,  // P consumed by the PV product
+  BAR_OFULL = 18,   // [2] O^T of one tile in TMEM
+  BAR_OEMPTY = 20,  // [2] O^T read by the softmax warps
+  BAR_DONE = 22,    // every MMA finished
+  BAR_COUNT = 23
 };
 
-template <int NR>
-struct Layout {
-  static constexpr uint32_t kQ = kStages * kStageBytes;
+// RW query rows per softmax warpgroup; NR = the MMA's N for S (>= 16).
+template <int RW>
+struct Cfg {
+  static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
+  static constexpr uint32_t kK = 0;                                 // K ring
+  static constexpr uint32_t kV = kStages * kKVBytes;                // V ring
+  static constexpr uint32_t kQ = 2 * kStages * kKVBytes;
   static constexpr uint32_t kQHalf = NR * 128;
-  static constexpr uint32_t kPHi = kQ + 2 * kQHalf;
-  static constexpr uint32_t kPBytes = kTileKeys * NR * 2;
-  static constexpr uint32_t kPLo = kPHi + kPBytes;
-  static constexpr uint32_t kRed = kPLo + kPBytes;            // float [2][4][32]
-  static constexpr uint32_t kAlpha = kRed + 2 * 4 * 32 * 4;   // float [2][32]
-  static constexpr uint32_t kLsum = kAlpha + 2 * 32 * 4;      // float [4][32]
-  static constexpr uint32_t kBars = kLsum + 4 * 32 * 4;       // uint64 [24]
-  static constexpr uint32_t kMisc = kBars + 24 * 8;           // small ints
+  // P^T of one tile: 2*NR "rows" (the fp16 high parts of the NR query rows,
+  // then their residuals), so one MMA with N = 2*NR multiplies both.
+  static constexpr uint32_t kP = kQ + 2 * kQHalf;
+  static constexpr uint32_t kPBytes = kTileKeys * 2 * NR * 2;
+  static constexpr uint32_t kRed = kP + kPBytes;                    // float [2 grp][2][4][32]
+  static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4][32]
+  static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
+  static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [8 warps][2][32]
+  static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [32]
+  static constexpr uint32_t kMisc = kBars + 32 * 8;                 // small ints
   static constexpr uint32_t kTotal = kMisc + 64;
-  static constexpr uint32_t kTmemCols = 4 * NR;              // S[2], O[2]
+  // TMEM columns: S^T[2] (NR each) then O^T[2] (2*NR each: high | residual).
+  static constexpr uint32_t kTmemUsed = 6 * NR;
+  static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
+                                        : kTmemUsed <= 128 ? 128 : 256;
 };
 
 struct Misc {
   uint32_t tmem_base;
   int abort;
-  uint32_t chunk_mask[kStages];
-  int n_consumed;
+  int k_consumed, v_consumed;
 };
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
@@ -104,19 +117,21 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
                : "l"(p));
   return r;
 }
-
 __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
 }
+__device__ __forceinline__ void sts_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
 
-// Warp transpose-reduction: lane l ends with op over all 32 lanes of row
-// (l % NR) in v[0].
-template <int NR, bool kMax>
-__device__ __forceinline__ float warp_row_reduce(float (&v)[NR], int lane) {
+// Warp transpose-reduction over the 32 lanes (= 32 keys): lane l ends with
+// the reduction of row (l % RW) in the return value.
+template <int RW, bool kMax>
+__device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
 #pragma unroll
-  for (int n = NR, o = NR / 2; n > 1; n >>= 1, o >>= 1) {
+  for (int n = RW, o = RW / 2; n > 1; n >>= 1, o >>= 1) {
     const bool upper = (lane & o) != 0;
 #pragma unroll
     for (int i = 0; i < n / 2; ++i) {
@@ -126,25 +141,28 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[NR], int lane) {
       v[i] = kMax ? fmaxf(keep, got) : keep + got;
     }
   }
-  if constexpr (NR == 16) {
-    const float got = __shfl_xor_sync(0xffffffffu, v[0], 16);
+#pragma unroll
+  for (int o = RW; o < 32; o <<= 1) {
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], o);
     v[0] = kMax ? fmaxf(v[0], got) : v[0] + got;
   }
   return v[0];
 }
 
-template <int NR>
+template <int RW>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using Lay = Layout<NR>;
+  using C = Cfg<RW>;
+  constexpr int NR = C::NR;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the __shared__ array by pointer
+  // arithmetic so that accesses through it stay shared-space loads/stores.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  Misc* misc = reinterpret_cast<Misc*>(smem + Lay::kMisc);
+  Misc* misc = reinterpret_cast<Misc*>(smem + C::kMisc);
   volatile int* abort = &misc->abort;
-  auto bar = [&](int i) { return sbase + Lay::kBars + 8u * i; };
+  auto bar = [&](int i) { return sbase + C::kBars + 8u * i; };
 
   const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -156,8 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- the CTA's key range (uniform across the CTA) -----------------------
   const int L = p.context_lens[s];
   int k0 = 0, k1 = -1;
-  const bool len_ok = context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size);
-  if (len_ok) {
+  if (context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size)) {
     int lo_u, hi_u;
     union_range(L, nq, p.causal, p.window, lo_u, hi_u);
     const long long sk0 = (long long)split * p.blocks_per_split * p.block_size;
@@ -177,43 +194,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int base = (k0 / kChunk) * kChunk;
   const int ntiles = (k1 + 1 - base + kTileKeys - 1) / kTileKeys;
+  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
+
+  const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
+  const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
 
   // ---- set-up ---------------------------------------------------------------
   if (warp == 1) {
-    tmem_alloc(sbase + Lay::kMisc + offsetof(Misc, tmem_base), Lay::kTmemCols);
+    tmem_alloc(sbase + C::kMisc + offsetof(Misc, tmem_base), C::kTmemCols);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar(BAR_FULL + i), 1);
-      mbar_init(bar(BAR_EMPTY + i), 1);
+      mbar_init(bar(BAR_KFULL + i), 1);
+      mbar_init(bar(BAR_KEMPTY + i), 1);
+      mbar_init(bar(BAR_VFULL + i), 1);
+      mbar_init(bar(BAR_VEMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_SFULL + i), 1);
-      mbar_init(bar(BAR_SEMPTY + i), 4);
+      mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
       mbar_init(bar(BAR_OFULL + i), 1);
-      mbar_init(bar(BAR_OEMPTY + i), 4);
+      mbar_init(bar(BAR_OEMPTY + i), 4 * kGroups);
     }
-    mbar_init(bar(BAR_PFULL), 4);
+    mbar_init(bar(BAR_PFULL), 4 * kGroups);
     mbar_init(bar(BAR_PEMPTY), 1);
     mbar_init(bar(BAR_DONE), 1);
     misc->abort = 0;
-    misc->n_consumed = 0;
+    misc->k_consumed = misc->v_consumed = 0;
     fence_mbar_init();
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < kVWarp) {
     // Q rows of this KV head -> shared memory, K-major with 128-byte swizzle:
     // row n, 16-byte chunk c of half h at h*NR*128 + n*128 + ((c ^ n%8) * 16).
+    // Rows >= R are zero; so are P's padding rows (never written later).  A
+    // negative scale is moved into Q (an exact sign flip) so that the kernel
+    // only ever multiplies scores by a non-negative factor.
     const int t = threadIdx.x - 64;
-    for (int c = t; c < NR * 16; c += kSoftmaxThreads) {
+    const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+    for (int c = t; c < NR * 16; c += kGroups * kSoftmaxThreads) {
       const int n = c / 16, cc = c % 16, h = cc / 8, k8 = cc % 8;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (n < R) {
         const long long qrow = ((long long)s * nq + n / G) * Hq + kvh * G + (n % G);
         v = ldg_nc_v4(p.q + qrow * kHeadDim + cc * 8);
+        v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
       }
-      sts_v4(sbase + Lay::kQ + h * Lay::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
+      sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
     }
+    for (uint32_t off = t * 16; off < C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
+      sts_v4(sP + off, make_uint4(0, 0, 0, 0));
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -221,133 +251,134 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
 
-  const uint32_t sQ = sbase + Lay::kQ;
-  const uint32_t sPhi = sbase + Lay::kPHi, sPlo = sbase + Lay::kPLo;
-  auto sK = [&](int st) { return sbase + st * kStageBytes; };
-  auto sV = [&](int st) { return sbase + st * kStageBytes + kKVBytes; };
-
-  if (warp == 0) {
-    // ======================= TMA producer ==================================
-    const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
+  if (warp == 0 || warp == kVWarp) {
+    // ======================= TMA producers (K: warp 0, V: last warp) =======
+    // Lane c < 8 owns chunk c of each tile; its block-table entry for the
+    // next tile is read one iteration early so the read overlaps the wait.
+    const bool is_k = warp == 0;
+    const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
+    const uint32_t ring = is_k ? sKr : sVr;
+    const int bfull = is_k ? BAR_KFULL : BAR_VFULL, bempty = is_k ? BAR_KEMPTY : BAR_VEMPTY;
+    const int c = lane;
+    auto lookup = [&](int t, long long& phys) {
+      const int key0 = base + t * kTileKeys + c * kChunk;
+      const bool want = t < ntiles && c < kChunksPerTile && key0 <= k1 && key0 + kChunk - 1 >= k0;
+      phys = want ? (long long)table[key0 / p.block_size] : 0;
+      return want;
+    };
+    long long ph_cur = 0, ph_nxt = 0;
+    bool w_cur = lookup(0, ph_cur);
     int issued = 0;
     for (int t = 0; t < ntiles; ++t) {
+      const bool w_nxt = lookup(t + 1, ph_nxt);
       const int st = t % kStages;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar(BAR_EMPTY + st), ((t / kStages) & 1) ^ 1, abort);
+      if (lane == 0) ok = mbar_wait(bar(bempty + st), ((t / kStages) & 1) ^ 1, abort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const int c = lane;
-      const int key0 = base + t * kTileKeys + c * kChunk;
-      bool want = c < kChunksPerTile && key0 <= k1 && key0 + kChunk - 1 >= k0;
-      long long phys = 0;
-      if (want) {
-        phys = table[key0 / p.block_size];
-        if (phys < 0 || phys >= p.num_blocks) {
-          atomicOr(p.flags, kFlagBadBlock);
-          want = false;
-        }
+      bool want = w_cur;
+      if (want && (ph_cur < 0 || ph_cur >= p.num_blocks)) {
+        if (is_k) atomicOr(p.flags, kFlagBadBlock);  // masked, never dereferenced
+        want = false;
       }
       const uint32_t mask = __ballot_sync(0xffffffffu, want);
-      const int row = want ? (int)((phys * p.num_kv_heads + kvh) * p.block_size +
-                                   key0 % p.block_size)
-                           : 0;
+      const int key0 = base + t * kTileKeys + c * kChunk;
+      const int row =
+          want ? (int)((ph_cur * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) : 0;
       int rows[kChunksPerTile];
 #pragma unroll
       for (int cc = 0; cc < kChunksPerTile; ++cc) rows[cc] = __shfl_sync(0xffffffffu, row, cc);
-      if (lane == 0) {  // the thread that saw the stage free issues its copies
-        misc->chunk_mask[st] = mask;
-        mbar_arrive_expect_tx(bar(BAR_FULL + st), __popc(mask) * 4 * kChunkBytes);
-        const uint32_t fb = bar(BAR_FULL + st);
+      if (lane == 0) {  // the thread that saw the slot free issues its copies
+        const uint32_t fb = bar(bfull + st);
+        const uint32_t dst = ring + st * kKVBytes;
+        mbar_arrive_expect_tx(fb, __popc(mask) * 2 * kChunkBytes);
 #pragma unroll
         for (int cc = 0; cc < kChunksPerTile; ++cc) {
           if (!((mask >> cc) & 1u)) continue;
-          tma_load_2d(sK(st) + cc * kChunkBytes, &tmap_k, 0, rows[cc], fb);
-          tma_load_2d(sK(st) + kHalfBytes + cc * kChunkBytes, &tmap_k, 64, rows[cc], fb);
-          tma_load_2d(sV(st) + cc * kChunkBytes, &tmap_v, 0, rows[cc], fb);
-          tma_load_2d(sV(st) + kHalfBytes + cc * kChunkBytes, &tmap_v, 64, rows[cc], fb);
+          tma_load_2d(dst + cc * kChunkBytes, tmap, 0, rows[cc], fb);
+          tma_load_2d(dst + kHalfBytes + cc * kChunkBytes, tmap, 64, rows[cc], fb);
         }
       }
       __syncwarp();
       issued = t + 1;
+      ph_cur = ph_nxt;
+      w_cur = w_nxt;
     }
     __syncthreads();  // (A) every role finished its loop
     if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
       volatile int no_abort = 0;
-      for (int t = misc->n_consumed; t < issued; ++t)
-        mbar_wait(bar(BAR_FULL + t % kStages), (t / kStages) & 1, &no_abort);
+      for (int t = is_k ? misc->k_consumed : misc->v_consumed; t < issued; ++t)
+        mbar_wait(bar(bfull + t % kStages), (t / kStages) & 1, &no_abort);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer ====================================
     if (lane == 0) {
       const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
-      const uint32_t id_pv = idesc_f16_f32(128, NR, true, true);
-      auto issue_qk = [&](int t) {
-        const int st = t % kStages;
-        const uint32_t d = tmem + (t % 2) * NR;
+      const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
+      // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
+      // start-address field is the low 14 bits, addresses stay < 256 KB).
+      const uint64_t dK = smem_desc(sKr, 16, 1024, kSwizzle128B);
+      const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
+      const uint64_t dV = smem_desc(sVr, kHalfBytes, 1024, kSwizzle128B);
+      const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
+      int nqk = 0;  // QK^T products issued (tiles whose K was consumed)
+      // Issue QK^T of tile nqk if its K tile and S buffer are ready (or wait
+      // for them when `block`).  1 = issued, 0 = not ready, -1 = gave up.
+      auto try_qk = [&](bool block) -> int {
+        if (nqk >= ntiles) return 0;
+        const uint32_t f = bar(BAR_KFULL + nqk % kStages), e = bar(BAR_SEMPTY + nqk % 2);
+        const uint32_t pf = (nqk / kStages) & 1, pe = ((nqk / 2) & 1) ^ 1;
+        if (block) {
+          if (!(mbar_wait(f, pf, abort) && mbar_wait(e, pe, abort))) return -1;
+        } else if (!(mbar_test_wait(f, pf) && mbar_test_wait(e, pe))) {
+          return 0;
+        }
+        tc_fence_after();
+        const uint64_t so = (uint64_t)((nqk % kStages) * kKVBytes) >> 4;
+        const uint32_t d = tmem + (nqk % 2) * NR;
 #pragma unroll
         for (int k = 0; k < kHeadDim / 16; ++k) {
-          const uint64_t a = smem_desc(sK(st) + (k / 4) * kHalfBytes + (k % 4) * 32, 16, 1024,
-                                       kSwizzle128B);
-          const uint64_t b = smem_desc(sQ + (k / 4) * Lay::kQHalf + (k % 4) * 32, 16, 1024,
-                                       kSwizzle128B);
-          tc_mma_f16_ss(d, a, b, id_qk, k > 0);
+          const uint64_t ko = ((k / 4) * kHalfBytes + (k % 4) * 32) >> 4;
+          const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
+          tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
         }
+        tc_commit(bar(BAR_SFULL + nqk % 2));
+        tc_commit(bar(BAR_KEMPTY + nqk % kStages));
+        ++nqk;
+        return 1;
       };
-      auto issue_pv = [&](int t) {
-        const int st = t % kStages;
-        const uint32_t d = tmem + 2 * NR + (t % 2) * NR;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t sp = half == 0 ? sPhi : sPlo;
-#pragma unroll
-          for (int k = 0; k < kTileKeys / 16; ++k) {
-            const uint64_t a = smem_desc(sV(st) + k * 2048, kHalfBytes, 1024, kSwizzle128B);
-            const uint64_t b = smem_desc(sp + k * 2 * NR * 16, NR * 16, 128, kSwizzleNone);
-            tc_mma_f16_ss(d, a, b, id_pv, (half | k) != 0);
-          }
-        }
-      };
-      auto qk_ready = [&](int t, bool block) {
-        const uint32_t f = bar(BAR_FULL + t % kStages), e = bar(BAR_SEMPTY + t % 2);
-        const uint32_t pf = (t / kStages) & 1, pe = ((t / 2) & 1) ^ 1;
-        if (!block) return mbar_test_wait(f, pf) && mbar_test_wait(e, pe);
-        return mbar_wait(f, pf, abort) && mbar_wait(e, pe, abort);
-      };
-      int consumed = 0;
-      bool ok = ntiles > 0 && qk_ready(0, true);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-        tc_commit(bar(BAR_SFULL + 0));
-        consumed = 1;
-      }
+      int npv = 0;
+      bool ok = true;
       for (int t = 0; ok && t < ntiles; ++t) {
-        bool next_done = false;
-        if (t + 1 < ntiles && qk_ready(t + 1, false)) {
-          tc_fence_after();
-          issue_qk(t + 1);
-          tc_commit(bar(BAR_SFULL + (t + 1) % 2));
-          consumed = t + 2;
-          next_done = true;
+        if (nqk <= t && try_qk(true) < 0) { ok = false; break; }  // QK(t) comes first
+        if (nqk == t + 1) try_qk(false);
+        // Wait for P(t), issuing QK(t+1) as soon as its K tile lands.
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait_ns(bar(BAR_PFULL), t & 1, 200)) {
+          if (nqk == t + 1) try_qk(false);
+          if (*abort || globaltimer() - t0 > kWaitLimitNs) { *abort = 1; ok = false; break; }
         }
-        ok = mbar_wait(bar(BAR_PFULL), t & 1, abort) &&
+        if (!ok) break;
+        ok = mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, abort) &&
              mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(t);
+        const uint64_t so = (uint64_t)((t % kStages) * kKVBytes) >> 4;
+        const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
+#pragma unroll
+        for (int k = 0; k < kTileKeys / 16; ++k) {
+          const uint64_t vo = (k * 2048) >> 4;
+          const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
+          tc_mma_f16_ss(d, dV + so + vo, dP + po, id_pv, k > 0);
+        }
         tc_commit(bar(BAR_OFULL + t % 2));
         tc_commit(bar(BAR_PEMPTY));
-        tc_commit(bar(BAR_EMPTY + t % kStages));
-        if (t + 1 < ntiles && !next_done) {
-          ok = qk_ready(t + 1, true);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(t + 1);
-          tc_commit(bar(BAR_SFULL + (t + 1) % 2));
-          consumed = t + 2;
-        }
+        tc_commit(bar(BAR_VEMPTY + t % kStages));
+        npv = t + 1;
+        if (nqk == t + 1) try_qk(false);
       }
-      misc->n_consumed = consumed;
+      misc->k_consumed = nqk;
+      misc->v_consumed = npv;
       tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
       volatile int no_abort = 0;
       mbar_wait(bar(BAR_DONE), 0, &no_abort);
@@ -356,164 +387,218 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();  // (A)
   } else {
     // ======================= softmax + correction ==========================
-    const int q4 = warp & 3;             // TMEM lane quarter of this warp
-    const int j = q4 * 32 + lane;        // key within the tile / head_dim element
+    // Warpgroup g handles rows [g*RW, g*RW + RW); its warps cover the four
+    // TMEM lane quarters, i.e. keys (for S) and head_dim elements (for O).
+    const int g = (warp - 2) / 4, widx = (warp - 2) % 4;
+    const int row0 = g * RW;
+    const int q4 = warp & 3;
+    const int j = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + Lay::kRed);      // [2][4][32]
-    float* alpha_s = reinterpret_cast<float*>(smem + Lay::kAlpha);  // [2][32]
-    float* lsum = reinterpret_cast<float*>(smem + Lay::kLsum);      // [4][32]
-    const int widx = warp - 2;
+    float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
+    float* alpha_s = reinterpret_cast<float*>(smem + C::kAlpha);             // [4][32]
+    float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
+    float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
+    const uint32_t bar_id = 1 + g;
+    const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
 
+    // Per query token, the visible key range; keys inside every token's
+    // range (and the CTA's) see all rows: the fast path of interior tiles.
     int tlo[kMaxQuery], thi[kMaxQuery];
+    int lo_all = k0, hi_all = k1;
 #pragma unroll
     for (int i = 0; i < kMaxQuery; ++i) {
       tlo[i] = 1;
       thi[i] = 0;
-      if (i < nq) key_range(L, nq, i, p.causal, p.window, tlo[i], thi[i]);
+      if (i < nq) {
+        key_range(L, nq, i, p.causal, p.window, tlo[i], thi[i]);
+        lo_all = max(lo_all, tlo[i]);
+        hi_all = min(hi_all, thi[i]);
+      }
     }
     const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
+    const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
 
-    float acc[NR], lpart[NR];
+    float acc[RW], lpart[RW];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) acc[r] = lpart[r] = 0.f;
-    float m_lane = -INFINITY;  // running max of row lane % NR (log2 domain)
+    for (int r = 0; r < RW; ++r) acc[r] = lpart[r] = 0.f;
+    float m_lane = -INFINITY;  // running raw-score max of row row0 + lane % RW
     bool ok = true;
+    // Block-table entry of this thread's key, one tile ahead.
+    auto phys_of = [&](int t) -> long long {
+      const int key = base + t * kTileKeys + j;
+      return (t < ntiles && key >= k0 && key <= k1) ? (long long)table[key / p.block_size] : -1;
+    };
+    long long ph_cur = phys_of(0);
 
-    // Iteration t scores tile t and folds tile t-1's O^T into the registers;
-    // the extra last iteration only folds.
-    for (int t = 0; t <= ntiles; ++t) {
-     if (t < ntiles) {
-      const int sb = t % 2, st = t % kStages;
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
-      float sv[NR];
+    // Iteration t scores tile t and folds tile t-2's O^T (finished long ago)
+    // into the register accumulators; the two extra iterations only fold.
+    // Tile u's rescale factors live in alpha_s[u % 4].
+    for (int t = 0; t < ntiles + 2; ++t) {
+      const bool has_s = t < ntiles, has_o = t >= 2;
+      const int sb = t % 2, st = t % kStages, ob = t % 2;  // O of tile t-2 sits in buffer t%2
+      const long long ph_nxt = phys_of(t + 1);
+      if (has_o)
+        ok = __all_sync(0xffffffffu,
+                        ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
+      if (has_s)
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+      float sv[RW], oh[RW], ol[RW];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) sv[r] = 0.f;
+      for (int r = 0; r < RW; ++r) sv[r] = oh[r] = ol[r] = 0.f;
       if (ok) {
         tc_fence_after();
-        tmem_ld16<0>(tmem + lane_off + sb * NR, sv);
-        if constexpr (NR == 32) tmem_ld16<16 % NR>(tmem + lane_off + sb * NR + 16, sv);
+        if (has_o) {
+          tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + row0, oh);
+          tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + NR + row0, ol);
+        }
+        if (has_s) tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
         tmem_ld_wait();
         tc_fence_before();
       }
       __syncwarp();
-      if (ok && lane == 0) mbar_arrive(bar(BAR_SEMPTY + sb));
-      ok = __all_sync(0xffffffffu,
-                      ok && mbar_wait(bar(BAR_FULL + st), (t / kStages) & 1, abort));  // complete
+      if (ok && lane == 0) {
+        if (has_o) mbar_arrive(bar(BAR_OEMPTY + ob));
+        if (has_s) mbar_arrive(bar(BAR_SEMPTY + sb));
+      }
 
-      // Which rows see this key?  (Only keys of loaded chunks inside the
-      // CTA's range; the per-token ranges are the ones key_range gives.)
-      const int key = base + t * kTileKeys + j;
-      const uint32_t cmask = ok ? misc->chunk_mask[st] : 0u;
       uint32_t rmask = 0;
-      if (((cmask >> (j / kChunk)) & 1u) && key >= k0 && key <= k1) {
+      if (has_s) {
+        // Which rows see this key?  Keys of out-of-range blocks see none.
+        const int key = base + t * kTileKeys + j;
+        if (ph_cur >= 0 && ph_cur < p.num_blocks) {
+          if (key >= lo_all && key <= hi_all) {
+            rmask = all_rows;
+          } else if (key >= k0 && key <= k1) {
 #pragma unroll
-        for (int i = 0; i < kMaxQuery; ++i)
-          if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
-      }
-      float sc[NR], red_in[NR];
-#pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        sc[r] = ((rmask >> r) & 1u) ? sv[r] * p.scale_log2 : -INFINITY;
-        red_in[r] = sc[r];
-      }
-      const float wmax = warp_row_reduce<NR, true>(red_in, lane);
-      if (lane < NR) red[(sb * 4 + widx) * 32 + lane] = wmax;
-      named_bar_sync(1, kSoftmaxThreads);
-      const int rl = lane % NR;
-      float tmax = red[(sb * 4 + 0) * 32 + rl];
-      tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
-      tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
-      tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
-      const float m_new = fmaxf(m_lane, tmax);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_lane - m_new);
-      m_lane = m_new;
-      if (widx == 0 && lane < NR) alpha_s[sb * 32 + lane] = alpha;
-
-      // Scaled weights, split into fp16 high part + fp16 residual.
-      uint32_t phi[NR / 2], plo[NR / 2];
-#pragma unroll
-      for (int r = 0; r < NR; r += 2) {
-        float pr[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float mr = __shfl_sync(0xffffffffu, m_new, r + e);
-          const float ar = __shfl_sync(0xffffffffu, alpha, r + e);
-          const float x = sc[r + e];
-          pr[e] = (x == -INFINITY) ? 0.f : exp2f(x - mr + (float)kPShift);
-          lpart[r + e] = fmaf(lpart[r + e], ar, pr[e]);
+            for (int i = 0; i < kMaxQuery; ++i)
+              if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
+          }
         }
-        const __half2 h = __floats2half2_rn(pr[0], pr[1]);
-        const float2 hf = __half22float2(h);
-        const __half2 l2 = __floats2half2_rn(pr[0] - hf.x, pr[1] - hf.y);
-        phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-        plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-      }
-
-      // A key no row can see must not reach the PV product: zero its V row.
-      if (ok && rmask == 0) {
-        const uint4 z = make_uint4(0, 0, 0, 0);
+        const uint32_t rm = rmask >> row0;
+        float tmp[RW];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          sts_v4(sV(st) + j * 128 + c * 16, z);
-          sts_v4(sV(st) + kHalfBytes + j * 128 + c * 16, z);
-        }
+        for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
+        const float wmax = warp_row_reduce<RW, true>(tmp, lane);
+        if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
       }
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_PEMPTY), (t & 1) ^ 1, abort));
-      if (ok) {
-        // P^T as no-swizzle MN-major core matrices: [key/8][row/8][key%8][row%8].
-#pragma unroll
-        for (int rg = 0; rg < NR / 8; ++rg) {
-          const uint32_t off = ((j >> 3) * (NR / 8) + rg) * 128 + (j & 7) * 16;
-          sts_v4(sPhi + off, make_uint4(phi[rg * 4], phi[rg * 4 + 1], phi[rg * 4 + 2], phi[rg * 4 + 3]));
-          sts_v4(sPlo + off, make_uint4(plo[rg * 4], plo[rg * 4 + 1], plo[rg * 4 + 2], plo[rg * 4 + 3]));
-        }
-        fence_proxy_async_smem();
-      }
+      // Reconverge before the group barrier: a warp that arrives diverged
+      // (after the lane-predicated store above) makes the barrier several
+      // times slower (measured: 61k verify 122 -> 67 us per call).
       __syncwarp();
-      if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL));
-     } else {
-      named_bar_sync(1, kSoftmaxThreads);  // alpha of the last tile visible to all
-     }
-      if (t > 0) {  // O^T of tile u = t-1: acc = acc * alpha_u + O_u
-        const int u = t - 1, ob = u % 2;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL + ob), (u / 2) & 1, abort));
-        float ov[NR];
+      named_bar_sync(bar_id, kSoftmaxThreads);
+      if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
+        const float* al = alpha_s + ((t - 2) % 4) * 32 + row0;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) ov[r] = 0.f;
-        if (ok) {
-          tc_fence_after();
-          tmem_ld16<0>(tmem + lane_off + 2 * NR + ob * NR, ov);
-          if constexpr (NR == 32) tmem_ld16<16 % NR>(tmem + lane_off + 2 * NR + ob * NR + 16, ov);
-          tmem_ld_wait();
-          tc_fence_before();
+        for (int r = 0; r < RW; ++r) acc[r] = fmaf(acc[r], al[r], oh[r] + ol[r]);
+      }
+      if (has_s) {
+        const int rl = lane % RW;
+        float tmax = red[(sb * 4 + 0) * 32 + rl];
+        tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
+        tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
+        tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
+        const float m_new = fmaxf(m_lane, tmax);
+        // alpha = 2^(cs (m_old - m_new)); bias makes p = 2^(cs s + bias) =
+        // 2^(cs (s - m_new) + kPShift).
+        const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
+        const float bias = (m_new == -INFINITY) ? 0.f : fmaf(-cs, m_new, (float)kPShift);
+        m_lane = m_new;
+        if (lane < RW) {
+          if (widx == 0) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
+          bc[lane] = bias;
+          bc[32 + lane] = alpha;
         }
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(bar(BAR_OEMPTY + ob));
-        if (ok) {
+        float bv[RW], av[RW];
 #pragma unroll
-          for (int r = 0; r < NR; ++r) acc[r] = fmaf(acc[r], alpha_s[ob * 32 + r], ov[r]);
+        for (int r = 0; r < RW; r += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
+          const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
+          bv[r] = a4.x; bv[r + 1] = a4.y; bv[r + 2] = a4.z; bv[r + 3] = a4.w;
+          av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
         }
+
+        // Scaled weights, split into an fp16 high part and an fp16 residual.
+        const uint32_t rm = rmask >> row0;
+        uint32_t phi[RW / 2], plo[RW / 2];
+#pragma unroll
+        for (int r = 0; r < RW; r += 2) {
+          float pr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            pr[e] = ((rm >> (r + e)) & 1u) ? fast_exp2(fmaf(sv[r + e], cs, bv[r + e])) : 0.f;
+            lpart[r + e] = fmaf(lpart[r + e], av[r + e], pr[e]);
+          }
+          const __half2 h = __floats2half2_rn(pr[0], pr[1]);
+          const float2 hf = __half22float2(h);
+          const __half2 l2 = __floats2half2_rn(pr[0] - hf.x, pr[1] - hf.y);
+          phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+          plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+
+        // A key no row can see must not reach the PV product: zero its V
+        // row (after its V tile has landed).
+        if (g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
+          ok = __all_sync(0xffffffffu,
+                          ok && mbar_wait(bar(BAR_VFULL + st), (t / kStages) & 1, abort));
+          if (ok && rmask == 0) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            const uint32_t vrow = sVr + st * kKVBytes + j * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              sts_v4(vrow + c * 16, z);
+              sts_v4(vrow + kHalfBytes + c * 16, z);
+            }
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_PEMPTY), (t & 1) ^ 1, abort));
+        if (ok) {
+          // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8][row'%8]
+          // with row' < NR the high parts and row' >= NR the residuals.
+          const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
+          constexpr uint32_t lo_off = (NR / 8) * 128;
+          if constexpr (RW >= 8) {
+#pragma unroll
+            for (int r8 = 0; r8 < RW / 8; ++r8) {
+              const uint32_t off = kb + ((row0 / 8) + r8) * 128;
+              sts_v4(sP + off, make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
+              sts_v4(sP + lo_off + off,
+                     make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
+            }
+          } else {  // four rows: half of one 16-byte core-matrix row
+            const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
+            sts_v2(sP + off, phi[0], phi[1]);
+            sts_v2(sP + lo_off + off, plo[0], plo[1]);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL));
       }
+      ph_cur = ph_nxt;
     }
 
     // Row sums: per-thread partials -> per-warp (lane r) -> across warps.
-    const float wl = warp_row_reduce<NR, false>(lpart, lane);
-    if (lane < NR) lsum[widx * 32 + lane] = wl;
-    named_bar_sync(1, kSoftmaxThreads);
+    const float wl = warp_row_reduce<RW, false>(lpart, lane);
+    if (lane < RW) lsum[widx * 32 + lane] = wl;
+    __syncwarp();
+    named_bar_sync(bar_id, kSoftmaxThreads);
     const bool aborted = *abort != 0;
 #pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      if (r < R) {
+    for (int r = 0; r < RW; ++r) {
+      if (row0 + r < R) {
         const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
-        const long long pr = part_base + row_index(r);
+        const long long pr = part_base + row_index(row0 + r);
         p.part_out[pr * kHeadDim + j] = (!aborted && l > 0.f) ? acc[r] / l : 0.f;
       }
     }
-    if (widx == 0 && lane < R) {
+    if (widx == 0 && lane < RW && row0 + lane < R) {
+      // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
       const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
-      p.part_lse[part_base + row_index(lane)] =
-          (!aborted && l > 0.f) ? ((m_lane - (float)kPShift) + log2f(l)) * 0.69314718055994531f
-                                : -INFINITY;
+      p.part_lse[part_base + row_index(row0 + lane)] =
+          (!aborted && l > 0.f)
+              ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
+              : -INFINITY;
     }
     __syncthreads();  // (A)
   }
@@ -523,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, Lay::kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -556,29 +641,29 @@ bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NR>
-cudaError_t launch_nr(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+template <int RW>
+cudaError_t launch_rw(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                       cudaStream_t stream) {
-  const size_t smem = Layout<NR>::kTotal + 1024;
+  const size_t smem = Cfg<RW>::kTotal + 1024;
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !configured[dev]) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_tc_kernel<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
   const dim3 grid(p.num_splits, p.num_kv_heads, p.num_seqs);
-  decode_tc_kernel<NR><<<grid, kThreads, smem, stream>>>(mk, mv, p);
+  decode_tc_kernel<RW><<<grid, kThreads, smem, stream>>>(mk, mv, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool decode_tc_supported(int kv_dtype, int rows, int num_blocks, int num_kv_heads, int block_size) {
-  return kv_dtype == kKvFp16 && rows >= 1 && rows <= 32 &&
+  return kv_dtype == kKvFp16 && rows >= 1 && rows <= 2 * 16 &&
          (long long)num_blocks * num_kv_heads * block_size <= INT32_MAX;
 }
 
@@ -587,8 +672,9 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream) {
   const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
   if (!encode_cache_map(&mk, p.k, rows) || !encode_cache_map(&mv, p.v, rows))
     return cudaErrorInvalidValue;
-  if (p.rows <= 16) return launch_nr<16>(p, mk, mv, stream);
-  return launch_nr<32>(p, mk, mv, stream);
+  if (p.rows <= 8) return launch_rw<4>(p, mk, mv, stream);
+  if (p.rows <= 16) return launch_rw<8>(p, mk, mv, stream);
+  return launch_rw<16>(p, mk, mv, stream);
 }
 
 }  // namespace pa
