@@ -179,6 +179,12 @@ int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_
                               int32_t causal, int32_t window, float scale,
                               int32_t kv_dtype, void* out, void* stream);
 
+/* Kernel launches one paged_attn_decode call makes for these shapes and
+ * cache type on the current device: the split-KV kernel and the merge kernel
+ * (launched as a programmatic dependent so that it starts as soon as the
+ * split-KV kernel ends).  Host only; negative pa_status on error. */
+int32_t paged_attn_launches_per_call(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
+
 /* Static string for a pa_status. */
 const char* paged_attn_status_string(int32_t status);
 

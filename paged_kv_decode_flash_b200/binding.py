@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.paged_attn_trace.restype = ctypes.c_int
             L.paged_attn_num_splits.argtypes = [P, i32, i32]
             L.paged_attn_num_splits.restype = ctypes.c_int32
+            L.paged_attn_launches_per_call.argtypes = [P, i32, i32]
+            L.paged_attn_launches_per_call.restype = ctypes.c_int32
             L.paged_attn_status_string.argtypes = [i32]
             L.paged_attn_status_string.restype = ctypes.c_char_p
             _LIB = L
@@ -156,6 +158,12 @@ class PagedDecode:
         n = lib().paged_attn_num_splits(ctypes.byref(self.dims), self.n_query, int(kv_dtype))
         if n < 0:
             raise PagedAttnError(n, "num_splits")
+        return n
+
+    def launches_per_call(self, kv_dtype: int = KV_FP16) -> int:
+        n = lib().paged_attn_launches_per_call(ctypes.byref(self.dims), self.n_query, int(kv_dtype))
+        if n < 0:
+            raise PagedAttnError(n, "launches_per_call")
         return n
 
     def __call__(self, q, k_cache, v_cache, block_table, context_lens, *, causal: int,

@@ -18,6 +18,7 @@
 // anything, and the regression test fills them with NaN).
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace pa {
 namespace {
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeParam
       p.part_out[pr * kHeadDim + tid] = 0.f;
       if (tid == 0) p.part_lse[pr] = -INFINITY;
     }
+    sm100::griddep_launch_dependents();  // partial written: the merge may be scheduled
   };
 
   const int L = p.context_lens[s];
@@ -245,6 +247,7 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(const DecodeParam
       if (tid == 0) p.part_lse[pr] = l > 0.f ? (m_s[r] + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
+  sm100::griddep_launch_dependents();  // partial written: the merge may be scheduled
 }
 
 }  // namespace

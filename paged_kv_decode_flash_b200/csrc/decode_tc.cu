@@ -55,14 +55,24 @@ using namespace sm100;
 constexpr int kTileKeys = 128;                 // keys per pipeline tile (M of S^T)
 constexpr int kChunksPerTile = kTileKeys / kChunk;
 constexpr int kStages = 3;                     // slots per K ring and per V ring
-constexpr uint32_t kHalfBytes = kTileKeys * 128;   // 64 fp16 columns of 128 keys
-constexpr uint32_t kKVBytes = 2 * kHalfBytes;      // one K (or V) tile
-constexpr uint32_t kChunkBytes = kChunk * 128;     // one 16-key half-chunk (TMA box)
+// A K or V tile of 128 keys in shared memory: [key group of 8][half][8 keys]
+// [64 fp16] with the 128-byte swizzle, i.e. 1 KB swizzle atoms; the atoms of
+// one 64-column half sit 2 KB apart, the two halves of a key group 1 KB apart.
+// One 16-key chunk (a contiguous 4 KB (block, head) tile in the cache for
+// block_size 16) is a single TMA box.
+constexpr uint32_t kAtomBytes = 1024;              // 8 keys x 128 bytes
+constexpr uint32_t kGroupBytes = 2 * kAtomBytes;   // both halves of 8 keys
+constexpr uint32_t kKVBytes = kTileKeys / 8 * kGroupBytes;  // one K (or V) tile
+constexpr uint32_t kChunkBytes = kChunk * 256;     // one 16-key chunk (TMA box)
 constexpr int kGroups = 2;                     // softmax warpgroups (split the rows)
 constexpr int kSoftmaxThreads = 128;           // per warpgroup
 constexpr int kVWarp = 2 + kGroups * 4;        // the V producer's warp
 constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr int kPShift = 14;                    // weights scaled by 2^14 before fp16
+// A row's reference max is only raised when a score passes it by more than
+// kLazy (log2 units); scaled weights then stay below 2^(kPShift + kLazy),
+// inside fp16 range.
+constexpr float kLazy = 1.5f;
 
 enum : int {
   BAR_KFULL = 0,    // [3] K tile landed
@@ -190,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.part_out[(part_base + row_index(r)) * kHeadDim + t % kHeadDim] = 0.f;
       if (t % kHeadDim == 0) p.part_lse[part_base + row_index(r)] = -INFINITY;
     }
+    griddep_launch_dependents();
     return;
   }
   const int base = (k0 / kChunk) * kChunk;
@@ -253,8 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 || warp == kVWarp) {
     // ======================= TMA producers (K: warp 0, V: last warp) =======
-    // Lane c < 8 owns chunk c of each tile; its block-table entry for the
-    // next tile is read one iteration early so the read overlaps the wait.
+    // Lane c < 8 owns chunk c of each tile and issues its copy; its
+    // block-table entry for the next tile is read one iteration early so the
+    // read overlaps the wait.  Lane 0 waits for the free slot and arms the
+    // slot's barrier before any lane issues.
     const bool is_k = warp == 0;
     const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
     const uint32_t ring = is_k ? sKr : sVr;
@@ -282,22 +295,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         want = false;
       }
       const uint32_t mask = __ballot_sync(0xffffffffu, want);
-      const int key0 = base + t * kTileKeys + c * kChunk;
-      const int row =
-          want ? (int)((ph_cur * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) : 0;
-      int rows[kChunksPerTile];
-#pragma unroll
-      for (int cc = 0; cc < kChunksPerTile; ++cc) rows[cc] = __shfl_sync(0xffffffffu, row, cc);
-      if (lane == 0) {  // the thread that saw the slot free issues its copies
-        const uint32_t fb = bar(bfull + st);
-        const uint32_t dst = ring + st * kKVBytes;
-        mbar_arrive_expect_tx(fb, __popc(mask) * 2 * kChunkBytes);
-#pragma unroll
-        for (int cc = 0; cc < kChunksPerTile; ++cc) {
-          if (!((mask >> cc) & 1u)) continue;
-          tma_load_2d(dst + cc * kChunkBytes, tmap, 0, rows[cc], fb);
-          tma_load_2d(dst + kHalfBytes + cc * kChunkBytes, tmap, 64, rows[cc], fb);
-        }
+      const uint32_t fb = bar(bfull + st);
+      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
+      __syncwarp();
+      // Each lane issues its own chunk's copy: one warp instruction moves the
+      // whole tile (a single issuing thread tops out near 17 GB/s per SM).
+      if (want) {
+        const int key0 = base + t * kTileKeys + c * kChunk;
+        const int row = (int)((ph_cur * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size);
+        tma_load_4d(ring + st * kKVBytes + c * kChunkBytes, tmap, 0, 0, 0, row / 8, fb);
       }
       __syncwarp();
       issued = t + 1;
@@ -317,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
       // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
       // start-address field is the low 14 bits, addresses stay < 256 KB).
-      const uint64_t dK = smem_desc(sKr, 16, 1024, kSwizzle128B);
+      const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
       const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
-      const uint64_t dV = smem_desc(sVr, kHalfBytes, 1024, kSwizzle128B);
+      const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
       const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
       int nqk = 0;  // QK^T products issued (tiles whose K was consumed)
       // Issue QK^T of tile nqk if its K tile and S buffer are ready (or wait
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + (nqk % 2) * NR;
 #pragma unroll
         for (int k = 0; k < kHeadDim / 16; ++k) {
-          const uint64_t ko = ((k / 4) * kHalfBytes + (k % 4) * 32) >> 4;
+          const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
           const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
           tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
         }
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
 #pragma unroll
         for (int k = 0; k < kTileKeys / 16; ++k) {
-          const uint64_t vo = (k * 2048) >> 4;
+          const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
           const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
           tc_mma_f16_ss(d, dV + so + vo, dP + po, id_pv, k > 0);
         }
@@ -418,10 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
     const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
 
-    float acc[RW], lpart[RW];
+    float acc[RW], lpart[RW], bias[RW];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) acc[r] = lpart[r] = 0.f;
-    float m_lane = -INFINITY;  // running raw-score max of row row0 + lane % RW
+    for (int r = 0; r < RW; ++r) {
+      acc[r] = lpart[r] = 0.f;
+      bias[r] = INFINITY;  // no reference yet: the row's first key forces one
+    }
+    // Reference max (raw score) of row row0 + lane % RW; -inf until the row
+    // sees a key.  bias[r] = kPShift - cs * (row r's reference max).
+    float m_lane = -INFINITY;
     bool ok = true;
     // Block-table entry of this thread's key, one tile ahead.
     auto phys_of = [&](int t) -> long long {
@@ -462,6 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       uint32_t rmask = 0;
+      bool all_vis = false;  // every key of this warp is seen by every row
+      float x[RW];           // cs * s + bias: log2 of the scaled weight
+      bool exceed = false;
       if (has_s) {
         // Which rows see this key?  Keys of out-of-range blocks see none.
         const int key = base + t * kTileKeys + j;
@@ -474,60 +488,83 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
           }
         }
+        all_vis = __all_sync(0xffffffffu, rmask == all_rows);
         const uint32_t rm = rmask >> row0;
-        float tmp[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
-        const float wmax = warp_row_reduce<RW, true>(tmp, lane);
-        if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
+        for (int r = 0; r < RW; ++r) {
+          x[r] = fmaf(sv[r], cs, bias[r]);
+          const bool vis = all_vis || ((rm >> r) & 1u);
+          exceed |= vis && x[r] > (float)kPShift + kLazy;
+        }
       }
       // Reconverge before the group barrier: a warp that arrives diverged
-      // (after the lane-predicated store above) makes the barrier several
-      // times slower (measured: 61k verify 122 -> 67 us per call).
+      // (after lane-predicated code) makes the barrier several times slower
+      // (measured: 61k verify 122 -> 67 us per call).
       __syncwarp();
-      named_bar_sync(bar_id, kSoftmaxThreads);
+      // One barrier per tile: orders the shared-memory traffic of the group
+      // and tells every thread whether any score passed its row's reference.
+      const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
       if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
         const float* al = alpha_s + ((t - 2) % 4) * 32 + row0;
 #pragma unroll
         for (int r = 0; r < RW; ++r) acc[r] = fmaf(acc[r], al[r], oh[r] + ol[r]);
       }
       if (has_s) {
-        const int rl = lane % RW;
-        float tmax = red[(sb * 4 + 0) * 32 + rl];
-        tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
-        tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
-        tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
-        const float m_new = fmaxf(m_lane, tmax);
-        // alpha = 2^(cs (m_old - m_new)); bias makes p = 2^(cs s + bias) =
-        // 2^(cs (s - m_new) + kPShift).
-        const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
-        const float bias = (m_new == -INFINITY) ? 0.f : fmaf(-cs, m_new, (float)kPShift);
-        m_lane = m_new;
-        if (lane < RW) {
-          if (widx == 0) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
-          bc[lane] = bias;
-          bc[32 + lane] = alpha;
-        }
-        __syncwarp();
-        float bv[RW], av[RW];
+        const uint32_t rm = rmask >> row0;
+        float alpha = 1.f;
+        if (rescale) {
+          // New reference max per row: warp transpose-reduction, then across
+          // the group's four warps.
+          float tmp[RW];
 #pragma unroll
-        for (int r = 0; r < RW; r += 4) {
-          const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
-          const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
-          bv[r] = a4.x; bv[r + 1] = a4.y; bv[r + 2] = a4.z; bv[r + 3] = a4.w;
-          av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
+          for (int r = 0; r < RW; ++r) tmp[r] = (all_vis || ((rm >> r) & 1u)) ? sv[r] : -INFINITY;
+          const float wmax = warp_row_reduce<RW, true>(tmp, lane);
+          if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
+          __syncwarp();
+          named_bar_sync(bar_id, kSoftmaxThreads);
+          const int rl = lane % RW;
+          float tmax = red[(sb * 4 + 0) * 32 + rl];
+          tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
+          tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
+          tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
+          const float m_new = fmaxf(m_lane, tmax);
+          // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
+          // 2^(cs (s - m_new) + kPShift).
+          alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
+          const float bias_l =
+              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
+          m_lane = m_new;
+          if (lane < RW) {
+            bc[lane] = bias_l;
+            bc[32 + lane] = alpha;
+          }
+          __syncwarp();
+          float av[RW];
+#pragma unroll
+          for (int r = 0; r < RW; r += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
+            const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
+            bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
+            av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            x[r] = fmaf(sv[r], cs, bias[r]);
+            lpart[r] *= av[r];
+          }
         }
+        if (widx == 0 && lane < RW) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
 
         // Scaled weights, split into an fp16 high part and an fp16 residual.
-        const uint32_t rm = rmask >> row0;
         uint32_t phi[RW / 2], plo[RW / 2];
 #pragma unroll
         for (int r = 0; r < RW; r += 2) {
           float pr[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            pr[e] = ((rm >> (r + e)) & 1u) ? fast_exp2(fmaf(sv[r + e], cs, bv[r + e])) : 0.f;
-            lpart[r + e] = fmaf(lpart[r + e], av[r + e], pr[e]);
+            const bool vis = all_vis || ((rm >> (r + e)) & 1u);
+            pr[e] = vis ? fast_exp2(x[r + e]) : 0.f;
+            lpart[r + e] += pr[e];
           }
           const __half2 h = __floats2half2_rn(pr[0], pr[1]);
           const float2 hf = __half22float2(h);
@@ -543,11 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                           ok && mbar_wait(bar(BAR_VFULL + st), (t / kStages) & 1, abort));
           if (ok && rmask == 0) {
             const uint4 z = make_uint4(0, 0, 0, 0);
-            const uint32_t vrow = sVr + st * kKVBytes + j * 128;
+            const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               sts_v4(vrow + c * 16, z);
-              sts_v4(vrow + kHalfBytes + c * 16, z);
+              sts_v4(vrow + kAtomBytes + c * 16, z);
             }
           }
         }
@@ -603,6 +640,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();  // (A)
   }
 
+  // This CTA's partial is written: the merge kernel that follows on the
+  // stream may be scheduled (it waits for the whole grid before reading).
+  // Triggering any earlier lets idle merge CTAs share the SMs with the
+  // decode and slows it (measured: 61k verify 64 -> 70 us per call).
+  griddep_launch_dependents();
   // ---- tear-down (every thread passed (A)) -----------------------------------
   if (threadIdx.x == 0 && misc->abort) atomicOr(p.flags, kFlagTimeout);
   tc_fence_after();
@@ -626,17 +668,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// The fp16 cache viewed as a 2-D tensor: 128 columns (head_dim) by
-// num_blocks * Hkv * block_size rows; one TMA box = 16 rows x 64 columns,
-// 128-byte swizzle (the layout the tcgen05 descriptors expect).
+// The fp16 cache viewed as a 4-D tensor {64 columns, 8 rows, 2 halves,
+// rows/8 groups} (row = one key of one KV head, 256 bytes): one box
+// {64, 8, 2, 2} is a 16-row chunk, stored in shared memory as
+// [group][half][8 rows][64 columns] with the 128-byte swizzle the tcgen05
+// descriptors expect.
 bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
   auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kChunk};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(cache), dims, strides, box,
+  if (fn == nullptr || rows % 8 != 0) return false;
+  cuuint64_t dims[4] = {64, 8, 2, (cuuint64_t)(rows / 8)};
+  cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, 128, 8 * (cuuint64_t)kHeadDim * 2};
+  cuuint32_t box[4] = {64, 8, 2, 2};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(cache), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -12,11 +12,15 @@
 // element; reads are coalesced along head_dim.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace pa {
 namespace {
 
 __global__ void merge_kernel(const MergeParams p) {
+  // Launched as a programmatic dependent of the decode kernel: wait for its
+  // partials (returns at once when launched normally).
+  sm100::griddep_wait();
   const long long row = blockIdx.x;               // over num_seqs * rows_per_seq
   const int s = (int)(row / p.rows_per_seq);
   const int r = (int)(row % p.rows_per_seq);
@@ -48,8 +52,19 @@ __global__ void merge_kernel(const MergeParams p) {
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
   const long long rows = (long long)p.num_seqs * p.rows_per_seq;
   if (rows == 0) return cudaSuccess;
-  merge_kernel<<<(unsigned)rows, p.head_dim, 0, stream>>>(p);
-  return cudaGetLastError();
+  // Programmatic stream serialization: the merge grid may be scheduled while
+  // the preceding decode kernel still runs and starts the moment it ends.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(p.head_dim);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, p);
 }
 
 }  // namespace pa
