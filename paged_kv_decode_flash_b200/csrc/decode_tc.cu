@@ -86,8 +86,10 @@ enum : int {
   BAR_OFULL = 18,   // [2] O^T of one tile in TMEM
   BAR_OEMPTY = 20,  // [2] O^T read by the softmax warps
   BAR_DONE = 22,    // every MMA finished
-  BAR_COUNT = 23
+  BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
+  BAR_COUNT = 31
 };
+constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
 // RW query rows per softmax warpgroup; NR = the MMA's N for S (>= 16).
 template <int RW>
@@ -106,7 +108,8 @@ struct Cfg {
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
   static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [8 warps][2][32]
   static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [32]
-  static constexpr uint32_t kMisc = kBars + 32 * 8;                 // small ints
+  static constexpr uint32_t kInfo = kBars + 32 * 8;                 // TileInfo [8]
+  static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
   static constexpr uint32_t kTotal = kMisc + 64;
   // TMEM columns: S^T[2] (NR each) then O^T[2] (2*NR each: high | residual).
   static constexpr uint32_t kTmemUsed = 6 * NR;
@@ -119,6 +122,17 @@ struct Misc {
   int abort;
   int k_consumed, v_consumed;
 };
+
+// What the K producer publishes for each local tile of a CTA: the tile's
+// number in the head's key space (-1: no more tiles), which of its 16-key
+// chunks were loaded, and each loaded chunk's TMA row coordinate (row / 8).
+struct TileInfo {
+  int tile;
+  uint32_t mask;
+  int row8[kChunksPerTile];
+  int pad[2];
+};
+static_assert(sizeof(TileInfo) == 48, "TileInfo layout");
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 r;
@@ -171,30 +185,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   Misc* misc = reinterpret_cast<Misc*>(smem + C::kMisc);
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + C::kInfo);
   volatile int* abort = &misc->abort;
   auto bar = [&](int i) { return sbase + C::kBars + 8u * i; };
 
   const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int S = p.num_splits;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nq = p.n_query, G = p.group, Hq = p.num_q_heads, R = p.rows;
   const int rps = nq * Hq;
-  const long long part_base = ((long long)s * p.num_splits + split) * rps;
+  const long long part_base = ((long long)s * S + split) * rps;
   auto row_index = [&](int r) { return (r / G) * Hq + kvh * G + (r % G); };
 
-  // ---- the CTA's key range (uniform across the CTA) -----------------------
+  // ---- the head's visible keys and its tiles (uniform across the CTA) ------
+  // The keys of (sequence s, KV head kvh) that any query token sees form
+  // [lo_u, hi_u]; they are cut into 128-key tiles from `base`, and the S
+  // splits take contiguous runs of them, as even as whole tiles allow.  The
+  // partition depends only on the context length and S, so every call on the
+  // same inputs adds the same tiles in the same order: results are
+  // bit-reproducible.
   const int L = p.context_lens[s];
-  int k0 = 0, k1 = -1;
+  int lo_u = 0, hi_u = -1;
   if (context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size)) {
-    int lo_u, hi_u;
     union_range(L, nq, p.causal, p.window, lo_u, hi_u);
-    const long long sk0 = (long long)split * p.blocks_per_split * p.block_size;
-    const long long sk1 = sk0 + (long long)p.blocks_per_split * p.block_size - 1;
-    k0 = (int)max((long long)lo_u, sk0);
-    k1 = (int)min((long long)hi_u, sk1);
   } else if (split == 0 && kvh == 0 && threadIdx.x == 0) {
     atomicOr(p.flags, kFlagBadLen);
   }
-  if (k0 > k1) {  // nothing visible here: an empty partial
+  const int base = (lo_u / kChunk) * kChunk;
+  const int ntiles_h = hi_u >= lo_u ? (hi_u + 1 - base + kTileKeys - 1) / kTileKeys : 0;
+  const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
+  const int t_first = split * t_per + min(split, t_rem);
+  const int t_count = t_per + (split < t_rem ? 1 : 0);
+  if (t_count == 0) {  // every tile is another CTA's: an empty partial
     for (int t = threadIdx.x; t < R * kHeadDim; t += kThreads) {
       const int r = t / kHeadDim;
       p.part_out[(part_base + row_index(r)) * kHeadDim + t % kHeadDim] = 0.f;
@@ -203,455 +225,518 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_launch_dependents();
     return;
   }
-  const int base = (k0 / kChunk) * kChunk;
-  const int ntiles = (k1 + 1 - base + kTileKeys - 1) / kTileKeys;
   const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
 
   const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
   const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
 
-  // ---- set-up ---------------------------------------------------------------
-  if (warp == 1) {
-    tmem_alloc(sbase + C::kMisc + offsetof(Misc, tmem_base), C::kTmemCols);
-    tmem_relinquish();
-  }
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar(BAR_KFULL + i), 1);
-      mbar_init(bar(BAR_KEMPTY + i), 1);
-      mbar_init(bar(BAR_VFULL + i), 1);
-      mbar_init(bar(BAR_VEMPTY + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(BAR_SFULL + i), 1);
-      mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
-      mbar_init(bar(BAR_OFULL + i), 1);
-      mbar_init(bar(BAR_OEMPTY + i), 4 * kGroups);
-    }
-    mbar_init(bar(BAR_PFULL), 4 * kGroups);
-    mbar_init(bar(BAR_PEMPTY), 1);
-    mbar_init(bar(BAR_DONE), 1);
-    misc->abort = 0;
-    misc->k_consumed = misc->v_consumed = 0;
-    fence_mbar_init();
-  }
-  if (warp >= 2 && warp < kVWarp) {
-    // Q rows of this KV head -> shared memory, K-major with 128-byte swizzle:
-    // row n, 16-byte chunk c of half h at h*NR*128 + n*128 + ((c ^ n%8) * 16).
-    // Rows >= R are zero; so are P's padding rows (never written later).  A
-    // negative scale is moved into Q (an exact sign flip) so that the kernel
-    // only ever multiplies scores by a non-negative factor.
-    const int t = threadIdx.x - 64;
-    const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-    for (int c = t; c < NR * 16; c += kGroups * kSoftmaxThreads) {
-      const int n = c / 16, cc = c % 16, h = cc / 8, k8 = cc % 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n < R) {
-        const long long qrow = ((long long)s * nq + n / G) * Hq + kvh * G + (n % G);
-        v = ldg_nc_v4(p.q + qrow * kHeadDim + cc * 8);
-        v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
+  if (warp == 0) {
+    // ======================= K producer (also sets up the barriers) ========
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(bar(BAR_KFULL + i), 1);
+        mbar_init(bar(BAR_KEMPTY + i), 1);
+        mbar_init(bar(BAR_VFULL + i), 1);
+        mbar_init(bar(BAR_VEMPTY + i), 1);
       }
-      sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(bar(BAR_SFULL + i), 1);
+        mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
+        mbar_init(bar(BAR_OFULL + i), 1);
+        mbar_init(bar(BAR_OEMPTY + i), 4 * kGroups);
+      }
+      mbar_init(bar(BAR_PFULL), 4 * kGroups);
+      mbar_init(bar(BAR_PEMPTY), 1);
+      mbar_init(bar(BAR_DONE), 1);
+      for (int i = 0; i < kInfoSlots; ++i) mbar_init(bar(BAR_INFO + i), 1);
+      misc->abort = 0;
+      misc->k_consumed = misc->v_consumed = 0;
+      fence_mbar_init();
     }
-    for (uint32_t off = t * 16; off < C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
-      sts_v4(sP + off, make_uint4(0, 0, 0, 0));
-    fence_proxy_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = misc->tmem_base;
+    __syncwarp();
+    // The other roles wait for these barriers; this warp starts loading now.
+    named_bar_arrive(3, kThreads);
 
-  if (warp == 0 || warp == kVWarp) {
-    // ======================= TMA producers (K: warp 0, V: last warp) =======
-    // Lane c < 8 owns chunk c of each tile and issues its copy; its
-    // block-table entry for the next tile is read one iteration early so the
-    // read overlaps the wait.  Lane 0 waits for the free slot and arms the
-    // slot's barrier before any lane issues.
-    const bool is_k = warp == 0;
-    const CUtensorMap* tmap = is_k ? &tmap_k : &tmap_v;
-    const uint32_t ring = is_k ? sKr : sVr;
-    const int bfull = is_k ? BAR_KFULL : BAR_VFULL, bempty = is_k ? BAR_KEMPTY : BAR_VEMPTY;
+    // Lane c < 8 owns chunk c of every tile and reads its block-table entry
+    // one tile ahead.
     const int c = lane;
-    auto lookup = [&](int t, long long& phys) {
-      const int key0 = base + t * kTileKeys + c * kChunk;
-      const bool want = t < ntiles && c < kChunksPerTile && key0 <= k1 && key0 + kChunk - 1 >= k0;
-      phys = want ? (long long)table[key0 / p.block_size] : 0;
-      return want;
+    auto lookup = [&](int g, int& row8) -> bool {
+      if (g < 0 || c >= kChunksPerTile) return false;
+      const int key0 = base + g * kTileKeys + c * kChunk;
+      if (key0 > hi_u || key0 + kChunk - 1 < lo_u) return false;
+      const long long phys = table[key0 / p.block_size];
+      if (phys < 0 || phys >= p.num_blocks) {
+        atomicOr(p.flags, kFlagBadBlock);  // masked, never dereferenced
+        return false;
+      }
+      row8 = (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
+      return true;
     };
-    long long ph_cur = 0, ph_nxt = 0;
-    bool w_cur = lookup(0, ph_cur);
+    auto tile_of = [&](int t) { return t < t_count ? t_first + t : -1; };
+    int g_cur = tile_of(0);
+    int row_cur = 0, row_nxt = 0;
+    bool w_cur = lookup(g_cur, row_cur);
     int issued = 0;
-    for (int t = 0; t < ntiles; ++t) {
-      const bool w_nxt = lookup(t + 1, ph_nxt);
+    for (int t = 0;; ++t) {
+      // Publish tile t for the V producer, the MMA issuer and the softmax.
+      const uint32_t mask = __ballot_sync(0xffffffffu, w_cur);
+      TileInfo& ti = info[t % kInfoSlots];
+      if (lane < kChunksPerTile) ti.row8[lane] = row_cur;
+      if (lane == 0) {
+        ti.tile = g_cur;
+        ti.mask = mask;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_INFO + t % kInfoSlots));
+      if (g_cur < 0) break;
+      // Tile t + 1's block-table entries, read while tile t's slot frees up.
+      const int g_nxt = tile_of(t + 1);
+      const bool w_nxt = lookup(g_nxt, row_nxt);
+      // Wait for the slot, then every lane issues its chunk's copy.
       const int st = t % kStages;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar(bempty + st), ((t / kStages) & 1) ^ 1, abort);
+      if (lane == 0) ok = mbar_wait(bar(BAR_KEMPTY + st), ((t / kStages) & 1) ^ 1, abort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      bool want = w_cur;
-      if (want && (ph_cur < 0 || ph_cur >= p.num_blocks)) {
-        if (is_k) atomicOr(p.flags, kFlagBadBlock);  // masked, never dereferenced
-        want = false;
-      }
-      const uint32_t mask = __ballot_sync(0xffffffffu, want);
-      const uint32_t fb = bar(bfull + st);
+      const uint32_t fb = bar(BAR_KFULL + st);
       if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
       __syncwarp();
-      // Each lane issues its own chunk's copy: one warp instruction moves the
-      // whole tile (a single issuing thread tops out near 17 GB/s per SM).
-      if (want) {
-        const int key0 = base + t * kTileKeys + c * kChunk;
-        const int row = (int)((ph_cur * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size);
-        tma_load_4d(ring + st * kKVBytes + c * kChunkBytes, tmap, 0, 0, 0, row / 8, fb);
-      }
+      if (w_cur) tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
       __syncwarp();
       issued = t + 1;
-      ph_cur = ph_nxt;
+      g_cur = g_nxt;
       w_cur = w_nxt;
+      row_cur = row_nxt;
     }
     __syncthreads();  // (A) every role finished its loop
     if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
       volatile int no_abort = 0;
-      for (int t = is_k ? misc->k_consumed : misc->v_consumed; t < issued; ++t)
-        mbar_wait(bar(bfull + t % kStages), (t / kStages) & 1, &no_abort);
+      for (int t = misc->k_consumed; t < issued; ++t)
+        mbar_wait(bar(BAR_KFULL + t % kStages), (t / kStages) & 1, &no_abort);
     }
-  } else if (warp == 1) {
-    // ======================= MMA issuer ====================================
-    if (lane == 0) {
-      const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
-      const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
-      // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
-      // start-address field is the low 14 bits, addresses stay < 256 KB).
-      const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
-      const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
-      const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
-      const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
-      int nqk = 0;  // QK^T products issued (tiles whose K was consumed)
-      // Issue QK^T of tile nqk if its K tile and S buffer are ready (or wait
-      // for them when `block`).  1 = issued, 0 = not ready, -1 = gave up.
-      auto try_qk = [&](bool block) -> int {
-        if (nqk >= ntiles) return 0;
-        const uint32_t f = bar(BAR_KFULL + nqk % kStages), e = bar(BAR_SEMPTY + nqk % 2);
-        const uint32_t pf = (nqk / kStages) & 1, pe = ((nqk / 2) & 1) ^ 1;
-        if (block) {
-          if (!(mbar_wait(f, pf, abort) && mbar_wait(e, pe, abort))) return -1;
-        } else if (!(mbar_test_wait(f, pf) && mbar_test_wait(e, pe))) {
-          return 0;
-        }
-        tc_fence_after();
-        const uint64_t so = (uint64_t)((nqk % kStages) * kKVBytes) >> 4;
-        const uint32_t d = tmem + (nqk % 2) * NR;
-#pragma unroll
-        for (int k = 0; k < kHeadDim / 16; ++k) {
-          const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
-          const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
-          tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
-        }
-        tc_commit(bar(BAR_SFULL + nqk % 2));
-        tc_commit(bar(BAR_KEMPTY + nqk % kStages));
-        ++nqk;
-        return 1;
-      };
-      int npv = 0;
-      bool ok = true;
-      for (int t = 0; ok && t < ntiles; ++t) {
-        if (nqk <= t && try_qk(true) < 0) { ok = false; break; }  // QK(t) comes first
-        if (nqk == t + 1) try_qk(false);
-        // Wait for P(t), issuing QK(t+1) as soon as its K tile lands.
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait_ns(bar(BAR_PFULL), t & 1, 200)) {
-          if (nqk == t + 1) try_qk(false);
-          if (*abort || globaltimer() - t0 > kWaitLimitNs) { *abort = 1; ok = false; break; }
-        }
-        if (!ok) break;
-        ok = mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, abort) &&
-             mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t so = (uint64_t)((t % kStages) * kKVBytes) >> 4;
-        const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
-#pragma unroll
-        for (int k = 0; k < kTileKeys / 16; ++k) {
-          const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
-          const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
-          tc_mma_f16_ss(d, dV + so + vo, dP + po, id_pv, k > 0);
-        }
-        tc_commit(bar(BAR_OFULL + t % 2));
-        tc_commit(bar(BAR_PEMPTY));
-        tc_commit(bar(BAR_VEMPTY + t % kStages));
-        npv = t + 1;
-        if (nqk == t + 1) try_qk(false);
-      }
-      misc->k_consumed = nqk;
-      misc->v_consumed = npv;
-      tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
-      volatile int no_abort = 0;
-      mbar_wait(bar(BAR_DONE), 0, &no_abort);
-    }
-    __syncwarp();
-    __syncthreads();  // (A)
   } else {
-    // ======================= softmax + correction ==========================
-    // Warpgroup g handles rows [g*RW, g*RW + RW); its warps cover the four
-    // TMEM lane quarters, i.e. keys (for S) and head_dim elements (for O).
-    const int g = (warp - 2) / 4, widx = (warp - 2) % 4;
-    const int row0 = g * RW;
-    const int q4 = warp & 3;
-    const int j = q4 * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
-    float* alpha_s = reinterpret_cast<float*>(smem + C::kAlpha);             // [4][32]
-    float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
-    float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
-    const uint32_t bar_id = 1 + g;
-    const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
-
-    // Per query token, the visible key range; keys inside every token's
-    // range (and the CTA's) see all rows: the fast path of interior tiles.
-    int tlo[kMaxQuery], thi[kMaxQuery];
-    int lo_all = k0, hi_all = k1;
-#pragma unroll
-    for (int i = 0; i < kMaxQuery; ++i) {
-      tlo[i] = 1;
-      thi[i] = 0;
-      if (i < nq) {
-        key_range(L, nq, i, p.causal, p.window, tlo[i], thi[i]);
-        lo_all = max(lo_all, tlo[i]);
-        hi_all = min(hi_all, thi[i]);
-      }
+    // ---- set-up of the other roles ----------------------------------------
+    if (warp == 1) {
+      tmem_alloc(sbase + C::kMisc + offsetof(Misc, tmem_base), C::kTmemCols);
+      tmem_relinquish();
     }
-    const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
-    const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
-
-    float acc[RW], lpart[RW], bias[RW];
-#pragma unroll
-    for (int r = 0; r < RW; ++r) {
-      acc[r] = lpart[r] = 0.f;
-      bias[r] = INFINITY;  // no reference yet: the row's first key forces one
-    }
-    // Reference max (raw score) of row row0 + lane % RW; -inf until the row
-    // sees a key.  bias[r] = kPShift - cs * (row r's reference max).
-    float m_lane = -INFINITY;
-    bool ok = true;
-    // Block-table entry of this thread's key, one tile ahead.
-    auto phys_of = [&](int t) -> long long {
-      const int key = base + t * kTileKeys + j;
-      return (t < ntiles && key >= k0 && key <= k1) ? (long long)table[key / p.block_size] : -1;
-    };
-    long long ph_cur = phys_of(0);
-
-    // Iteration t scores tile t and folds tile t-2's O^T (finished long ago)
-    // into the register accumulators; the two extra iterations only fold.
-    // Tile u's rescale factors live in alpha_s[u % 4].
-    for (int t = 0; t < ntiles + 2; ++t) {
-      const bool has_s = t < ntiles, has_o = t >= 2;
-      const int sb = t % 2, st = t % kStages, ob = t % 2;  // O of tile t-2 sits in buffer t%2
-      const long long ph_nxt = phys_of(t + 1);
-      if (has_o)
-        ok = __all_sync(0xffffffffu,
-                        ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
-      if (has_s)
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
-      float sv[RW], oh[RW], ol[RW];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) sv[r] = oh[r] = ol[r] = 0.f;
-      if (ok) {
-        tc_fence_after();
-        if (has_o) {
-          tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + row0, oh);
-          tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + NR + row0, ol);
+    if (warp >= 2 && warp < kVWarp) {
+      // Q rows of this KV head -> shared memory, K-major with 128-byte
+      // swizzle: row n, 16-byte chunk c of half h at h*NR*128 + n*128 +
+      // ((c ^ n%8) * 16).  Rows >= R are zero; so are P's padding rows (never
+      // written later).  A negative scale is moved into Q (an exact sign
+      // flip) so that the kernel only multiplies scores by a factor >= 0.
+      const int t = threadIdx.x - 64;
+      const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+      for (int c = t; c < NR * 16; c += kGroups * kSoftmaxThreads) {
+        const int n = c / 16, cc = c % 16, h = cc / 8, k8 = cc % 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < R) {
+          const long long qrow = ((long long)s * nq + n / G) * Hq + kvh * G + (n % G);
+          v = ldg_nc_v4(p.q + qrow * kHeadDim + cc * 8);
+          v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
         }
-        if (has_s) tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
-        tmem_ld_wait();
-        tc_fence_before();
+        sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
+      }
+      for (uint32_t off = t * 16; off < C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
+        sts_v4(sP + off, make_uint4(0, 0, 0, 0));
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    named_bar_sync(3, kThreads);  // barriers initialised, TMEM allocated, Q staged
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+
+    if (warp == kVWarp) {
+      // ===================== V producer ======================================
+      // Follows the K producer's published tiles; lane c < 8 issues chunk c.
+      const int c = lane;
+      int issued = 0;
+      for (int t = 0;; ++t) {
+        int ok = 1;
+        if (lane == 0)
+          ok = mbar_wait(bar(BAR_INFO + t % kInfoSlots), (t / kInfoSlots) & 1, abort);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();  // lane 0's acquire orders the other lanes' reads below
+        if (!ok) break;
+        const TileInfo& ti = info[t % kInfoSlots];
+        if (ti.tile < 0) break;
+        const uint32_t mask = ti.mask;
+        const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;
+        const int st = t % kStages;
+        if (lane == 0) ok = mbar_wait(bar(BAR_VEMPTY + st), ((t / kStages) & 1) ^ 1, abort);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const uint32_t fb = bar(BAR_VFULL + st);
+        if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
+        __syncwarp();
+        if (c < kChunksPerTile && ((mask >> c) & 1u))
+          tma_load_4d(sVr + st * kKVBytes + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
+        __syncwarp();
+        issued = t + 1;
+      }
+      __syncthreads();  // (A)
+      if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
+        volatile int no_abort = 0;
+        for (int t = misc->v_consumed; t < issued; ++t)
+          mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, &no_abort);
+      }
+    } else if (warp == 1) {
+      // ===================== MMA issuer ======================================
+      if (lane == 0) {
+        const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
+        const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
+        // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
+        // start-address field is the low 14 bits, addresses stay < 256 KB).
+        const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
+        const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
+        const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
+        const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
+        int nqk = 0;              // QK^T products issued
+        int end_t = 0x7fffffff;   // number of tiles, once the producer said so
+        // Issue QK^T of tile nqk if it exists and its K tile and S buffer are
+        // ready (or wait for them when `block`).  1 = issued, 0 = not ready or
+        // no such tile, -1 = gave up.
+        auto try_qk = [&](bool block) -> int {
+          if (nqk >= end_t) return 0;
+          const uint32_t ib = bar(BAR_INFO + nqk % kInfoSlots), ip = (nqk / kInfoSlots) & 1;
+          if (block) {
+            if (!mbar_wait(ib, ip, abort)) return -1;
+          } else if (!mbar_test_wait(ib, ip)) {
+            return 0;
+          }
+          if (info[nqk % kInfoSlots].tile < 0) {
+            end_t = nqk;
+            return 0;
+          }
+          const uint32_t f = bar(BAR_KFULL + nqk % kStages), e = bar(BAR_SEMPTY + nqk % 2);
+          const uint32_t pf = (nqk / kStages) & 1, pe = ((nqk / 2) & 1) ^ 1;
+          if (block) {
+            if (!(mbar_wait(f, pf, abort) && mbar_wait(e, pe, abort))) return -1;
+          } else if (!(mbar_test_wait(f, pf) && mbar_test_wait(e, pe))) {
+            return 0;
+          }
+          tc_fence_after();
+          const uint64_t so = (uint64_t)((nqk % kStages) * kKVBytes) >> 4;
+          const uint32_t d = tmem + (nqk % 2) * NR;
+#pragma unroll
+          for (int k = 0; k < kHeadDim / 16; ++k) {
+            const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
+            const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
+            tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
+          }
+          tc_commit(bar(BAR_SFULL + nqk % 2));
+          tc_commit(bar(BAR_KEMPTY + nqk % kStages));
+          ++nqk;
+          return 1;
+        };
+        int npv = 0;
+        bool ok = true;
+        for (int t = 0; ok; ++t) {
+          if (nqk <= t && try_qk(true) < 0) { ok = false; break; }  // QK(t) comes first
+          if (t >= end_t) break;                                     // no tile t
+          if (nqk == t + 1) try_qk(false);
+          // Wait for P(t), issuing QK(t+1) as soon as its K tile lands.
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_try_wait_ns(bar(BAR_PFULL), t & 1, 200)) {
+            if (nqk == t + 1) try_qk(false);
+            if (*abort || globaltimer() - t0 > kWaitLimitNs) { *abort = 1; ok = false; break; }
+          }
+          if (!ok) break;
+          ok = mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, abort) &&
+               mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)((t % kStages) * kKVBytes) >> 4;
+          const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
+#pragma unroll
+          for (int k = 0; k < kTileKeys / 16; ++k) {
+            const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
+            const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
+            tc_mma_f16_ss(d, dV + so + vo, dP + po, id_pv, k > 0);
+          }
+          tc_commit(bar(BAR_OFULL + t % 2));
+          tc_commit(bar(BAR_PEMPTY));
+          tc_commit(bar(BAR_VEMPTY + t % kStages));
+          npv = t + 1;
+          if (nqk == t + 1) try_qk(false);
+        }
+        misc->k_consumed = nqk;
+        misc->v_consumed = npv;
+        tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
+        volatile int no_abort = 0;
+        mbar_wait(bar(BAR_DONE), 0, &no_abort);
       }
       __syncwarp();
-      if (ok && lane == 0) {
-        if (has_o) mbar_arrive(bar(BAR_OEMPTY + ob));
-        if (has_s) mbar_arrive(bar(BAR_SEMPTY + sb));
-      }
+      __syncthreads();  // (A)
+    } else {
+      // ===================== softmax + correction ============================
+      // Warpgroup g handles rows [g*RW, g*RW + RW); its warps cover the four
+      // TMEM lane quarters, i.e. keys (for S) and head_dim elements (for O).
+      const int g = (warp - 2) / 4, widx = (warp - 2) % 4;
+      const int row0 = g * RW;
+      const int q4 = warp & 3;
+      const int j = q4 * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+      float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
+      float* alpha_s = reinterpret_cast<float*>(smem + C::kAlpha);             // [4][32]
+      float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
+      float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
+      const uint32_t bar_id = 1 + g;
+      const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
 
-      uint32_t rmask = 0;
-      bool all_vis = false;  // every key of this warp is seen by every row
-      float x[RW];           // cs * s + bias: log2 of the scaled weight
-      bool exceed = false;
-      if (has_s) {
-        // Which rows see this key?  Keys of out-of-range blocks see none.
-        const int key = base + t * kTileKeys + j;
-        if (ph_cur >= 0 && ph_cur < p.num_blocks) {
-          if (key >= lo_all && key <= hi_all) {
-            rmask = all_rows;
-          } else if (key >= k0 && key <= k1) {
+      // Per query token, the visible key range; keys inside every token's
+      // range see all rows: the fast path of interior tiles.
+      int tlo[kMaxQuery], thi[kMaxQuery];
+      int lo_all = lo_u, hi_all = hi_u;
 #pragma unroll
-            for (int i = 0; i < kMaxQuery; ++i)
-              if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
-          }
-        }
-        all_vis = __all_sync(0xffffffffu, rmask == all_rows);
-        const uint32_t rm = rmask >> row0;
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          x[r] = fmaf(sv[r], cs, bias[r]);
-          const bool vis = all_vis || ((rm >> r) & 1u);
-          exceed |= vis && x[r] > (float)kPShift + kLazy;
+      for (int i = 0; i < kMaxQuery; ++i) {
+        tlo[i] = 1;
+        thi[i] = 0;
+        if (i < nq) {
+          key_range(L, nq, i, p.causal, p.window, tlo[i], thi[i]);
+          lo_all = max(lo_all, tlo[i]);
+          hi_all = min(hi_all, thi[i]);
         }
       }
-      // Reconverge before the group barrier: a warp that arrives diverged
-      // (after lane-predicated code) makes the barrier several times slower
-      // (measured: 61k verify 122 -> 67 us per call).
-      __syncwarp();
-      // One barrier per tile: orders the shared-memory traffic of the group
-      // and tells every thread whether any score passed its row's reference.
-      const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
-      if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
-        const float* al = alpha_s + ((t - 2) % 4) * 32 + row0;
+      const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
+      const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
+
+      float acc[RW], lpart[RW], bias[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) acc[r] = fmaf(acc[r], al[r], oh[r] + ol[r]);
+      for (int r = 0; r < RW; ++r) {
+        acc[r] = lpart[r] = 0.f;
+        bias[r] = INFINITY;  // no reference yet: the row's first key forces one
       }
-      if (has_s) {
-        const uint32_t rm = rmask >> row0;
-        float alpha = 1.f;
-        if (rescale) {
-          // New reference max per row: warp transpose-reduction, then across
-          // the group's four warps.
-          float tmp[RW];
+      // Reference max (raw score) of row row0 + lane % RW; -inf until the
+      // row sees a key.  bias[r] = kPShift - cs * (row r's reference max).
+      float m_lane = -INFINITY;
+      bool ok = true;
+      int end_t = 0x7fffffff;  // number of tiles, once published
+
+      // Iteration t scores tile t and folds tile t-2's O^T (finished long
+      // ago) into the register accumulators; the two iterations after the
+      // last tile only fold.  Tile u's rescale factors live in alpha_s[u % 4].
+      for (int t = 0;; ++t) {
+        int gt = -1;  // tile number of local tile t
+        if (t < end_t) {
+          ok = __all_sync(0xffffffffu,
+                          ok && mbar_wait(bar(BAR_INFO + t % kInfoSlots),
+                                          (t / kInfoSlots) & 1, abort));
+          gt = ok ? info[t % kInfoSlots].tile : -1;
+          if (gt < 0) end_t = t;
+        }
+        if (t - 2 >= end_t) break;  // the last tile (end_t - 1) was folded at end_t + 1
+        const bool has_s = t < end_t, has_o = t >= 2;
+        const int sb = t % 2, st = t % kStages, ob = t % 2;  // O of tile t-2 sits in buffer t%2
+        if (has_o)
+          ok = __all_sync(0xffffffffu,
+                          ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
+        if (has_s)
+          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+        float sv[RW], oh[RW], ol[RW];
 #pragma unroll
-          for (int r = 0; r < RW; ++r) tmp[r] = (all_vis || ((rm >> r) & 1u)) ? sv[r] : -INFINITY;
-          const float wmax = warp_row_reduce<RW, true>(tmp, lane);
-          if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
-          __syncwarp();
-          named_bar_sync(bar_id, kSoftmaxThreads);
-          const int rl = lane % RW;
-          float tmax = red[(sb * 4 + 0) * 32 + rl];
-          tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
-          tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
-          tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
-          const float m_new = fmaxf(m_lane, tmax);
-          // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
-          // 2^(cs (s - m_new) + kPShift).
-          alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
-          const float bias_l =
-              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
-          m_lane = m_new;
-          if (lane < RW) {
-            bc[lane] = bias_l;
-            bc[32 + lane] = alpha;
+        for (int r = 0; r < RW; ++r) sv[r] = oh[r] = ol[r] = 0.f;
+        if (ok) {
+          tc_fence_after();
+          if (has_o) {
+            tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + row0, oh);
+            tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + NR + row0, ol);
           }
-          __syncwarp();
-          float av[RW];
+          if (has_s) tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
+          tmem_ld_wait();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (ok && lane == 0) {
+          if (has_o) mbar_arrive(bar(BAR_OEMPTY + ob));
+          if (has_s) mbar_arrive(bar(BAR_SEMPTY + sb));
+        }
+
+        uint32_t rmask = 0;
+        bool all_vis = false;  // every key of this warp is seen by every row
+        float x[RW];           // cs * s + bias: log2 of the scaled weight
+        bool exceed = false;
+        if (has_s) {
+          // Which rows see this key?  Keys of chunks that were not loaded
+          // (outside the visible range or an out-of-range block) see none.
+          const int key = base + gt * kTileKeys + j;
+          if (ok && ((info[t % kInfoSlots].mask >> (j / kChunk)) & 1u) && key >= lo_u &&
+              key <= hi_u) {
+            if (key >= lo_all && key <= hi_all) {
+              rmask = all_rows;
+            } else {
 #pragma unroll
-          for (int r = 0; r < RW; r += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
-            const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
-            bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
-            av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
+              for (int i = 0; i < kMaxQuery; ++i)
+                if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
+            }
           }
+          all_vis = __all_sync(0xffffffffu, rmask == all_rows);
+          const uint32_t rm = rmask >> row0;
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
             x[r] = fmaf(sv[r], cs, bias[r]);
-            lpart[r] *= av[r];
+            const bool vis = all_vis || ((rm >> r) & 1u);
+            exceed |= vis && x[r] > (float)kPShift + kLazy;
           }
         }
-        if (widx == 0 && lane < RW) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
-
-        // Scaled weights, split into an fp16 high part and an fp16 residual.
-        uint32_t phi[RW / 2], plo[RW / 2];
-#pragma unroll
-        for (int r = 0; r < RW; r += 2) {
-          float pr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const bool vis = all_vis || ((rm >> (r + e)) & 1u);
-            pr[e] = vis ? fast_exp2(x[r + e]) : 0.f;
-            lpart[r + e] += pr[e];
-          }
-          const __half2 h = __floats2half2_rn(pr[0], pr[1]);
-          const float2 hf = __half22float2(h);
-          const __half2 l2 = __floats2half2_rn(pr[0] - hf.x, pr[1] - hf.y);
-          phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-          plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-        }
-
-        // A key no row can see must not reach the PV product: zero its V
-        // row (after its V tile has landed).
-        if (g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
-          ok = __all_sync(0xffffffffu,
-                          ok && mbar_wait(bar(BAR_VFULL + st), (t / kStages) & 1, abort));
-          if (ok && rmask == 0) {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              sts_v4(vrow + c * 16, z);
-              sts_v4(vrow + kAtomBytes + c * 16, z);
-            }
-          }
-        }
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_PEMPTY), (t & 1) ^ 1, abort));
-        if (ok) {
-          // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8][row'%8]
-          // with row' < NR the high parts and row' >= NR the residuals.
-          const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
-          constexpr uint32_t lo_off = (NR / 8) * 128;
-          if constexpr (RW >= 8) {
-#pragma unroll
-            for (int r8 = 0; r8 < RW / 8; ++r8) {
-              const uint32_t off = kb + ((row0 / 8) + r8) * 128;
-              sts_v4(sP + off, make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
-              sts_v4(sP + lo_off + off,
-                     make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
-            }
-          } else {  // four rows: half of one 16-byte core-matrix row
-            const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
-            sts_v2(sP + off, phi[0], phi[1]);
-            sts_v2(sP + lo_off + off, plo[0], plo[1]);
-          }
-          fence_proxy_async_smem();
-        }
+        // Reconverge before the group barrier: a warp that arrives diverged
+        // (after lane-predicated code) makes the barrier several times slower
+        // (measured: 61k verify 122 -> 67 us per call).
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL));
-      }
-      ph_cur = ph_nxt;
-    }
-
-    // Row sums: per-thread partials -> per-warp (lane r) -> across warps.
-    const float wl = warp_row_reduce<RW, false>(lpart, lane);
-    if (lane < RW) lsum[widx * 32 + lane] = wl;
-    __syncwarp();
-    named_bar_sync(bar_id, kSoftmaxThreads);
-    const bool aborted = *abort != 0;
+        // One barrier per tile: orders the shared-memory traffic of the group
+        // and tells every thread whether any score passed its row's reference.
+        const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
+        if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
+          const float* al = alpha_s + ((t - 2) % 4) * 32 + row0;
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
-      if (row0 + r < R) {
-        const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
-        const long long pr = part_base + row_index(row0 + r);
-        p.part_out[pr * kHeadDim + j] = (!aborted && l > 0.f) ? acc[r] / l : 0.f;
-      }
-    }
-    if (widx == 0 && lane < RW && row0 + lane < R) {
-      // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
-      const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
-      p.part_lse[part_base + row_index(row0 + lane)] =
-          (!aborted && l > 0.f)
-              ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
-              : -INFINITY;
-    }
-    __syncthreads();  // (A)
-  }
+          for (int r = 0; r < RW; ++r) acc[r] = fmaf(acc[r], al[r], oh[r] + ol[r]);
+        }
+        if (has_s) {
+          const uint32_t rm = rmask >> row0;
+          float alpha = 1.f;
+          if (rescale) {
+            // New reference max per row: warp transpose-reduction, then
+            // across the group's four warps.
+            float tmp[RW];
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+              tmp[r] = (all_vis || ((rm >> r) & 1u)) ? sv[r] : -INFINITY;
+            const float wmax = warp_row_reduce<RW, true>(tmp, lane);
+            if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
+            __syncwarp();
+            named_bar_sync(bar_id, kSoftmaxThreads);
+            const int rl = lane % RW;
+            float tmax = red[(sb * 4 + 0) * 32 + rl];
+            tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
+            tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
+            tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
+            const float m_new = fmaxf(m_lane, tmax);
+            // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
+            // 2^(cs (s - m_new) + kPShift).
+            alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
+            const float bias_l =
+                (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
+            m_lane = m_new;
+            if (lane < RW) {
+              bc[lane] = bias_l;
+              bc[32 + lane] = alpha;
+            }
+            __syncwarp();
+            float av[RW];
+#pragma unroll
+            for (int r = 0; r < RW; r += 4) {
+              const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
+              const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
+              bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
+              av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
+            }
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+              x[r] = fmaf(sv[r], cs, bias[r]);
+              lpart[r] *= av[r];
+            }
+          }
+          if (widx == 0 && lane < RW) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
 
+          // Scaled weights, split into an fp16 high part and an fp16 residual.
+          uint32_t phi[RW / 2], plo[RW / 2];
+#pragma unroll
+          for (int r = 0; r < RW; r += 2) {
+            float pr[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const bool vis = all_vis || ((rm >> (r + e)) & 1u);
+              pr[e] = vis ? fast_exp2(x[r + e]) : 0.f;
+              lpart[r + e] += pr[e];
+            }
+            const __half2 h = __floats2half2_rn(pr[0], pr[1]);
+            const float2 hf = __half22float2(h);
+            const __half2 l2 = __floats2half2_rn(pr[0] - hf.x, pr[1] - hf.y);
+            phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+            plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+
+          // A key no row can see must not reach the PV product: zero its V
+          // row (after its V tile has landed).
+          if (g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
+            ok = __all_sync(0xffffffffu,
+                            ok && mbar_wait(bar(BAR_VFULL + st), (t / kStages) & 1, abort));
+            if (ok && rmask == 0) {
+              const uint4 z = make_uint4(0, 0, 0, 0);
+              const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                sts_v4(vrow + c * 16, z);
+                sts_v4(vrow + kAtomBytes + c * 16, z);
+              }
+            }
+          }
+          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_PEMPTY), (t & 1) ^ 1, abort));
+          if (ok) {
+            // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
+            // [row'%8] with row' < NR the high parts and row' >= NR the
+            // residuals.
+            const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
+            constexpr uint32_t lo_off = (NR / 8) * 128;
+            if constexpr (RW >= 8) {
+#pragma unroll
+              for (int r8 = 0; r8 < RW / 8; ++r8) {
+                const uint32_t off = kb + ((row0 / 8) + r8) * 128;
+                sts_v4(sP + off,
+                       make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
+                sts_v4(sP + lo_off + off,
+                       make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
+              }
+            } else {  // four rows: half of one 16-byte core-matrix row
+              const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
+              sts_v2(sP + off, phi[0], phi[1]);
+              sts_v2(sP + lo_off + off, plo[0], plo[1]);
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL));
+        }
+      }
+
+      // Row sums: per-thread partials -> per-warp (lane r) -> across warps.
+      const float wl = warp_row_reduce<RW, false>(lpart, lane);
+      if (lane < RW) lsum[widx * 32 + lane] = wl;
+      __syncwarp();
+      named_bar_sync(bar_id, kSoftmaxThreads);
+      const bool aborted = *abort != 0;
+#pragma unroll
+      for (int r = 0; r < RW; ++r) {
+        if (row0 + r < R) {
+          const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
+          const long long pr = part_base + row_index(row0 + r);
+          p.part_out[pr * kHeadDim + j] = (!aborted && l > 0.f) ? acc[r] / l : 0.f;
+        }
+      }
+      if (widx == 0 && lane < RW && row0 + lane < R) {
+        // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
+        const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
+        p.part_lse[part_base + row_index(row0 + lane)] =
+            (!aborted && l > 0.f)
+                ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
+                : -INFINITY;
+      }
+      __syncthreads();  // (A)
+    }
+    // ---- tear-down (every thread passed (A)) ---------------------------------
+    if (threadIdx.x == 32 && misc->abort) atomicOr(p.flags, kFlagTimeout);
+    tc_fence_after();
+    if (warp == 1) {
+      __syncwarp();
+      tmem_dealloc(tmem, C::kTmemCols);
+    }
+  }
   // This CTA's partial is written: the merge kernel that follows on the
   // stream may be scheduled (it waits for the whole grid before reading).
   // Triggering any earlier lets idle merge CTAs share the SMs with the
   // decode and slows it (measured: 61k verify 64 -> 70 us per call).
   griddep_launch_dependents();
-  // ---- tear-down (every thread passed (A)) -----------------------------------
-  if (threadIdx.x == 0 && misc->abort) atomicOr(p.flags, kFlagTimeout);
-  tc_fence_after();
-  if (warp == 1) {
-    __syncwarp();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
 }
 
 // ---- host side ----------------------------------------------------------------

@@ -116,6 +116,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Arrive at a named barrier without waiting for it.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 // Named barrier that also ORs a predicate over the participating threads.
 __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t threads, bool v) {
   uint32_t r;

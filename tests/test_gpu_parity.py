@@ -263,7 +263,18 @@ def test_cuda_graph_replay_matches_eager(B):
                                         ("mixed_q8_0", 24), ("sliding_window", 256)])
 def test_full_size_sampled(B, orc, name, nrows):
     case = gen.CONFIGS[name](0)
-    out, _ = run(B, case)
+    dev = B.case_to_device(case)
+    dec = B.PagedDecode.for_case(case)
+    kw = dict(causal=case.causal, window=case.window, scale=case.scale, kv_dtype=case.kv_dtype)
+    args = (dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["context_lens"])
+    first = dec(*args, **kw)
+    second = dec(*args, **kw)
+    torch.cuda.synchronize()
+    assert dec.get_error() == 0
+    # the split partition depends only on the inputs: a repeated call is
+    # bit-identical
+    assert torch.equal(first.view(torch.int16), second.view(torch.int16))
+    out = first.cpu().numpy()
     o = out.reshape(case.rows, case.head_dim)
     assert np.all(np.isfinite(o)), "non-finite output at full size"
     rows = sampled_rows(case, nrows)
