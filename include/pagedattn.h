@@ -96,20 +96,24 @@ typedef struct {
   size_t workspace_bytes;     /* >= paged_attn_workspace_size(dims, n_query) */
 } pa_dims;
 
-/* Bytes of workspace paged_attn_decode needs for these shapes (split
- * partials plus a 256-byte status header).  Host only, no device access.
- * Returns 0 for invalid shapes. */
+/* Bytes of workspace paged_attn_decode needs for these shapes: a 256-byte
+ * status header, one int32 arrival counter per (sequence, KV head) and the
+ * split partials.  Host only, no device access.  Returns 0 for invalid
+ * shapes. */
 size_t paged_attn_workspace_size(const pa_dims* dims, int32_t n_query);
 
-/* Zero the workspace status header (enqueued on `stream`).  Call once after
- * allocating a workspace, before its first paged_attn_decode. */
+/* Zero the workspace status header and arrival counters (enqueued on
+ * `stream`).  Call once after allocating a workspace, before its first
+ * paged_attn_decode; every decode call leaves the counters at zero again. */
 int paged_attn_workspace_init(const pa_dims* dims, void* stream);
 
 /* Decode attention (see the header comment for the exact definition).
  * q, k_cache, v_cache, block_table, context_lens, out: device pointers,
  * 16-byte aligned.  n_query in 1..8; causal 0 or 1; window >= 0 (0 = no
  * window); scale multiplies q.k (usually 1/sqrt(head_dim)); kv_dtype a
- * pa_kv_dtype.  Enqueues the split-KV kernel and the merge on `stream`. */
+ * pa_kv_dtype.  Enqueues the split-KV kernel and the merge of its partials
+ * on `stream` (see paged_attn_launches_per_call).  Calls that share a
+ * workspace must not overlap on the GPU (order them on one stream). */
 int paged_attn_decode(const pa_dims* dims, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* block_table,
                       const int32_t* context_lens, int32_t n_query,
@@ -180,9 +184,11 @@ int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_
                               int32_t kv_dtype, void* out, void* stream);
 
 /* Kernel launches one paged_attn_decode call makes for these shapes and
- * cache type on the current device: the split-KV kernel and the merge kernel
- * (launched as a programmatic dependent so that it starts as soon as the
- * split-KV kernel ends).  Host only; negative pa_status on error. */
+ * cache type on the current device: 1 where the tensor-core kernel runs (the
+ * last CTA of each (sequence, KV head) merges that group's partials), 2 for
+ * the CUDA-core kernel followed by the merge kernel (launched as a
+ * programmatic dependent so that it starts as soon as the split-KV kernel
+ * ends).  Host only; negative pa_status on error. */
 int32_t paged_attn_launches_per_call(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
 
 /* Static string for a pa_status. */

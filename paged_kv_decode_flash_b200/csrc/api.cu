@@ -37,8 +37,8 @@ int32_t paged_attn_launches_per_call(const pa_dims* dims, int32_t n_query, int32
   if (kv_dtype != PA_KV_FP16 && kv_dtype != PA_KV_Q8_0) return PA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  (void)make_plan(dims, n_query, kv_dtype, sms);
-  return 2;  // the split-KV kernel, then the merge kernel
+  // tensor-core kernel: merges in its last CTAs; CUDA-core kernel: + merge kernel
+  return make_plan(dims, n_query, kv_dtype, sms).tensor_cores ? 1 : 2;
 }
 
 int paged_attn_workspace_init(const pa_dims* dims, void* stream) {

@@ -39,6 +39,12 @@ struct DecodeParams {
   float* part_out;            // [B][S][nq*Hq][D]
   float* part_lse;            // [B][S][nq*Hq], natural log
   unsigned* flags;            // workspace status word
+  int* arrivals;              // [B][Hkv][2] per (sequence, KV head): CTAs that
+                              // finished their split / finished merging in
+                              // this call; zero between calls
+  __half* out;                // [B][nq][Hq][D], written by the fused merge
+  int coop;                   // every CTA of the grid is resident at once
+                              // (cooperative launch): groups merge together
 };
 
 struct MergeParams {

@@ -13,11 +13,15 @@
 // Hardware mapping (one CTA per SM, 11 warps):
 //   warps 0, 10 TMA producers for K and for V: resolve the block table and
 //               load whole 16-key chunks (two 64-column halves each, 128-byte
-//               swizzle) into separate 3-slot rings of 128-key tiles; K slots
-//               are released as soon as QK^T has read them, so K runs ahead.
-//   warp 1      MMA issuer (one thread): S^T = K Q^T with M = 128 keys and
-//               N = the query rows, then O^T = V^T [P_hi | P_lo]^T with
-//               M = 128 head_dim lanes; accumulators live in TMEM.
+//               swizzle) into separate rings of 128-key tiles (2-3 slots);
+//               K slots are released as soon as QK^T has read them, so K runs
+//               ahead.
+//   warp 1      MMA issuer (one thread), in a fixed order: QK(0), QK(1), then
+//               PV(t), QK(t+2) for t = 0, 1, ...; S^T = K Q^T with M = 128
+//               keys and N = the query rows, O^T = V^T [P_hi | P_lo]^T with
+//               M = 128 head_dim lanes; accumulators live in TMEM, P is
+//               double-buffered in shared memory so that the softmax of tile
+//               t+1 overlaps the PV product of tile t.
 //   warps 2-9   two softmax warpgroups, each owning half of the query rows:
 //               thread = key for S (row max by a warp transpose-reduction
 //               plus one named barrier per group), thread = head_dim element
@@ -35,8 +39,15 @@
 // zero-filled in shared memory before the PV product (the NaN-poisoned
 // out-of-window blocks of the pages' regression test must not leak).
 //
+// Merge: every CTA counts itself in the arrival counter of its (sequence,
+// KV head) once its partial is written; the last one to arrive merges the
+// group's partials into the fp16 output rows (log-sum-exp weights, splits in
+// a fixed order) and resets the counter.  No CTA ever waits for another, and
+// a call is one launch.
+//
 // Every wait is bounded (sm100::mbar_wait): on a timeout the kernel raises
-// kFlagTimeout, drains its own copies and MMAs, frees TMEM and returns.
+// kFlagTimeout, drains its own copies and MMAs, frees TMEM and still takes
+// part in the merge (its rows count as empty).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -54,7 +65,7 @@ using namespace sm100;
 
 constexpr int kTileKeys = 128;                 // keys per pipeline tile (M of S^T)
 constexpr int kChunksPerTile = kTileKeys / kChunk;
-constexpr int kStages = 3;                     // slots per K ring and per V ring
+constexpr int kMaxStages = 3;                  // slots per K ring and per V ring (at most)
 // A K or V tile of 128 keys in shared memory: [key group of 8][half][8 keys]
 // [64 fp16] with the 128-byte swizzle, i.e. 1 KB swizzle atoms; the atoms of
 // one 64-column half sit 2 KB apart, the two halves of a key group 1 KB apart.
@@ -81,9 +92,8 @@ enum : int {
   BAR_VEMPTY = 9,   // [3] V tile read by PV
   BAR_SFULL = 12,   // [2] S^T in TMEM
   BAR_SEMPTY = 14,  // [2] S^T read by the softmax warps
-  BAR_PFULL = 16,   // P written to shared memory
-  BAR_PEMPTY = 17,  // P consumed by the PV product
-  BAR_OFULL = 18,   // [2] O^T of one tile in TMEM
+  BAR_PFULL = 16,   // [2] P of one tile written to shared memory
+  BAR_OFULL = 18,   // [2] O^T of one tile in TMEM (also: its P buffer is free)
   BAR_OEMPTY = 20,  // [2] O^T read by the softmax warps
   BAR_DONE = 22,    // every MMA finished
   BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
@@ -92,18 +102,23 @@ enum : int {
 constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
 // RW query rows per softmax warpgroup; NR = the MMA's N for S (>= 16).
+// KS / VS slots in the K / V rings: 3 + 3 where shared memory allows, 3 + 2
+// at 32 rows (whose two P buffers take 32 KB).
 template <int RW>
 struct Cfg {
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
+  static constexpr int KS = 3;
+  static constexpr int VS = NR > 16 ? 2 : 3;
   static constexpr uint32_t kK = 0;                                 // K ring
-  static constexpr uint32_t kV = kStages * kKVBytes;                // V ring
-  static constexpr uint32_t kQ = 2 * kStages * kKVBytes;
+  static constexpr uint32_t kV = KS * kKVBytes;                     // V ring
+  static constexpr uint32_t kQ = (KS + VS) * kKVBytes;
   static constexpr uint32_t kQHalf = NR * 128;
   // P^T of one tile: 2*NR "rows" (the fp16 high parts of the NR query rows,
-  // then their residuals), so one MMA with N = 2*NR multiplies both.
+  // then their residuals), so one MMA with N = 2*NR multiplies both.  Two
+  // buffers: tile t uses buffer t % 2.
   static constexpr uint32_t kP = kQ + 2 * kQHalf;
   static constexpr uint32_t kPBytes = kTileKeys * 2 * NR * 2;
-  static constexpr uint32_t kRed = kP + kPBytes;                    // float [2 grp][2][4][32]
+  static constexpr uint32_t kRed = kP + 2 * kPBytes;                // float [2 grp][2][4][32]
   static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4][32]
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
   static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [8 warps][2][32]
@@ -115,12 +130,15 @@ struct Cfg {
   static constexpr uint32_t kTmemUsed = 6 * NR;
   static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
                                         : kTmemUsed <= 128 ? 128 : 256;
+  static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
+  static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
 };
 
 struct Misc {
   uint32_t tmem_base;
   int abort;
   int k_consumed, v_consumed;
+  int last;  // this CTA arrived last in its (sequence, KV head): it merges
 };
 
 // What the K producer publishes for each local tile of a CTA: the tile's
@@ -173,12 +191,195 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
   return v[0];
 }
 
+// The last CTA of a (sequence, KV head) merges the group's split partials
+// into the output rows: M = max_k lse_k, w_k = exp(lse_k - M) (0 for an
+// empty split), out = sum_k w_k O_k / sum_k w_k, splits added in index
+// order.  The group's partial rows are staged in shared memory with 16-byte
+// asynchronous copies, as many splits per round as fit, all of a round in
+// flight at once, so that the merge costs a few memory latencies rather than
+// one per split.
+template <int RW>
+__device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, uint8_t* smem,
+                                            uint32_t sbase) {
+  using C = Cfg<RW>;
+  constexpr int kRowF4 = kHeadDim / 4;  // float4 per partial row
+  constexpr int kWarps = kThreads / 32;
+  constexpr int kPairsMax = (2 * RW * kRowF4 + kThreads - 1) / kThreads;
+  const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
+  const long long rps = (long long)p.n_query * Hq;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  float* w = reinterpret_cast<float*>(smem);  // [S][R]
+  float* inv = w + S * R;                     // [R]
+  const uint32_t stage_off = ((uint32_t)(S * R + R) * 4u + 1023u) & ~1023u;
+  const uint32_t stage = sbase + stage_off;
+  const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);
+  const int per_round = max(1, (int)((C::kRed - stage_off) / (uint32_t)(R * kHeadDim * 4)));
+  auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
+  const long long split0 = (long long)s * S * rps;  // row offset of split 0 of sequence s
+
+  // Raw log-sum-exps, all loads in flight together.
+  for (int i0 = 0; i0 < S * R; i0 += 8 * kThreads) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kThreads + threadIdx.x;
+      v[u] = i < S * R ? __ldcg(p.part_lse + split0 + (long long)(i / R) * rps + row_index(i % R))
+                       : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kThreads + threadIdx.x;
+      if (i < S * R) w[i] = v[u];
+    }
+  }
+  __syncthreads();
+  for (int r = warp; r < R; r += kWarps) {
+    float M = -INFINITY;
+    for (int k = lane; k < S; k += 32) M = fmaxf(M, w[k * R + r]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float sum = 0.f;
+    for (int k = lane; k < S; k += 32) {
+      const float l = w[k * R + r];
+      const float wk = (l == -INFINITY) ? 0.f : expf(l - M);
+      w[k * R + r] = wk;
+      sum += wk;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) inv[r] = sum > 0.f ? 1.f / sum : 0.f;
+  }
+
+  // Thread = (row, 4 consecutive head_dim elements), up to kPairsMax pairs;
+  // empty splits carry weight 0 and a zero partial.
+  float4 acc[kPairsMax];
+#pragma unroll
+  for (int q = 0; q < kPairsMax; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < S; k0 += per_round) {
+    const int k1 = min(S, k0 + per_round);
+    __syncthreads();  // weights ready / the previous round's reads done
+    // Staged row q = (k - k0) * R + r; lane = its float4 column (kThreads is
+    // a multiple of 32, so every copy of this thread has column `lane`).
+    const int nrows = (k1 - k0) * R;
+    for (int q = warp; q < nrows; q += kWarps) {
+      const int k = k0 + q / R, r = q % R;
+      const float* src = p.part_out + (split0 + k * rps + row_index(r)) * kHeadDim + lane * 4;
+      cp_async_16(stage + (uint32_t)(q * kRowF4 + lane) * 16u, src);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kPairsMax; ++q) {
+      const int pr = threadIdx.x + q * kThreads;
+      if (pr < R * kRowF4) {
+        const int r = pr / kRowF4, c4 = pr % kRowF4;
+        for (int k = k0; k < k1; ++k) {
+          const float wk = w[k * R + r];
+          const float4 v = stage4[((k - k0) * R + r) * kRowF4 + c4];
+          acc[q].x = fmaf(wk, v.x, acc[q].x);
+          acc[q].y = fmaf(wk, v.y, acc[q].y);
+          acc[q].z = fmaf(wk, v.z, acc[q].z);
+          acc[q].w = fmaf(wk, v.w, acc[q].w);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kPairsMax; ++q) {
+    const int pr = threadIdx.x + q * kThreads;
+    if (pr < R * kRowF4) {
+      const int r = pr / kRowF4, c4 = pr % kRowF4;
+      const float iv = inv[r];
+      const __half2 h0 = __floats2half2_rn(acc[q].x * iv, acc[q].y * iv);
+      const __half2 h1 = __floats2half2_rn(acc[q].z * iv, acc[q].w * iv);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&h0);
+      u.y = *reinterpret_cast<const uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
+    }
+  }
+}
+
+// Cooperative merge (every CTA of the grid resident): once its whole group
+// has written its partials, split k of a (sequence, KV head) merges pairs
+// [k*P/S, (k+1)*P/S) of the group's P = R*32 (row, float4 column) pairs.
+// Same arithmetic as merge_group (log-sum-exp weights, splits added in index
+// order), spread over all S CTAs of the group so that each stages only a
+// few kilobytes of partials with one round of 16-byte asynchronous copies.
+template <int RW>
+__device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split,
+                                            uint8_t* smem, uint32_t sbase) {
+  constexpr int kRowF4 = kHeadDim / 4;
+  constexpr int kWarps = kThreads / 32;
+  const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
+  const long long rps = (long long)p.n_query * Hq;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int P = R * kRowF4;
+  const int pa = (int)((long long)split * P / S), pb = (int)((long long)(split + 1) * P / S);
+  if (pa >= pb) return;  // uniform across the CTA
+  const int r_lo = pa / kRowF4, nr = (pb - 1) / kRowF4 - r_lo + 1, np = pb - pa;
+  auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
+  const long long split0 = (long long)s * S * rps;  // row offset of split 0 of sequence s
+  float* w = reinterpret_cast<float*>(smem);  // [nr][S]
+  float* inv = w + nr * S;                    // [nr]
+  const uint32_t stage_off = ((uint32_t)(nr * S + nr) * 4u + 1023u) & ~1023u;
+  const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);  // [S][np]
+
+  // The partial columns first (the longest wait), then the log-sum-exps.
+  for (int e = threadIdx.x; e < S * np; e += kThreads) {
+    const int k = e / np, pr = pa + e % np;
+    const float* src =
+        p.part_out + (split0 + k * rps + row_index(pr / kRowF4)) * kHeadDim + (pr % kRowF4) * 4;
+    cp_async_16(sbase + stage_off + (uint32_t)e * 16u, src);
+  }
+  for (int e = threadIdx.x; e < nr * S; e += kThreads)
+    w[e] = __ldcg(p.part_lse + split0 + (long long)(e % S) * rps + row_index(r_lo + e / S));
+  __syncthreads();
+  for (int j = warp; j < nr; j += kWarps) {
+    float M = -INFINITY;
+    for (int k = lane; k < S; k += 32) M = fmaxf(M, w[j * S + k]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float sum = 0.f;
+    for (int k = lane; k < S; k += 32) {
+      const float l = w[j * S + k];
+      const float wk = (l == -INFINITY) ? 0.f : expf(l - M);
+      w[j * S + k] = wk;
+      sum += wk;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) inv[j] = sum > 0.f ? 1.f / sum : 0.f;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  for (int q = threadIdx.x; q < np; q += kThreads) {
+    const int pr = pa + q, r = pr / kRowF4, c4 = pr % kRowF4, j = r - r_lo;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < S; ++k) {
+      const float wk = w[j * S + k];
+      const float4 v = stage4[k * np + q];
+      acc.x = fmaf(wk, v.x, acc.x);
+      acc.y = fmaf(wk, v.y, acc.y);
+      acc.z = fmaf(wk, v.z, acc.z);
+      acc.w = fmaf(wk, v.w, acc.w);
+    }
+    const float iv = inv[j];
+    const __half2 h0 = __floats2half2_rn(acc.x * iv, acc.y * iv);
+    const __half2 h1 = __floats2half2_rn(acc.z * iv, acc.w * iv);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&h0);
+    u.y = *reinterpret_cast<const uint32_t*>(&h1);
+    *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
+  }
+}
+
 template <int RW>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using C = Cfg<RW>;
-  constexpr int NR = C::NR;
+  constexpr int NR = C::NR, KS = C::KS, VS = C::VS;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the __shared__ array by pointer
   // arithmetic so that accesses through it stay shared-space loads/stores.
@@ -216,24 +417,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
   const int t_first = split * t_per + min(split, t_rem);
   const int t_count = t_per + (split < t_rem ? 1 : 0);
-  if (t_count == 0) {  // every tile is another CTA's: an empty partial
-    for (int t = threadIdx.x; t < R * kHeadDim; t += kThreads) {
-      const int r = t / kHeadDim;
-      p.part_out[(part_base + row_index(r)) * kHeadDim + t % kHeadDim] = 0.f;
-      if (t % kHeadDim == 0) p.part_lse[part_base + row_index(r)] = -INFINITY;
-    }
-    griddep_launch_dependents();
-    return;
-  }
   const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
 
   const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
   const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
 
-  if (warp == 0) {
+  if (t_count == 0) {
+    // Every tile is another CTA's: an empty partial (weight 0 in the merge).
+    for (int t = threadIdx.x; t < R * kHeadDim; t += kThreads) {
+      const int r = t / kHeadDim;
+      p.part_out[(part_base + row_index(r)) * kHeadDim + t % kHeadDim] = 0.f;
+      if (t % kHeadDim == 0) p.part_lse[part_base + row_index(r)] = -INFINITY;
+    }
+  } else if (warp == 0) {
     // ======================= K producer (also sets up the barriers) ========
     if (lane == 0) {
-      for (int i = 0; i < kStages; ++i) {
+      for (int i = 0; i < kMaxStages; ++i) {
         mbar_init(bar(BAR_KFULL + i), 1);
         mbar_init(bar(BAR_KEMPTY + i), 1);
         mbar_init(bar(BAR_VFULL + i), 1);
@@ -242,11 +441,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 2; ++i) {
         mbar_init(bar(BAR_SFULL + i), 1);
         mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
+        mbar_init(bar(BAR_PFULL + i), 4 * kGroups);
         mbar_init(bar(BAR_OFULL + i), 1);
         mbar_init(bar(BAR_OEMPTY + i), 4 * kGroups);
       }
-      mbar_init(bar(BAR_PFULL), 4 * kGroups);
-      mbar_init(bar(BAR_PEMPTY), 1);
       mbar_init(bar(BAR_DONE), 1);
       for (int i = 0; i < kInfoSlots; ++i) mbar_init(bar(BAR_INFO + i), 1);
       misc->abort = 0;
@@ -257,27 +455,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The other roles wait for these barriers; this warp starts loading now.
     named_bar_arrive(3, kThreads);
 
-    // Lane c < 8 owns chunk c of every tile and reads its block-table entry
-    // one tile ahead.
+    // Lane c < 8 owns chunk c of every tile.  Its block-table entry for tile
+    // t + 1 is read right after tile t's copy is issued and used one slot
+    // wait later, so the load's latency hides behind that wait.
     const int c = lane;
-    auto lookup = [&](int g, int& row8) -> bool {
-      if (g < 0 || c >= kChunksPerTile) return false;
+    constexpr long long kNone = -(1LL << 40);
+    auto tile_of = [&](int t) { return t < t_count ? t_first + t : -1; };
+    // Physical block of chunk c of local tile t (kNone: not loaded).
+    auto lookup_raw = [&](int t) -> long long {
+      const int g = tile_of(t);
+      if (g < 0 || c >= kChunksPerTile) return kNone;
       const int key0 = base + g * kTileKeys + c * kChunk;
-      if (key0 > hi_u || key0 + kChunk - 1 < lo_u) return false;
-      const long long phys = table[key0 / p.block_size];
+      if (key0 > hi_u || key0 + kChunk - 1 < lo_u) return kNone;
+      return table[key0 / p.block_size];
+    };
+    // TMA row coordinate (row / 8) of that chunk, -1 if it is not loaded.
+    auto to_row8 = [&](long long phys, int t) -> int {
+      if (phys == kNone) return -1;
       if (phys < 0 || phys >= p.num_blocks) {
         atomicOr(p.flags, kFlagBadBlock);  // masked, never dereferenced
-        return false;
+        return -1;
       }
-      row8 = (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
-      return true;
+      const int key0 = base + tile_of(t) * kTileKeys + c * kChunk;
+      return (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
     };
-    auto tile_of = [&](int t) { return t < t_count ? t_first + t : -1; };
-    int g_cur = tile_of(0);
-    int row_cur = 0, row_nxt = 0;
-    bool w_cur = lookup(g_cur, row_cur);
+    int row_cur = to_row8(lookup_raw(0), 0);
+    long long raw_nxt = lookup_raw(1);
     int issued = 0;
     for (int t = 0;; ++t) {
+      const int g_cur = tile_of(t);
+      const bool w_cur = row_cur >= 0;
       // Publish tile t for the V producer, the MMA issuer and the softmax.
       const uint32_t mask = __ballot_sync(0xffffffffu, w_cur);
       TileInfo& ti = info[t % kInfoSlots];
@@ -289,13 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_INFO + t % kInfoSlots));
       if (g_cur < 0) break;
-      // Tile t + 1's block-table entries, read while tile t's slot frees up.
-      const int g_nxt = tile_of(t + 1);
-      const bool w_nxt = lookup(g_nxt, row_nxt);
       // Wait for the slot, then every lane issues its chunk's copy.
-      const int st = t % kStages;
+      const int st = t % KS;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar(BAR_KEMPTY + st), ((t / kStages) & 1) ^ 1, abort);
+      if (lane == 0) ok = mbar_wait(bar(BAR_KEMPTY + st), ((t / KS) & 1) ^ 1, abort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       const uint32_t fb = bar(BAR_KFULL + st);
@@ -304,15 +508,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w_cur) tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
       __syncwarp();
       issued = t + 1;
-      g_cur = g_nxt;
-      w_cur = w_nxt;
-      row_cur = row_nxt;
+      row_cur = to_row8(raw_nxt, t + 1);
+      raw_nxt = lookup_raw(t + 2);
     }
     __syncthreads();  // (A) every role finished its loop
     if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
       volatile int no_abort = 0;
       for (int t = misc->k_consumed; t < issued; ++t)
-        mbar_wait(bar(BAR_KFULL + t % kStages), (t / kStages) & 1, &no_abort);
+        mbar_wait(bar(BAR_KFULL + t % KS), (t / KS) & 1, &no_abort);
     }
   } else {
     // ---- set-up of the other roles ----------------------------------------
@@ -338,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
       }
-      for (uint32_t off = t * 16; off < C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
+      for (uint32_t off = t * 16; off < 2 * C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
         sts_v4(sP + off, make_uint4(0, 0, 0, 0));
       fence_proxy_async_smem();
     }
@@ -363,8 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ti.tile < 0) break;
         const uint32_t mask = ti.mask;
         const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;
-        const int st = t % kStages;
-        if (lane == 0) ok = mbar_wait(bar(BAR_VEMPTY + st), ((t / kStages) & 1) ^ 1, abort);
+        const int st = t % VS;
+        if (lane == 0) ok = mbar_wait(bar(BAR_VEMPTY + st), ((t / VS) & 1) ^ 1, abort);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const uint32_t fb = bar(BAR_VFULL + st);
@@ -379,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
         volatile int no_abort = 0;
         for (int t = misc->v_consumed; t < issued; ++t)
-          mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, &no_abort);
+          mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, &no_abort);
       }
     } else if (warp == 1) {
       // ===================== MMA issuer ======================================
@@ -392,74 +595,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
         const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
         const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
-        int nqk = 0;              // QK^T products issued
-        int end_t = 0x7fffffff;   // number of tiles, once the producer said so
-        // Issue QK^T of tile nqk if it exists and its K tile and S buffer are
-        // ready (or wait for them when `block`).  1 = issued, 0 = not ready or
-        // no such tile, -1 = gave up.
-        auto try_qk = [&](bool block) -> int {
-          if (nqk >= end_t) return 0;
-          const uint32_t ib = bar(BAR_INFO + nqk % kInfoSlots), ip = (nqk / kInfoSlots) & 1;
-          if (block) {
-            if (!mbar_wait(ib, ip, abort)) return -1;
-          } else if (!mbar_test_wait(ib, ip)) {
-            return 0;
-          }
-          if (info[nqk % kInfoSlots].tile < 0) {
-            end_t = nqk;
-            return 0;
-          }
-          const uint32_t f = bar(BAR_KFULL + nqk % kStages), e = bar(BAR_SEMPTY + nqk % 2);
-          const uint32_t pf = (nqk / kStages) & 1, pe = ((nqk / 2) & 1) ^ 1;
-          if (block) {
-            if (!(mbar_wait(f, pf, abort) && mbar_wait(e, pe, abort))) return -1;
-          } else if (!(mbar_test_wait(f, pf) && mbar_test_wait(e, pe))) {
-            return 0;
-          }
+        // QK^T of tile u once it exists and its K tile and S buffer are
+        // ready: 1 = issued, 0 = there is no tile u, -1 = gave up.
+        auto issue_qk = [&](int u) -> int {
+          if (!mbar_wait(bar(BAR_INFO + u % kInfoSlots), (u / kInfoSlots) & 1, abort)) return -1;
+          if (info[u % kInfoSlots].tile < 0) return 0;
+          if (!(mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, abort) &&
+                mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
+            return -1;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((nqk % kStages) * kKVBytes) >> 4;
-          const uint32_t d = tmem + (nqk % 2) * NR;
+          const uint64_t so = (uint64_t)((u % KS) * kKVBytes) >> 4;
+          const uint32_t d = tmem + (u % 2) * NR;
 #pragma unroll
           for (int k = 0; k < kHeadDim / 16; ++k) {
             const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
             const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
             tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
           }
-          tc_commit(bar(BAR_SFULL + nqk % 2));
-          tc_commit(bar(BAR_KEMPTY + nqk % kStages));
-          ++nqk;
+          tc_commit(bar(BAR_SFULL + u % 2));
+          tc_commit(bar(BAR_KEMPTY + u % KS));
           return 1;
         };
-        int npv = 0;
+        int nqk = 0, npv = 0;
+        int end_t = 0x7fffffff;  // number of tiles, once known
         bool ok = true;
-        for (int t = 0; ok; ++t) {
-          if (nqk <= t && try_qk(true) < 0) { ok = false; break; }  // QK(t) comes first
-          if (t >= end_t) break;                                     // no tile t
-          if (nqk == t + 1) try_qk(false);
-          // Wait for P(t), issuing QK(t+1) as soon as its K tile lands.
-          const unsigned long long t0 = globaltimer();
-          while (!mbar_try_wait_ns(bar(BAR_PFULL), t & 1, 200)) {
-            if (nqk == t + 1) try_qk(false);
-            if (*abort || globaltimer() - t0 > kWaitLimitNs) { *abort = 1; ok = false; break; }
-          }
-          if (!ok) break;
-          ok = mbar_wait(bar(BAR_VFULL + t % kStages), (t / kStages) & 1, abort) &&
+        for (int u = 0; u < 2 && ok && u < end_t; ++u) {
+          const int r = issue_qk(u);
+          if (r < 0) ok = false;
+          else if (r == 0) end_t = u;
+          else nqk = u + 1;
+        }
+        for (int t = 0; ok && t < end_t; ++t) {
+          // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2)
+          // (its S buffer is free once the softmax has taken S(t)).
+          ok = mbar_wait(bar(BAR_PFULL + t % 2), (t / 2) & 1, abort) &&
+               mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort) &&
                mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((t % kStages) * kKVBytes) >> 4;
+          const uint64_t so = (uint64_t)((t % VS) * kKVBytes) >> 4;
+          const uint64_t pb = (uint64_t)((t % 2) * C::kPBytes) >> 4;
           const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
 #pragma unroll
           for (int k = 0; k < kTileKeys / 16; ++k) {
             const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
             const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
-            tc_mma_f16_ss(d, dV + so + vo, dP + po, id_pv, k > 0);
+            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, k > 0);
           }
           tc_commit(bar(BAR_OFULL + t % 2));
-          tc_commit(bar(BAR_PEMPTY));
-          tc_commit(bar(BAR_VEMPTY + t % kStages));
+          tc_commit(bar(BAR_VEMPTY + t % VS));
           npv = t + 1;
-          if (nqk == t + 1) try_qk(false);
+          if (t + 2 < end_t) {
+            const int r = issue_qk(t + 2);
+            if (r < 0) ok = false;
+            else if (r == 0) end_t = t + 2;
+            else nqk = t + 3;
+          }
         }
         misc->k_consumed = nqk;
         misc->v_consumed = npv;
@@ -517,6 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Iteration t scores tile t and folds tile t-2's O^T (finished long
       // ago) into the register accumulators; the two iterations after the
       // last tile only fold.  Tile u's rescale factors live in alpha_s[u % 4].
+      // Waiting for O(t-2) also frees P buffer t % 2 (PV(t-2) read it).
       for (int t = 0;; ++t) {
         int gt = -1;  // tile number of local tile t
         if (t < end_t) {
@@ -528,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t - 2 >= end_t) break;  // the last tile (end_t - 1) was folded at end_t + 1
         const bool has_s = t < end_t, has_o = t >= 2;
-        const int sb = t % 2, st = t % kStages, ob = t % 2;  // O of tile t-2 sits in buffer t%2
+        const int sb = t % 2, st = t % VS, ob = t % 2;  // O of tile t-2 sits in buffer t%2
         if (has_o)
           ok = __all_sync(0xffffffffu,
                           ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
@@ -661,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // row (after its V tile has landed).
           if (g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
             ok = __all_sync(0xffffffffu,
-                            ok && mbar_wait(bar(BAR_VFULL + st), (t / kStages) & 1, abort));
+                            ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
             if (ok && rmask == 0) {
               const uint4 z = make_uint4(0, 0, 0, 0);
               const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
@@ -672,31 +864,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_PEMPTY), (t & 1) ^ 1, abort));
           if (ok) {
             // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
             // [row'%8] with row' < NR the high parts and row' >= NR the
-            // residuals.
+            // residuals, in P buffer t % 2.
+            const uint32_t pbuf = sP + (t % 2) * C::kPBytes;
             const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
             constexpr uint32_t lo_off = (NR / 8) * 128;
             if constexpr (RW >= 8) {
 #pragma unroll
               for (int r8 = 0; r8 < RW / 8; ++r8) {
                 const uint32_t off = kb + ((row0 / 8) + r8) * 128;
-                sts_v4(sP + off,
+                sts_v4(pbuf + off,
                        make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
-                sts_v4(sP + lo_off + off,
+                sts_v4(pbuf + lo_off + off,
                        make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
               }
             } else {  // four rows: half of one 16-byte core-matrix row
               const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
-              sts_v2(sP + off, phi[0], phi[1]);
-              sts_v2(sP + lo_off + off, plo[0], plo[1]);
+              sts_v2(pbuf + off, phi[0], phi[1]);
+              sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
             }
             fence_proxy_async_smem();
           }
           __syncwarp();
-          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL));
+          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % 2));
         }
       }
 
@@ -732,11 +924,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, C::kTmemCols);
     }
   }
-  // This CTA's partial is written: the merge kernel that follows on the
-  // stream may be scheduled (it waits for the whole grid before reading).
-  // Triggering any earlier lets idle merge CTAs share the SMs with the
-  // decode and slows it (measured: 61k verify 64 -> 70 us per call).
-  griddep_launch_dependents();
+
+  // ---- arrival and merge --------------------------------------------------------
+  // Writers make their partials visible device-wide before they are counted.
+  // Counters (two per group) are zero at the start of a call and are reset
+  // by the call itself once no CTA of the group needs them any more (the
+  // next launch on the stream starts after this grid ends).
+  if (t_count == 0 && threadIdx.x == 0) misc->abort = 0;  // set by the K producer otherwise
+  __threadfence();
+  __syncthreads();  // (B) partials written, copies drained, TMEM freed
+  int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
+  if (p.coop) {
+    // Every CTA of the grid is resident: wait (bounded) until the whole group
+    // has written its partials, then merge this CTA's share of the group.
+    if (threadIdx.x == 0) {
+      atomicAdd(cnt, 1);
+      const unsigned long long t0 = globaltimer();
+      int ok = 1;
+      while (ld_acquire_gpu(cnt) < S) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          ok = 0;
+          break;
+        }
+        __nanosleep(32);
+      }
+      misc->last = ok;
+    }
+    __syncthreads();
+    __threadfence();
+    if (misc->last) {
+      merge_slice<RW>(p, s, kvh, split, smem, sbase);
+    } else if (threadIdx.x == 0) {
+      atomicOr(p.flags, kFlagTimeout);
+    }
+    __syncthreads();
+    // The last CTA of the group to finish merging: every CTA of the group
+    // has passed its wait, so both counters can return to zero.
+    if (threadIdx.x == 0 && atomicAdd(cnt + 1, 1) == S - 1) {
+      atomicExch(cnt, 0);
+      atomicExch(cnt + 1, 0);
+    }
+    return;
+  }
+  // Otherwise the last CTA of the group to arrive merges all of it.
+  if (threadIdx.x == 0) misc->last = (atomicAdd(cnt, 1) == S - 1);
+  __syncthreads();
+  if (!misc->last) return;
+  __threadfence();  // the other CTAs' partials, published before their counts
+  merge_group<RW>(p, s, kvh, smem, sbase);
+  if (threadIdx.x == 0) *cnt = 0;
 }
 
 // ---- host side ----------------------------------------------------------------
@@ -771,22 +1007,40 @@ bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
 }
 
 template <int RW>
-cudaError_t launch_rw(const DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& mv,
                       cudaStream_t stream) {
   const size_t smem = Cfg<RW>::kTotal + 1024;
-  static bool configured[64] = {};
+  static int resident[64] = {};  // CTAs of this kernel the device holds at once (0: unknown)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  if (dev < 0 || dev >= 64 || resident[dev] == 0) {
     e = cudaFuncSetAttribute(decode_tc_kernel<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW>, kThreads,
+                                                      smem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) resident[dev] = per_sm * sms;
   }
-  const dim3 grid(p.num_splits, p.num_kv_heads, p.num_seqs);
-  decode_tc_kernel<RW><<<grid, kThreads, smem, stream>>>(mk, mv, p);
-  return cudaGetLastError();
+  const long long ctas = (long long)p.num_splits * p.num_kv_heads * p.num_seqs;
+  // A cooperative launch guarantees that every CTA is resident at once, which
+  // the group-wide merge waits rely on; larger grids merge in their last CTA.
+  p.coop = (dev >= 0 && dev < 64 && ctas <= resident[dev]) ? 1 : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_splits, p.num_kv_heads, p.num_seqs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.coop ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW>, mk, mv, p);
 }
 
 }  // namespace

@@ -92,7 +92,10 @@ Plan max_plan(const pa_dims* d) {
   return pl;
 }
 
-size_t ws_zero_prefix(const pa_dims*) { return kWsHeader; }
+// Status header, then two arrival counters per (sequence, KV head).
+size_t ws_zero_prefix(const pa_dims* d) {
+  return kWsHeader + align256((size_t)d->num_seqs * d->num_kv_heads * 2 * sizeof(int));
+}
 
 WsLayout ws_layout(const pa_dims* d, int n_query, int splits) {
   const size_t rows = (size_t)d->num_seqs * splits * n_query * d->num_q_heads;
@@ -144,9 +147,12 @@ int enqueue_decode(const pa_dims* d, const Plan& plan, const void* q, const void
   p.part_out = reinterpret_cast<float*>(ws + w.part_out);
   p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
   p.flags = reinterpret_cast<unsigned*>(ws);
+  p.arrivals = reinterpret_cast<int*>(ws + kWsHeader);
+  p.out = static_cast<__half*>(out);
 
-  const cudaError_t e = plan.tensor_cores ? launch_decode_tc(p, st) : launch_decode_simt(p, st);
-  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (plan.tensor_cores)  // one launch: the last CTA of each group merges
+    return launch_decode_tc(p, st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  if (launch_decode_simt(p, st) != cudaSuccess) return PA_ERR_CUDA;
   MergeParams m{};
   m.part_out = p.part_out;
   m.part_lse = p.part_lse;

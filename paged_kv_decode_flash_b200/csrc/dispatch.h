@@ -17,8 +17,9 @@ struct Plan {
   int splits, blocks_per_split;
 };
 
-// Workspace: status header | split partial outputs | split partial
-// log-sum-exps.  The header must be zero before the first call.
+// Workspace: status header | arrival counters | split partial outputs |
+// split partial log-sum-exps.  Header and counters (the zero prefix) must be
+// zero before the first call; every call leaves the counters at zero.
 struct WsLayout {
   size_t part_out, part_lse, total;
 };
