@@ -56,8 +56,11 @@
  * errors are found on the host before anything is enqueued.  Data errors
  * that only the device can see (a block index outside [0, num_blocks), a
  * context length outside [n_query, max_blocks_per_seq * block_size]) do not
- * trap: the keys of an out-of-range block are treated as masked, the rows of
- * a sequence with a bad length are written as 0, and a flag is raised in the
+ * trap and never dereference the bad index: the rows of a sequence with a
+ * bad length are written as 0; rows whose visible keys reach an out-of-range
+ * block get finite values that are otherwise unspecified (the tensor-core
+ * kernel writes the rows of that (sequence, KV head) as 0, the CUDA-core
+ * kernel leaves the block's keys out); either way a flag is raised in the
  * workspace that paged_attn_get_error reports.
  */
 #ifndef PAGEDATTN_H

@@ -10,18 +10,18 @@
 // left for the log-sum-exp merge.  Masks and block-table resolution follow
 // section "Bug 2: the drafter read freed memory".
 //
-// Hardware mapping (one CTA per SM, 11 warps):
+// Hardware mapping (one CTA per SM, 12 warps):
 //   warps 0, 10 TMA producers for K and for V: resolve the block table and
 //               load whole 16-key chunks (two 64-column halves each, 128-byte
 //               swizzle) into separate rings of 128-key tiles (2-3 slots);
 //               K slots are released as soon as QK^T has read them, so K runs
-//               ahead.
-//   warp 1      MMA issuer (one thread), in a fixed order: QK(0), QK(1), then
-//               PV(t), QK(t+2) for t = 0, 1, ...; S^T = K Q^T with M = 128
-//               keys and N = the query rows, O^T = V^T [P_hi | P_lo]^T with
-//               M = 128 head_dim lanes; accumulators live in TMEM, P is
-//               double-buffered in shared memory so that the softmax of tile
-//               t+1 overlaps the PV product of tile t.
+//               ahead.  With each K copy the same chunk of V is prefetched
+//               into L2, so that V's own copy a tile later is short.
+//   warps 1, 11 MMA issuers (one thread each): warp 1 S^T = K Q^T with
+//               M = 128 keys and N = the query rows, warp 11 O^T = V^T
+//               [P_hi | P_lo]^T with M = 128 head_dim lanes; accumulators live
+//               in TMEM, P is double-buffered in shared memory so that the
+//               softmax of tile t+1 overlaps the PV product of tile t.
 //   warps 2-9   two softmax warpgroups, each owning half of the query rows:
 //               thread = key for S (row max by a warp transpose-reduction
 //               plus one named barrier per group), thread = head_dim element
@@ -102,23 +102,27 @@ enum : int {
 constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
 // RW query rows per softmax warpgroup; NR = the MMA's N for S (>= 16).
-// KS / VS slots in the K / V rings: 3 + 3 where shared memory allows, 3 + 2
-// at 32 rows (whose two P buffers take 32 KB).
+// KS / VS slots in the K / V rings, PB buffers for P (two, so that the
+// softmax of tile t+1 never waits for PV(t)).  At 32 rows the two P buffers
+// take 32 KB and the V ring keeps two slots (measured: three V slots with
+// one P buffer is slower).  With one P buffer the softmax of tile t waits
+// for PV(t-1) before it stores P(t).
 template <int RW>
 struct Cfg {
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
   static constexpr int KS = 3;
   static constexpr int VS = NR > 16 ? 2 : 3;
+  static constexpr int PB = 2;
   static constexpr uint32_t kK = 0;                                 // K ring
   static constexpr uint32_t kV = KS * kKVBytes;                     // V ring
   static constexpr uint32_t kQ = (KS + VS) * kKVBytes;
   static constexpr uint32_t kQHalf = NR * 128;
   // P^T of one tile: 2*NR "rows" (the fp16 high parts of the NR query rows,
-  // then their residuals), so one MMA with N = 2*NR multiplies both.  Two
-  // buffers: tile t uses buffer t % 2.
+  // then their residuals), so one MMA with N = 2*NR multiplies both.  Tile t
+  // uses buffer t % PB.
   static constexpr uint32_t kP = kQ + 2 * kQHalf;
   static constexpr uint32_t kPBytes = kTileKeys * 2 * NR * 2;
-  static constexpr uint32_t kRed = kP + 2 * kPBytes;                // float [2 grp][2][4][32]
+  static constexpr uint32_t kRed = kP + PB * kPBytes;               // float [2 grp][2][4][32]
   static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4][32]
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
   static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [8 warps][2][32]
@@ -139,6 +143,7 @@ struct Misc {
   int abort;
   int k_consumed, v_consumed;
   int last;  // this CTA arrived last in its (sequence, KV head): it merges
+  int bad;   // a block index of this CTA's keys was out of range
 };
 
 // What the K producer publishes for each local tile of a CTA: the tile's
@@ -235,13 +240,18 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
   __syncthreads();
   for (int r = warp; r < R; r += kWarps) {
     float M = -INFINITY;
-    for (int k = lane; k < S; k += 32) M = fmaxf(M, w[k * R + r]);
+    bool bad = false;  // a split read a stand-in for an out-of-range block
+    for (int k = lane; k < S; k += 32) {
+      M = fmaxf(M, w[k * R + r]);
+      bad |= isnan(w[k * R + r]);
+    }
+    bad = __any_sync(0xffffffffu, bad);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float sum = 0.f;
     for (int k = lane; k < S; k += 32) {
       const float l = w[k * R + r];
-      const float wk = (l == -INFINITY) ? 0.f : expf(l - M);
+      const float wk = (bad || l == -INFINITY) ? 0.f : expf(l - M);
       w[k * R + r] = wk;
       sum += wk;
     }
@@ -337,13 +347,18 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   __syncthreads();
   for (int j = warp; j < nr; j += kWarps) {
     float M = -INFINITY;
-    for (int k = lane; k < S; k += 32) M = fmaxf(M, w[j * S + k]);
+    bool bad = false;  // a split read a stand-in for an out-of-range block
+    for (int k = lane; k < S; k += 32) {
+      M = fmaxf(M, w[j * S + k]);
+      bad |= isnan(w[j * S + k]);
+    }
+    bad = __any_sync(0xffffffffu, bad);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float sum = 0.f;
     for (int k = lane; k < S; k += 32) {
       const float l = w[j * S + k];
-      const float wk = (l == -INFINITY) ? 0.f : expf(l - M);
+      const float wk = (bad || l == -INFINITY) ? 0.f : expf(l - M);
       w[j * S + k] = wk;
       sum += wk;
     }
@@ -379,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using C = Cfg<RW>;
-  constexpr int NR = C::NR, KS = C::KS, VS = C::VS;
+  constexpr int NR = C::NR, KS = C::KS, VS = C::VS, PB = C::PB;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the __shared__ array by pointer
   // arithmetic so that accesses through it stay shared-space loads/stores.
@@ -448,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BAR_DONE), 1);
       for (int i = 0; i < kInfoSlots; ++i) mbar_init(bar(BAR_INFO + i), 1);
       misc->abort = 0;
+      misc->bad = 0;
       misc->k_consumed = misc->v_consumed = 0;
       fence_mbar_init();
     }
@@ -470,11 +486,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       return table[key0 / p.block_size];
     };
     // TMA row coordinate (row / 8) of that chunk, -1 if it is not loaded.
+    // An out-of-range block is never dereferenced: row 0 of the cache stands
+    // in for it (so that every visible key has finite-or-not data the
+    // softmax need not know about), the error flag is raised, and the CTA's
+    // partial is marked invalid so that the merge writes the group's rows
+    // as 0.
     auto to_row8 = [&](long long phys, int t) -> int {
       if (phys == kNone) return -1;
       if (phys < 0 || phys >= p.num_blocks) {
-        atomicOr(p.flags, kFlagBadBlock);  // masked, never dereferenced
-        return -1;
+        atomicOr(p.flags, kFlagBadBlock);
+        misc->bad = 1;
+        return 0;
       }
       const int key0 = base + tile_of(t) * kTileKeys + c * kChunk;
       return (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
@@ -505,7 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t fb = bar(BAR_KFULL + st);
       if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
       __syncwarp();
-      if (w_cur) tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
+      if (w_cur) {
+        tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
+        tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+      }
       __syncwarp();
       issued = t + 1;
       row_cur = to_row8(raw_nxt, t + 1);
@@ -541,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
       }
-      for (uint32_t off = t * 16; off < 2 * C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
+      for (uint32_t off = t * 16; off < PB * C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
         sts_v4(sP + off, make_uint4(0, 0, 0, 0));
       fence_proxy_async_smem();
     }
@@ -586,6 +611,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ===================== MMA issuer ======================================
+      // One thread, in a fixed order: QK(0), QK(1), then PV(t), QK(t+2) for
+      // t = 0, 1, ...  A commit completes once every MMA this thread issued
+      // before it has finished, so S(t) in TMEM also means that O(t-2) is:
+      // the softmax waits for one barrier per tile.  The number of tiles is
+      // t_count (uniform), so the issuer reads no published tile information.
       if (lane == 0) {
         const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
         const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
@@ -595,14 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
         const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
         const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
-        // QK^T of tile u once it exists and its K tile and S buffer are
-        // ready: 1 = issued, 0 = there is no tile u, -1 = gave up.
-        auto issue_qk = [&](int u) -> int {
-          if (!mbar_wait(bar(BAR_INFO + u % kInfoSlots), (u / kInfoSlots) & 1, abort)) return -1;
-          if (info[u % kInfoSlots].tile < 0) return 0;
+        // QK(u) once K(u) landed and the softmax took S(u-2) from its buffer.
+        auto issue_qk = [&](int u) -> bool {
           if (!(mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, abort) &&
                 mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
-            return -1;
+            return false;
           tc_fence_after();
           const uint64_t so = (uint64_t)((u % KS) * kKVBytes) >> 4;
           const uint32_t d = tmem + (u % 2) * NR;
@@ -614,27 +641,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(BAR_SFULL + u % 2));
           tc_commit(bar(BAR_KEMPTY + u % KS));
-          return 1;
+          return true;
         };
         int nqk = 0, npv = 0;
-        int end_t = 0x7fffffff;  // number of tiles, once known
         bool ok = true;
-        for (int u = 0; u < 2 && ok && u < end_t; ++u) {
-          const int r = issue_qk(u);
-          if (r < 0) ok = false;
-          else if (r == 0) end_t = u;
-          else nqk = u + 1;
+        for (int u = 0; u < 2 && u < t_count && ok; ++u) {
+          ok = issue_qk(u);
+          if (ok) nqk = u + 1;
         }
-        for (int t = 0; ok && t < end_t; ++t) {
-          // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2)
-          // (its S buffer is free once the softmax has taken S(t)).
-          ok = mbar_wait(bar(BAR_PFULL + t % 2), (t / 2) & 1, abort) &&
+        for (int t = 0; ok && t < t_count; ++t) {
+          // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
+          ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
                mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort) &&
                mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
           if (!ok) break;
           tc_fence_after();
           const uint64_t so = (uint64_t)((t % VS) * kKVBytes) >> 4;
-          const uint64_t pb = (uint64_t)((t % 2) * C::kPBytes) >> 4;
+          const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
           const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
 #pragma unroll
           for (int k = 0; k < kTileKeys / 16; ++k) {
@@ -645,11 +668,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(BAR_OFULL + t % 2));
           tc_commit(bar(BAR_VEMPTY + t % VS));
           npv = t + 1;
-          if (t + 2 < end_t) {
-            const int r = issue_qk(t + 2);
-            if (r < 0) ok = false;
-            else if (r == 0) end_t = t + 2;
-            else nqk = t + 3;
+          if (t + 2 < t_count) {
+            ok = issue_qk(t + 2);
+            if (ok) nqk = t + 3;
           }
         }
         misc->k_consumed = nqk;
@@ -703,29 +724,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // row sees a key.  bias[r] = kPShift - cs * (row r's reference max).
       float m_lane = -INFINITY;
       bool ok = true;
-      int end_t = 0x7fffffff;  // number of tiles, once published
+      const int end_t = t_count;  // tiles of this CTA (local t -> tile t_first + t)
 
       // Iteration t scores tile t and folds tile t-2's O^T (finished long
       // ago) into the register accumulators; the two iterations after the
       // last tile only fold.  Tile u's rescale factors live in alpha_s[u % 4].
-      // Waiting for O(t-2) also frees P buffer t % 2 (PV(t-2) read it).
+      // S(t) in TMEM implies O(t-2) (the issuer commits S(t) after issuing
+      // PV(t-2)), so one wait per tile suffices; the fold-only iterations
+      // wait for O itself.  With two P buffers, O(t-2) done also frees P
+      // buffer t % 2 (PV(t-2) read it).
       for (int t = 0;; ++t) {
-        int gt = -1;  // tile number of local tile t
-        if (t < end_t) {
-          ok = __all_sync(0xffffffffu,
-                          ok && mbar_wait(bar(BAR_INFO + t % kInfoSlots),
-                                          (t / kInfoSlots) & 1, abort));
-          gt = ok ? info[t % kInfoSlots].tile : -1;
-          if (gt < 0) end_t = t;
-        }
         if (t - 2 >= end_t) break;  // the last tile (end_t - 1) was folded at end_t + 1
         const bool has_s = t < end_t, has_o = t >= 2;
+        const int gt = t_first + t;  // tile number of local tile t (when has_s)
         const int sb = t % 2, st = t % VS, ob = t % 2;  // O of tile t-2 sits in buffer t%2
-        if (has_o)
-          ok = __all_sync(0xffffffffu,
-                          ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
         if (has_s)
           ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+        else if (has_o)
+          ok = __all_sync(0xffffffffu,
+                          ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
         float sv[RW], oh[RW], ol[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) sv[r] = oh[r] = ol[r] = 0.f;
@@ -750,11 +767,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float x[RW];           // cs * s + bias: log2 of the scaled weight
         bool exceed = false;
         if (has_s) {
-          // Which rows see this key?  Keys of chunks that were not loaded
-          // (outside the visible range or an out-of-range block) see none.
+          // Which rows see this key?  Chunks that were not loaded lie wholly
+          // outside [lo_u, hi_u], so their keys see none.
           const int key = base + gt * kTileKeys + j;
-          if (ok && ((info[t % kInfoSlots].mask >> (j / kChunk)) & 1u) && key >= lo_u &&
-              key <= hi_u) {
+          if (ok && key >= lo_u && key <= hi_u) {
             if (key >= lo_all && key <= hi_all) {
               rmask = all_rows;
             } else {
@@ -764,13 +780,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           all_vis = __all_sync(0xffffffffu, rmask == all_rows);
-          const uint32_t rm = rmask >> row0;
+          // x = -inf for a row that does not see this key: its weight is
+          // exactly 0 and it cannot raise the row's reference.
+          float xmax = -INFINITY;
+          if (all_vis) {  // interior tiles: every row sees every key
 #pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            x[r] = fmaf(sv[r], cs, bias[r]);
-            const bool vis = all_vis || ((rm >> r) & 1u);
-            exceed |= vis && x[r] > (float)kPShift + kLazy;
+            for (int r = 0; r < RW; ++r) {
+              x[r] = fmaf(sv[r], cs, bias[r]);
+              xmax = fmaxf(xmax, x[r]);
+            }
+          } else {
+            const uint32_t rm = rmask >> row0;
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+              x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
+              xmax = fmaxf(xmax, x[r]);
+            }
           }
+          exceed = xmax > (float)kPShift + kLazy;
         }
         // Reconverge before the group barrier: a warp that arrives diverged
         // (after lane-predicated code) makes the barrier several times slower
@@ -780,20 +807,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // and tells every thread whether any score passed its row's reference.
         const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
         if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
-          const float* al = alpha_s + ((t - 2) % 4) * 32 + row0;
+          const float4* al = reinterpret_cast<const float4*>(alpha_s + ((t - 2) % 4) * 32 + row0);
 #pragma unroll
-          for (int r = 0; r < RW; ++r) acc[r] = fmaf(acc[r], al[r], oh[r] + ol[r]);
+          for (int r = 0; r < RW; r += 4) {
+            const float4 a = al[r / 4];
+            acc[r] = fmaf(acc[r], a.x, oh[r] + ol[r]);
+            acc[r + 1] = fmaf(acc[r + 1], a.y, oh[r + 1] + ol[r + 1]);
+            acc[r + 2] = fmaf(acc[r + 2], a.z, oh[r + 2] + ol[r + 2]);
+            acc[r + 3] = fmaf(acc[r + 3], a.w, oh[r + 3] + ol[r + 3]);
+          }
         }
         if (has_s) {
-          const uint32_t rm = rmask >> row0;
           float alpha = 1.f;
           if (rescale) {
             // New reference max per row: warp transpose-reduction, then
             // across the group's four warps.
+            const uint32_t rm = all_vis ? 0xffffffffu : (rmask >> row0);
             float tmp[RW];
 #pragma unroll
-            for (int r = 0; r < RW; ++r)
-              tmp[r] = (all_vis || ((rm >> r) & 1u)) ? sv[r] : -INFINITY;
+            for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
             const float wmax = warp_row_reduce<RW, true>(tmp, lane);
             if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
             __syncwarp();
@@ -825,33 +857,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 #pragma unroll
             for (int r = 0; r < RW; ++r) {
-              x[r] = fmaf(sv[r], cs, bias[r]);
+              x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
               lpart[r] *= av[r];
             }
           }
           if (widx == 0 && lane < RW) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
 
-          // Scaled weights, split into an fp16 high part and an fp16 residual.
+          // Scaled weights (2^-inf = 0 for keys a row does not see), split
+          // into an fp16 high part (the weight truncated to 11 significant
+          // bits: exact in fp16 over the weights' range) and an fp16 residual.
           uint32_t phi[RW / 2], plo[RW / 2];
 #pragma unroll
           for (int r = 0; r < RW; r += 2) {
-            float pr[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const bool vis = all_vis || ((rm >> (r + e)) & 1u);
-              pr[e] = vis ? fast_exp2(x[r + e]) : 0.f;
-              lpart[r + e] += pr[e];
-            }
-            const __half2 h = __floats2half2_rn(pr[0], pr[1]);
-            const float2 hf = __half22float2(h);
-            const __half2 l2 = __floats2half2_rn(pr[0] - hf.x, pr[1] - hf.y);
+            const float p0 = fast_exp2(x[r]), p1 = fast_exp2(x[r + 1]);
+            lpart[r] += p0;
+            lpart[r + 1] += p1;
+            const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+            const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+            const __half2 h = __floats2half2_rn(h0, h1);
+            const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
             phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
             plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
           }
 
           // A key no row can see must not reach the PV product: zero its V
           // row (after its V tile has landed).
-          if (g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
+          if (g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
             ok = __all_sync(0xffffffffu,
                             ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
             if (ok && rmask == 0) {
@@ -864,11 +895,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
+          if (PB == 1 && t >= 1)  // the single P buffer: PV(t-1) must have read it
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL + (t - 1) % 2),
+                                                         ((t - 1) / 2) & 1, abort));
           if (ok) {
             // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
             // [row'%8] with row' < NR the high parts and row' >= NR the
-            // residuals, in P buffer t % 2.
-            const uint32_t pbuf = sP + (t % 2) * C::kPBytes;
+            // residuals, in P buffer t % PB.
+            const uint32_t pbuf = sP + (t % PB) * C::kPBytes;
             const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
             constexpr uint32_t lo_off = (NR / 8) * 128;
             if constexpr (RW >= 8) {
@@ -888,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
           }
           __syncwarp();
-          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % 2));
+          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % PB));
         }
       }
 
@@ -897,24 +931,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane < RW) lsum[widx * 32 + lane] = wl;
       __syncwarp();
       named_bar_sync(bar_id, kSoftmaxThreads);
+      __syncthreads();  // (A): also makes the K producer's bad-block mark visible
       const bool aborted = *abort != 0;
+      const bool bad = misc->bad != 0;
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         if (row0 + r < R) {
           const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
           const long long pr = part_base + row_index(row0 + r);
-          p.part_out[pr * kHeadDim + j] = (!aborted && l > 0.f) ? acc[r] / l : 0.f;
+          p.part_out[pr * kHeadDim + j] = (!aborted && !bad && l > 0.f) ? acc[r] / l : 0.f;
         }
       }
       if (widx == 0 && lane < RW && row0 + lane < R) {
         // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
+        // NaN marks a partial that read a stand-in for an out-of-range block.
         const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
         p.part_lse[part_base + row_index(row0 + lane)] =
-            (!aborted && l > 0.f)
+            bad ? __int_as_float(0x7fc00000)
+            : (!aborted && l > 0.f)
                 ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
                 : -INFINITY;
       }
-      __syncthreads();  // (A)
     }
     // ---- tear-down (every thread passed (A)) ---------------------------------
     if (threadIdx.x == 32 && misc->abort) atomicOr(p.flags, kFlagTimeout);

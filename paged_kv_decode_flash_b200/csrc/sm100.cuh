@@ -81,18 +81,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 // Wait for the phase with the given parity to complete.  Returns false
 // (and sets *abort) once the time limit passes, or if another role already
-// gave up (*abort set): the caller then stops issuing work.
+// gave up (*abort set): the caller then stops issuing work.  Between checks
+// the thread is suspended in try_wait (woken when the phase completes)
+// instead of spinning, so that waiting warps leave their issue slots to the
+// warps that compute.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_ns(bar, parity, 20000)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      return false;
     }
   }
 }
