@@ -48,6 +48,17 @@ WORKLOAD_TEXT = {
 }
 
 
+OTHER_CONFIGS = ("tiny", "sliding_window", "mixed_q8_0")
+CONFIG_TEXT = {
+    "tiny": "tiny decode: B=1, 1 query token, Hq/Hkv=8/2, L=1024, block_size 16, fp16, "
+            "64 of 128 pool blocks (latency-bound: the whole KV is 1 MB)",
+    "sliding_window": "sliding-window drafter: B=1, 8 non-causal query tokens, window 2048 "
+                      "of L=24576, Hq/Hkv=32/8, fp16; blocks outside the window hold NaN",
+    "mixed_q8_0": "mixed batch: B=8, 4 causal query tokens, L_s ~ U[4096, 65536], "
+                  "Hq/Hkv=32/8, q8_0 cache (int8 + fp16 scale per 32)",
+}
+
+
 def env_int(name, default):
     try:
         return int(os.environ.get(name, default))
@@ -263,6 +274,13 @@ def bench_ours(args, rank, world, dist):
     prim = measure(primary, args.steps, args.warmup, with_e2e=True)
     sec = measure(secondary, max(1, args.steps // 2), args.warmup, with_e2e=False) \
         if not args.primary_only else None
+    # The parity-test configurations, timed the same way (reported, not the
+    # headline): tiny decode, sliding window, mixed batch over a q8_0 cache.
+    others = {}
+    if not args.primary_only:
+        for name in OTHER_CONFIGS:
+            r = measure(name, max(3, min(args.steps // 10, 200)), args.warmup, with_e2e=False)
+            others[name] = r
 
     peak, peak_kind = measured_peaks()
     kv = prim["kv_bytes"]
@@ -322,6 +340,19 @@ def bench_ours(args, rank, world, dist):
             "kv_bytes_per_step": kv2, "num_splits": sec["splits"],
             "traffic": recorded_traffic(secondary),
         }
+    if others:
+        line["configs"] = {}
+        for name, r in others.items():
+            kvb = r["kv_bytes"]
+            gbs = kvb / (r["ms_per_step"] * 1e-3) / 1e9
+            line["configs"][name] = {
+                "workload": CONFIG_TEXT[name], "kv_bytes_per_step": kvb,
+                "us_per_call": round(r["ms_per_step"] * 1e3, 2), "GB/s": round(gbs, 1),
+                "roofline_frac": round(gbs / peak, 4), "num_splits": r["splits"],
+                "launches_per_call": r["launches"],
+                "per_call_us": {"median": round(r["us_median"], 2), "min": round(r["us_min"], 2)},
+                "l2": f"{r['copies']} KV pool copies rotated",
+            }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(prim["case"], budget_s=args.cpu_seconds)
     return line

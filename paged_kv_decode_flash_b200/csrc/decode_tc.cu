@@ -75,10 +75,9 @@ constexpr uint32_t kAtomBytes = 1024;              // 8 keys x 128 bytes
 constexpr uint32_t kGroupBytes = 2 * kAtomBytes;   // both halves of 8 keys
 constexpr uint32_t kKVBytes = kTileKeys / 8 * kGroupBytes;  // one K (or V) tile
 constexpr uint32_t kChunkBytes = kChunk * 256;     // one 16-key chunk (TMA box)
-constexpr int kGroups = 2;                     // softmax warpgroups (split the rows)
-constexpr int kSoftmaxThreads = 128;           // per warpgroup
-constexpr int kVWarp = 2 + kGroups * 4;        // the V producer's warp
-constexpr int kThreads = 32 * (kVWarp + 1);
+constexpr int kSoftmaxThreads = 128;           // per softmax warpgroup
+constexpr uint32_t kBarSetup = 1;              // named barrier: set-up done
+constexpr uint32_t kBarGroup0 = 2;             // named barriers 2.. : softmax groups
 constexpr int kPShift = 14;                    // weights scaled by 2^14 before fp16
 // A row's reference max is only raised when a score passes it by more than
 // kLazy (log2 units); scaled weights then stay below 2^(kPShift + kLazy),
@@ -101,14 +100,19 @@ enum : int {
 };
 constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
-// RW query rows per softmax warpgroup; NR = the MMA's N for S (>= 16).
+// NG softmax warpgroups of RW query rows each; NR = the MMA's N for S
+// (>= 16).  Warps: 0 K producer, 1 MMA issuer, 2 .. 4*NG+1 softmax, then the
+// V producer.
 // KS / VS slots in the K / V rings, PB buffers for P (two, so that the
 // softmax of tile t+1 never waits for PV(t)).  At 32 rows the two P buffers
 // take 32 KB and the V ring keeps two slots (measured: three V slots with
 // one P buffer is slower).  With one P buffer the softmax of tile t waits
 // for PV(t-1) before it stores P(t).
-template <int RW>
+template <int RW, int NG>
 struct Cfg {
+  static constexpr int kGroups = NG;
+  static constexpr int kVWarp = 2 + NG * 4;  // the V producer's warp
+  static constexpr int kThreads = 32 * (kVWarp + 1);
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
   static constexpr int KS = 3;
   static constexpr int VS = NR > 16 ? 2 : 3;
@@ -123,9 +127,9 @@ struct Cfg {
   static constexpr uint32_t kP = kQ + 2 * kQHalf;
   static constexpr uint32_t kPBytes = kTileKeys * 2 * NR * 2;
   static constexpr uint32_t kRed = kP + PB * kPBytes;               // float [2 grp][2][4][32]
-  static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4][32]
+  static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4 tiles][32 rows]
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
-  static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [8 warps][2][32]
+  static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [4*NG warps][2][32]
   static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [32]
   static constexpr uint32_t kInfo = kBars + 32 * 8;                 // TileInfo [8]
   static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
@@ -203,13 +207,14 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
 // asynchronous copies, as many splits per round as fit, all of a round in
 // flight at once, so that the merge costs a few memory latencies rather than
 // one per split.
-template <int RW>
+template <int RW, int NG>
 __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, uint8_t* smem,
                                             uint32_t sbase) {
-  using C = Cfg<RW>;
+  using C = Cfg<RW, NG>;
+  constexpr int kThreads = C::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;  // float4 per partial row
   constexpr int kWarps = kThreads / 32;
-  constexpr int kPairsMax = (2 * RW * kRowF4 + kThreads - 1) / kThreads;
+  constexpr int kPairsMax = (NG * RW * kRowF4 + kThreads - 1) / kThreads;  // rows <= NG * RW
   const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
   const long long rps = (long long)p.n_query * Hq;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -316,9 +321,10 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
 // Same arithmetic as merge_group (log-sum-exp weights, splits added in index
 // order), spread over all S CTAs of the group so that each stages only a
 // few kilobytes of partials with one round of 16-byte asynchronous copies.
-template <int RW>
+template <int RW, int NG>
 __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split,
                                             uint8_t* smem, uint32_t sbase) {
+  constexpr int kThreads = Cfg<RW, NG>::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;
   constexpr int kWarps = kThreads / 32;
   const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
@@ -389,11 +395,12 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   }
 }
 
-template <int RW>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int RW, int NG>
+__global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using C = Cfg<RW>;
+  using C = Cfg<RW, NG>;
+  constexpr int kThreads = C::kThreads, kGroups = NG, kVWarp = C::kVWarp;
   constexpr int NR = C::NR, KS = C::KS, VS = C::VS, PB = C::PB;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the __shared__ array by pointer
@@ -469,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     // The other roles wait for these barriers; this warp starts loading now.
-    named_bar_arrive(3, kThreads);
+    named_bar_arrive(kBarSetup, kThreads);
 
     // Lane c < 8 owns chunk c of every tile.  Its block-table entry for tile
     // t + 1 is read right after tile t's copy is issued and used one slot
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    named_bar_sync(3, kThreads);  // barriers initialised, TMEM allocated, Q staged
+    named_bar_sync(kBarSetup, kThreads);  // barriers initialised, TMEM allocated, Q staged
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
 
@@ -694,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* alpha_s = reinterpret_cast<float*>(smem + C::kAlpha);             // [4][32]
       float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
       float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
-      const uint32_t bar_id = 1 + g;
+      const uint32_t bar_id = kBarGroup0 + g;
       const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
 
       // Per query token, the visible key range; keys inside every token's
@@ -990,7 +997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     __threadfence();
     if (misc->last) {
-      merge_slice<RW>(p, s, kvh, split, smem, sbase);
+      merge_slice<RW, NG>(p, s, kvh, split, smem, sbase);
     } else if (threadIdx.x == 0) {
       atomicOr(p.flags, kFlagTimeout);
     }
@@ -1008,7 +1015,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (!misc->last) return;
   __threadfence();  // the other CTAs' partials, published before their counts
-  merge_group<RW>(p, s, kvh, smem, sbase);
+  merge_group<RW, NG>(p, s, kvh, smem, sbase);
   if (threadIdx.x == 0) *cnt = 0;
 }
 
@@ -1043,20 +1050,20 @@ bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int RW>
+template <int RW, int NG>
 cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& mv,
                       cudaStream_t stream) {
-  const size_t smem = Cfg<RW>::kTotal + 1024;
+  const size_t smem = Cfg<RW, NG>::kTotal + 1024;
   static int resident[64] = {};  // CTAs of this kernel the device holds at once (0: unknown)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || resident[dev] == 0) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<RW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_tc_kernel<RW, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW>, kThreads,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW, NG>, Cfg<RW, NG>::kThreads,
                                                       smem);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1069,7 +1076,7 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   p.coop = (dev >= 0 && dev < 64 && ctas <= resident[dev]) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.num_splits, p.num_kv_heads, p.num_seqs);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Cfg<RW, NG>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1077,7 +1084,7 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.coop ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW>, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW, NG>, mk, mv, p);
 }
 
 }  // namespace
@@ -1092,9 +1099,11 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream) {
   const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
   if (!encode_cache_map(&mk, p.k, rows) || !encode_cache_map(&mv, p.v, rows))
     return cudaErrorInvalidValue;
-  if (p.rows <= 8) return launch_rw<4>(p, mk, mv, stream);
-  if (p.rows <= 16) return launch_rw<8>(p, mk, mv, stream);
-  return launch_rw<16>(p, mk, mv, stream);
+  // Two softmax warpgroups (measured: four groups of 8 rows at 32 rows are
+  // slower than two of 16).
+  if (p.rows <= 8) return launch_rw<4, 2>(p, mk, mv, stream);
+  if (p.rows <= 16) return launch_rw<8, 2>(p, mk, mv, stream);
+  return launch_rw<16, 2>(p, mk, mv, stream);
 }
 
 }  // namespace pa
