@@ -53,6 +53,7 @@
 #include <cuda_runtime.h>
 
 #include <cstddef>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -75,6 +76,12 @@ constexpr uint32_t kAtomBytes = 1024;              // 8 keys x 128 bytes
 constexpr uint32_t kGroupBytes = 2 * kAtomBytes;   // both halves of 8 keys
 constexpr uint32_t kKVBytes = kTileKeys / 8 * kGroupBytes;  // one K (or V) tile
 constexpr uint32_t kChunkBytes = kChunk * 256;     // one 16-key chunk (TMA box)
+// q8_0: a raw 128-key tile in shared memory is qs [128 keys][128 int8] then
+// d [128 keys][4 fp16]; a 16-key chunk arrives as two bulk copies (2048 B of
+// qs, 128 B of scales).
+constexpr uint32_t kRawQsBytes = kTileKeys * kHeadDim;              // 16 KB
+constexpr uint32_t kRawBytes = kRawQsBytes + kTileKeys * 8;         // 17 KB
+constexpr uint32_t kQ8ChunkBytes = kChunk * (kHeadDim + 8);         // 2176 B
 constexpr int kSoftmaxThreads = 128;           // per softmax warpgroup
 constexpr uint32_t kBarSetup = 1;              // named barrier: set-up done
 constexpr uint32_t kBarGroup0 = 2;             // named barriers 2.. : softmax groups
@@ -96,8 +103,13 @@ enum : int {
   BAR_OEMPTY = 20,  // [2] O^T read by the softmax warps
   BAR_DONE = 22,    // every MMA finished
   BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
-  BAR_COUNT = 31
+  BAR_CKFULL = 31,  // q8_0: converted K tile written
+  BAR_CKEMPTY = 32, // q8_0: converted K tile read by QK^T
+  BAR_CVFULL = 33,  // q8_0: converted V tile written
+  BAR_CVEMPTY = 34, // q8_0: converted V tile read by PV
+  BAR_COUNT = 35
 };
+constexpr int kBarSlots = 40;
 constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
 // NG softmax warpgroups of RW query rows each; NR = the MMA's N for S
@@ -108,18 +120,25 @@ constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 // take 32 KB and the V ring keeps two slots (measured: three V slots with
 // one P buffer is slower).  With one P buffer the softmax of tile t waits
 // for PV(t-1) before it stores P(t).
-template <int RW, int NG>
+template <int RW, int NG, bool Q8>
 struct Cfg {
   static constexpr int kGroups = NG;
-  static constexpr int kVWarp = 2 + NG * 4;  // the V producer's warp
-  static constexpr int kThreads = 32 * (kVWarp + 1);
+  static constexpr int kVWarp = 2 + NG * 4;      // the V producer's warp
+  static constexpr int kConvWarp = kVWarp + 1;   // q8_0: first of 4 converter warps
+  static constexpr int kThreads = 32 * (kVWarp + 1 + (Q8 ? 4 : 0));
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
-  static constexpr int KS = 3;
-  static constexpr int VS = NR > 16 ? 2 : 3;
+  // fp16: K/V rings of TMA-loaded tiles.  q8_0: rings of raw tiles (2 slots
+  // of kRawBytes) plus one converted K and one converted V tile, each an
+  // fp16 high part and an fp16 residual (2 * kKVBytes).
+  static constexpr int KS = Q8 ? 2 : 3;
+  static constexpr int VS = Q8 ? 2 : (NR > 16 ? 2 : 3);
   static constexpr int PB = 2;
+  static constexpr uint32_t kSlotBytes = Q8 ? kRawBytes : kKVBytes;
   static constexpr uint32_t kK = 0;                                 // K ring
-  static constexpr uint32_t kV = KS * kKVBytes;                     // V ring
-  static constexpr uint32_t kQ = (KS + VS) * kKVBytes;
+  static constexpr uint32_t kV = KS * kSlotBytes;                   // V ring
+  static constexpr uint32_t kConvK = (KS + VS) * kSlotBytes;        // q8_0: K hi | K lo
+  static constexpr uint32_t kConvV = kConvK + (Q8 ? 2 * kKVBytes : 0);  // q8_0: V hi | V lo
+  static constexpr uint32_t kQ = kConvV + (Q8 ? 2 * kKVBytes : 0);
   static constexpr uint32_t kQHalf = NR * 128;
   // P^T of one tile: 2*NR "rows" (the fp16 high parts of the NR query rows,
   // then their residuals), so one MMA with N = 2*NR multiplies both.  Tile t
@@ -130,8 +149,8 @@ struct Cfg {
   static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4 tiles][32 rows]
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
   static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [4*NG warps][2][32]
-  static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [32]
-  static constexpr uint32_t kInfo = kBars + 32 * 8;                 // TileInfo [8]
+  static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [kBarSlots]
+  static constexpr uint32_t kInfo = kBars + kBarSlots * 8;          // TileInfo [8]
   static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
   static constexpr uint32_t kTotal = kMisc + 64;
   // TMEM columns: S^T[2] (NR each) then O^T[2] (2*NR each: high | residual).
@@ -140,6 +159,7 @@ struct Cfg {
                                         : kTmemUsed <= 128 ? 128 : 256;
   static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
   static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
+  static_assert(kConvK % 1024 == 0, "converted tiles sit on 1 KB swizzle atoms");
 };
 
 struct Misc {
@@ -177,6 +197,30 @@ __device__ __forceinline__ void sts_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
+// q8_0 cache: byte offset of the qs rows of the 16-key chunk that starts at
+// key key0 of (block, head) tile `tile` (tiles are block_size * (128 + 8)
+// bytes: qs [block_size][128] then fp16 d [block_size][4]).
+__device__ __forceinline__ long long q8_chunk_offset(const DecodeParams& p, int tile, int key0) {
+  return (long long)tile * p.block_size * (kHeadDim + 8) + (long long)(key0 % p.block_size) * kHeadDim;
+}
+// ... and from there to the chunk's scales.
+__device__ __forceinline__ long long q8_scale_offset(const DecodeParams& p, int key0) {
+  const int slot = key0 % p.block_size;
+  return (long long)(p.block_size - slot) * kHeadDim + slot * 8;
+}
+
+// Eight signed bytes -> eight exact floats: byte b becomes the low mantissa
+// byte of 2^23 + (b + 128) (a float whose value is that integer), minus
+// 2^23 + 128.
+__device__ __forceinline__ void q8_to_float8(uint2 q, float (&x)[8]) {
+  const uint32_t w0 = q.x ^ 0x80808080u, w1 = q.y ^ 0x80808080u;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    x[e] = __uint_as_float(__byte_perm(w0, 0x4B00u, 0x5440u | e)) - 8388736.f;
+    x[4 + e] = __uint_as_float(__byte_perm(w1, 0x4B00u, 0x5440u | e)) - 8388736.f;
+  }
+}
+
 // Warp transpose-reduction over the 32 lanes (= 32 keys): lane l ends with
 // the reduction of row (l % RW) in the return value.
 template <int RW, bool kMax>
@@ -207,10 +251,10 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
 // asynchronous copies, as many splits per round as fit, all of a round in
 // flight at once, so that the merge costs a few memory latencies rather than
 // one per split.
-template <int RW, int NG>
+template <int RW, int NG, bool Q8>
 __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, uint8_t* smem,
                                             uint32_t sbase) {
-  using C = Cfg<RW, NG>;
+  using C = Cfg<RW, NG, Q8>;
   constexpr int kThreads = C::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;  // float4 per partial row
   constexpr int kWarps = kThreads / 32;
@@ -321,10 +365,10 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
 // Same arithmetic as merge_group (log-sum-exp weights, splits added in index
 // order), spread over all S CTAs of the group so that each stages only a
 // few kilobytes of partials with one round of 16-byte asynchronous copies.
-template <int RW, int NG>
+template <int RW, int NG, bool Q8>
 __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split,
                                             uint8_t* smem, uint32_t sbase) {
-  constexpr int kThreads = Cfg<RW, NG>::kThreads;
+  constexpr int kThreads = Cfg<RW, NG, Q8>::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;
   constexpr int kWarps = kThreads / 32;
   const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
@@ -395,11 +439,11 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   }
 }
 
-template <int RW, int NG>
-__global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
+template <int RW, int NG, bool Q8>
+__global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using C = Cfg<RW, NG>;
+  using C = Cfg<RW, NG, Q8>;
   constexpr int kThreads = C::kThreads, kGroups = NG, kVWarp = C::kVWarp;
   constexpr int NR = C::NR, KS = C::KS, VS = C::VS, PB = C::PB;
   extern __shared__ uint8_t smem_raw[];
@@ -454,11 +498,18 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
   } else if (warp == 0) {
     // ======================= K producer (also sets up the barriers) ========
     if (lane == 0) {
+      // q8_0: the raw K (V) slots are released by the 2 K (V) converter warps.
       for (int i = 0; i < kMaxStages; ++i) {
         mbar_init(bar(BAR_KFULL + i), 1);
-        mbar_init(bar(BAR_KEMPTY + i), 1);
+        mbar_init(bar(BAR_KEMPTY + i), Q8 ? 2 : 1);
         mbar_init(bar(BAR_VFULL + i), 1);
-        mbar_init(bar(BAR_VEMPTY + i), 1);
+        mbar_init(bar(BAR_VEMPTY + i), Q8 ? 2 : 1);
+      }
+      if (Q8) {
+        mbar_init(bar(BAR_CKFULL), 2);
+        mbar_init(bar(BAR_CKEMPTY), 1);
+        mbar_init(bar(BAR_CVFULL), 2);
+        mbar_init(bar(BAR_CVEMPTY), 1);
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(bar(BAR_SFULL + i), 1);
@@ -505,6 +556,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
         misc->bad = 1;
         return 0;
       }
+      if (Q8) return (int)(phys * p.num_kv_heads + kvh);  // q8_0: the (block, head) tile
       const int key0 = base + tile_of(t) * kTileKeys + c * kChunk;
       return (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
     };
@@ -532,11 +584,22 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       const uint32_t fb = bar(BAR_KFULL + st);
-      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
+      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8ChunkBytes : kChunkBytes));
       __syncwarp();
       if (w_cur) {
-        tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
-        tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+        if constexpr (Q8) {
+          const long long off = q8_chunk_offset(p, row_cur, base + g_cur * kTileKeys + c * kChunk);
+          const uint32_t dst = sKr + st * kRawBytes;
+          const uint8_t* src = static_cast<const uint8_t*>(p.k);
+          bulk_load(dst + c * kChunk * kHeadDim, src + off, kChunk * kHeadDim, fb);
+          bulk_load(dst + kRawQsBytes + c * kChunk * 8,
+                    src + off + q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk), kChunk * 8,
+                    fb);
+          bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off, kChunk * kHeadDim);
+        } else {
+          tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
+          tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+        }
       }
       __syncwarp();
       issued = t + 1;
@@ -597,16 +660,27 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
         const TileInfo& ti = info[t % kInfoSlots];
         if (ti.tile < 0) break;
         const uint32_t mask = ti.mask;
-        const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;
+        const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;  // q8_0: the tile index
         const int st = t % VS;
         if (lane == 0) ok = mbar_wait(bar(BAR_VEMPTY + st), ((t / VS) & 1) ^ 1, abort);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const uint32_t fb = bar(BAR_VFULL + st);
-        if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * kChunkBytes);
+        if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8ChunkBytes : kChunkBytes));
         __syncwarp();
-        if (c < kChunksPerTile && ((mask >> c) & 1u))
-          tma_load_4d(sVr + st * kKVBytes + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
+        if (c < kChunksPerTile && ((mask >> c) & 1u)) {
+          if constexpr (Q8) {
+            const long long off = q8_chunk_offset(p, row8, base + ti.tile * kTileKeys + c * kChunk);
+            const uint32_t dst = sVr + st * kRawBytes;
+            const uint8_t* src = static_cast<const uint8_t*>(p.v);
+            bulk_load(dst + c * kChunk * kHeadDim, src + off, kChunk * kHeadDim, fb);
+            bulk_load(dst + kRawQsBytes + c * kChunk * 8,
+                      src + off + q8_scale_offset(p, base + ti.tile * kTileKeys + c * kChunk),
+                      kChunk * 8, fb);
+          } else {
+            tma_load_4d(sVr + st * kKVBytes + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
+          }
+        }
         __syncwarp();
         issued = t + 1;
       }
@@ -628,26 +702,36 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
         const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
         // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
         // start-address field is the low 14 bits, addresses stay < 256 KB).
-        const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
+        // q8_0: K and V are the converted tiles (fp16 high part, then the
+        // fp16 residual kKVBytes further), each multiplied and accumulated in
+        // turn into the same TMEM accumulator.
+        const uint64_t dK = smem_desc(Q8 ? sbase + C::kConvK : sKr, 16, kGroupBytes, kSwizzle128B);
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
-        const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
+        const uint64_t dV =
+            smem_desc(Q8 ? sbase + C::kConvV : sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
         const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
-        // QK(u) once K(u) landed and the softmax took S(u-2) from its buffer.
+        constexpr int kParts = Q8 ? 2 : 1;  // operand parts per product (high, residual)
+        // QK(u) once K(u) is ready and the softmax took S(u-2) from its buffer.
         auto issue_qk = [&](int u) -> bool {
-          if (!(mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, abort) &&
-                mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
+          const bool ready = Q8 ? mbar_wait(bar(BAR_CKFULL), u & 1, abort)
+                                : mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, abort);
+          if (!(ready && mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
             return false;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((u % KS) * kKVBytes) >> 4;
+          const uint64_t so = Q8 ? 0 : (uint64_t)((u % KS) * kKVBytes) >> 4;
           const uint32_t d = tmem + (u % 2) * NR;
 #pragma unroll
-          for (int k = 0; k < kHeadDim / 16; ++k) {
-            const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
-            const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
-            tc_mma_f16_ss(d, dK + so + ko, dQ + qo, id_qk, k > 0);
+          for (int part = 0; part < kParts; ++part) {
+            const uint64_t po = (uint64_t)(part * kKVBytes) >> 4;
+#pragma unroll
+            for (int k = 0; k < kHeadDim / 16; ++k) {
+              const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
+              const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
+              tc_mma_f16_ss(d, dK + so + po + ko, dQ + qo, id_qk, part > 0 || k > 0);
+            }
           }
           tc_commit(bar(BAR_SFULL + u % 2));
-          tc_commit(bar(BAR_KEMPTY + u % KS));
+          tc_commit(bar(Q8 ? BAR_CKEMPTY : BAR_KEMPTY + u % KS));
           return true;
         };
         int nqk = 0, npv = 0;
@@ -659,34 +743,126 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
         for (int t = 0; ok && t < t_count; ++t) {
           // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
           ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
-               mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort) &&
+               (Q8 ? mbar_wait(bar(BAR_CVFULL), t & 1, abort)
+                   : mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort)) &&
                mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((t % VS) * kKVBytes) >> 4;
+          const uint64_t so = Q8 ? 0 : (uint64_t)((t % VS) * kKVBytes) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
           const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
 #pragma unroll
-          for (int k = 0; k < kTileKeys / 16; ++k) {
-            const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
-            const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
-            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, k > 0);
+          for (int part = 0; part < kParts; ++part) {
+            const uint64_t pt = (uint64_t)(part * kKVBytes) >> 4;
+#pragma unroll
+            for (int k = 0; k < kTileKeys / 16; ++k) {
+              const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
+              const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
+              tc_mma_f16_ss(d, dV + so + pt + vo, dP + pb + po, id_pv, part > 0 || k > 0);
+            }
           }
           tc_commit(bar(BAR_OFULL + t % 2));
-          tc_commit(bar(BAR_VEMPTY + t % VS));
+          tc_commit(bar(Q8 ? BAR_CVEMPTY : BAR_VEMPTY + t % VS));
           npv = t + 1;
           if (t + 2 < t_count) {
             ok = issue_qk(t + 2);
             if (ok) nqk = t + 3;
           }
         }
-        misc->k_consumed = nqk;
-        misc->v_consumed = npv;
+        if (!Q8) {  // q8_0: the converter consumes the raw rings
+          misc->k_consumed = nqk;
+          misc->v_consumed = npv;
+        }
         tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
         volatile int no_abort = 0;
         mbar_wait(bar(BAR_DONE), 0, &no_abort);
       }
       __syncwarp();
+      __syncthreads();  // (A)
+    } else if (Q8 && warp >= C::kConvWarp) {
+      // ===================== q8_0 converter (4 warps) ========================
+      // Raw tile t (int8 qs, fp16 scales d per 32 elements) -> the fp16 K and
+      // V operand tiles.  Each element is x = qs * d, exact in fp32 (an 8-bit
+      // integer times an 11-bit significand); the operand holds its high part
+      // (x truncated to 11 significant bits, exact in fp16) and, kKVBytes
+      // further, the fp16 residual x - high, so that the tensor core sees x to
+      // about 2^-22.  Layout as the fp16 TMA boxes: [key/8][half][key%8]
+      // [64 dims], 128-byte swizzle.  V rows of keys outside [lo_u, hi_u]
+      // (masked or never loaded) are written as zeros: they must not reach
+      // the PV product.
+      // Warps kConvWarp, +1 convert K; warps +2, +3 convert V, so that K is
+      // never held up by V waiting for its operand buffer.  Thread = one
+      // 8-element column cc of every other 4th key: with 64 threads per
+      // stream, key r = 8 * group + rr with rr in {r0, r0 + 4}, so that the
+      // swizzled destination offset is constant up to the key group.
+      const int kv = (warp - C::kConvWarp) >> 1;  // 0: K, 1: V
+      const int ct = threadIdx.x - 32 * (C::kConvWarp + 2 * kv);  // 0 .. 63
+      const int cc = ct & 15, r0 = ct >> 4;      // column, first key (0 .. 3)
+      const uint32_t col_off = (cc >> 3) * kAtomBytes;
+      const uint32_t off_a = col_off + r0 * 128 + (((cc & 7) ^ r0) << 4);
+      const uint32_t off_b = col_off + (r0 + 4) * 128 + (((cc & 7) ^ (r0 + 4)) << 4);
+      const int NSl = kv == 0 ? KS : VS;
+      const uint32_t bar_full = kv == 0 ? BAR_KFULL : BAR_VFULL;
+      const uint32_t bar_raw_empty = kv == 0 ? BAR_KEMPTY : BAR_VEMPTY;
+      const uint32_t bar_cfull = kv == 0 ? BAR_CKFULL : BAR_CVFULL;
+      const uint32_t bar_cempty = kv == 0 ? BAR_CKEMPTY : BAR_CVEMPTY;
+      const uint32_t dst = sbase + (kv == 0 ? C::kConvK : C::kConvV);
+      int n = 0;
+      bool ok = true;
+      // One 8-element item: x = qs * d split into an fp16 high part and an
+      // fp16 residual (zeros for a V row no query row may see).
+      auto convert = [&](const uint8_t* raw, int r, uint32_t off, bool live) {
+        uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+        if (live) {
+          const uint2 q = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
+          const float d = __half2float(
+              *reinterpret_cast<const __half*>(raw + kRawQsBytes + r * 8 + (cc >> 2) * 2));
+          float x[8];
+          q8_to_float8(q, x);
+          uint32_t h[4], l[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const float x0 = x[e] * d, x1 = x[e + 1] * d;
+            const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffffe000u);
+            const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffffe000u);
+            const __half2 hh = __floats2half2_rn(h0, h1);
+            const __half2 ll = __floats2half2_rn(x0 - h0, x1 - h1);
+            h[e / 2] = *reinterpret_cast<const uint32_t*>(&hh);
+            l[e / 2] = *reinterpret_cast<const uint32_t*>(&ll);
+          }
+          hi = make_uint4(h[0], h[1], h[2], h[3]);
+          lo = make_uint4(l[0], l[1], l[2], l[3]);
+        }
+        sts_v4(dst + off, hi);
+        sts_v4(dst + kKVBytes + off, lo);
+      };
+      for (int t = 0; t < t_count && ok; ++t) {
+        const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
+        const int rs = t % NSl;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort) &&
+                                         mbar_wait(bar(bar_cempty), (t & 1) ^ 1, abort));
+        if (!ok) break;
+        const uint8_t* raw = smem + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
+#pragma unroll 2
+        for (int grp = 0; grp < kTileKeys / 8; ++grp) {
+          const int ra = grp * 8 + r0, rb = ra + 4;
+          convert(raw, ra, grp * kGroupBytes + off_a,
+                  kv == 0 || (key_t + ra >= lo_u && key_t + ra <= hi_u));
+          convert(raw, rb, grp * kGroupBytes + off_b,
+                  kv == 0 || (key_t + rb >= lo_u && key_t + rb <= hi_u));
+        }
+        fence_proxy_async_smem();  // generic writes -> the tensor core's reads
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(bar_cfull));
+          mbar_arrive(bar(bar_raw_empty + rs));
+        }
+        n = t + 1;
+      }
+      if (ct == 0) {
+        if (kv == 0) misc->k_consumed = n;
+        else misc->v_consumed = n;
+      }
       __syncthreads();  // (A)
     } else {
       // ===================== softmax + correction ============================
@@ -889,7 +1065,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
 
           // A key no row can see must not reach the PV product: zero its V
           // row (after its V tile has landed).
-          if (g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
+          if (!Q8 && g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
             ok = __all_sync(0xffffffffu,
                             ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
             if (ok && rmask == 0) {
@@ -997,7 +1173,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
     __syncthreads();
     __threadfence();
     if (misc->last) {
-      merge_slice<RW, NG>(p, s, kvh, split, smem, sbase);
+      merge_slice<RW, NG, Q8>(p, s, kvh, split, smem, sbase);
     } else if (threadIdx.x == 0) {
       atomicOr(p.flags, kFlagTimeout);
     }
@@ -1015,7 +1191,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG>::kThreads, 1)
   __syncthreads();
   if (!misc->last) return;
   __threadfence();  // the other CTAs' partials, published before their counts
-  merge_group<RW, NG>(p, s, kvh, smem, sbase);
+  merge_group<RW, NG, Q8>(p, s, kvh, smem, sbase);
   if (threadIdx.x == 0) *cnt = 0;
 }
 
@@ -1050,20 +1226,20 @@ bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int RW, int NG>
+template <int RW, int NG, bool Q8>
 cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& mv,
                       cudaStream_t stream) {
-  const size_t smem = Cfg<RW, NG>::kTotal + 1024;
+  const size_t smem = Cfg<RW, NG, Q8>::kTotal + 1024;
   static int resident[64] = {};  // CTAs of this kernel the device holds at once (0: unknown)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || resident[dev] == 0) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<RW, NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_tc_kernel<RW, NG, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW, NG>, Cfg<RW, NG>::kThreads,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW, NG, Q8>, Cfg<RW, NG, Q8>::kThreads,
                                                       smem);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1076,7 +1252,7 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   p.coop = (dev >= 0 && dev < 64 && ctas <= resident[dev]) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.num_splits, p.num_kv_heads, p.num_seqs);
-  cfg.blockDim = dim3(Cfg<RW, NG>::kThreads);
+  cfg.blockDim = dim3(Cfg<RW, NG, Q8>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1084,26 +1260,36 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.coop ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW, NG>, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW, NG, Q8>, mk, mv, p);
 }
 
 }  // namespace
 
 bool decode_tc_supported(int kv_dtype, int rows, int num_blocks, int num_kv_heads, int block_size) {
-  return kv_dtype == kKvFp16 && rows >= 1 && rows <= 2 * 16 &&
+  // fp16: up to 32 rows per KV head; q8_0: up to 16 (the converted K and V
+  // tiles leave no shared memory for the 32-row P buffers).
+  const int max_rows = kv_dtype == kKvFp16 ? 2 * 16 : kv_dtype == kKvQ8_0 ? 16 : 0;
+  return rows >= 1 && rows <= max_rows && block_size % kChunk == 0 &&
          (long long)num_blocks * num_kv_heads * block_size <= INT32_MAX;
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream) {
+  if (p.kv_dtype == kKvQ8_0) {
+    // Raw q8_0 tiles arrive by untiled bulk copies: no tensor maps.
+    CUtensorMap none;
+    memset(&none, 0, sizeof(none));
+    if (p.rows <= 8) return launch_rw<4, 2, true>(p, none, none, stream);
+    return launch_rw<8, 2, true>(p, none, none, stream);
+  }
   CUtensorMap mk, mv;
   const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
   if (!encode_cache_map(&mk, p.k, rows) || !encode_cache_map(&mv, p.v, rows))
     return cudaErrorInvalidValue;
   // Two softmax warpgroups (measured: four groups of 8 rows at 32 rows are
   // slower than two of 16).
-  if (p.rows <= 8) return launch_rw<4, 2>(p, mk, mv, stream);
-  if (p.rows <= 16) return launch_rw<8, 2>(p, mk, mv, stream);
-  return launch_rw<16, 2>(p, mk, mv, stream);
+  if (p.rows <= 8) return launch_rw<4, 2, false>(p, mk, mv, stream);
+  if (p.rows <= 16) return launch_rw<8, 2, false>(p, mk, mv, stream);
+  return launch_rw<16, 2, false>(p, mk, mv, stream);
 }
 
 }  // namespace pa

@@ -172,6 +172,23 @@ __device__ __forceinline__ void tma_prefetch_4d(const void* tmap, int c0, int c1
                : "memory");
 }
 
+// Untiled bulk copy global -> shared (both addresses 16-byte aligned, size a
+// multiple of 16), completion on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Prefetch of a byte range (16-byte aligned, size a multiple of 16) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared, L2 only (generic proxy: no
 // proxy fence is needed against data other threads wrote with plain stores).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
