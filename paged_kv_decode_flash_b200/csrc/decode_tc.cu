@@ -17,15 +17,19 @@
 //               K slots are released as soon as QK^T has read them, so K runs
 //               ahead.  With each K copy the same chunk of V is prefetched
 //               into L2, so that V's own copy a tile later is short.
-//   warps 1, 11 MMA issuers (one thread each): warp 1 S^T = K Q^T with
-//               M = 128 keys and N = the query rows, warp 11 O^T = V^T
-//               [P_hi | P_lo]^T with M = 128 head_dim lanes; accumulators live
-//               in TMEM, P is double-buffered in shared memory so that the
-//               softmax of tile t+1 overlaps the PV product of tile t.
+//   warp 1      MMA issuer (one thread), fixed order QK(0), QK(1), then
+//               PV(t), QK(t+2): S^T = K Q^T with M = 128 keys and N = the
+//               query rows (double-buffered in TMEM), O^T += V^T
+//               [P_hi | P_lo]^T with M = 128 head_dim lanes (one TMEM
+//               accumulator over all tiles); P is double-buffered in shared
+//               memory so that the softmax of tile t+1 overlaps PV(t).
 //   warps 2-9   two softmax warpgroups, each owning half of the query rows:
 //               thread = key for S (row max by a warp transpose-reduction
-//               plus one named barrier per group), thread = head_dim element
-//               for O (running accumulators in registers).
+//               plus one named barrier per group); when a row's reference
+//               maximum rises, its O column is rescaled in TMEM in place
+//               (thread = head_dim lane) before the tile's P is published.
+//   warps 11-14 (q8_0 cache only) converters: raw int8 tiles -> fp16 operand
+//               tiles (see below).
 // Putting keys and head_dim on the MMA's M side keeps the tensor core free of
 // padding even at 4-32 query rows.
 //
@@ -99,8 +103,7 @@ enum : int {
   BAR_SFULL = 12,   // [2] S^T in TMEM
   BAR_SEMPTY = 14,  // [2] S^T read by the softmax warps
   BAR_PFULL = 16,   // [2] P of one tile written to shared memory
-  BAR_OFULL = 18,   // [2] O^T of one tile in TMEM (also: its P buffer is free)
-  BAR_OEMPTY = 20,  // [2] O^T read by the softmax warps
+  BAR_OFULL = 18,   // PV of one more tile accumulated into O^T
   BAR_DONE = 22,    // every MMA finished
   BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
   BAR_CKFULL = 31,  // q8_0: converted K tile written
@@ -153,8 +156,8 @@ struct Cfg {
   static constexpr uint32_t kInfo = kBars + kBarSlots * 8;          // TileInfo [8]
   static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
   static constexpr uint32_t kTotal = kMisc + 64;
-  // TMEM columns: S^T[2] (NR each) then O^T[2] (2*NR each: high | residual).
-  static constexpr uint32_t kTmemUsed = 6 * NR;
+  // TMEM columns: S^T[2] (NR each) then O^T (2*NR: high | residual).
+  static constexpr uint32_t kTmemUsed = 4 * NR;
   static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
                                         : kTmemUsed <= 128 ? 128 : 256;
   static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
@@ -515,9 +518,8 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         mbar_init(bar(BAR_SFULL + i), 1);
         mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
         mbar_init(bar(BAR_PFULL + i), 4 * kGroups);
-        mbar_init(bar(BAR_OFULL + i), 1);
-        mbar_init(bar(BAR_OEMPTY + i), 4 * kGroups);
       }
+      mbar_init(bar(BAR_OFULL), 1);
       mbar_init(bar(BAR_DONE), 1);
       for (int i = 0; i < kInfoSlots; ++i) mbar_init(bar(BAR_INFO + i), 1);
       misc->abort = 0;
@@ -744,13 +746,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
           ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
                (Q8 ? mbar_wait(bar(BAR_CVFULL), t & 1, abort)
-                   : mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort)) &&
-               mbar_wait(bar(BAR_OEMPTY + t % 2), ((t / 2) & 1) ^ 1, abort);
+                   : mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort));
           if (!ok) break;
           tc_fence_after();
           const uint64_t so = Q8 ? 0 : (uint64_t)((t % VS) * kKVBytes) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
-          const uint32_t d = tmem + 2 * NR + (t % 2) * 2 * NR;
+          const uint32_t d = tmem + 2 * NR;  // O^T accumulates over all tiles
 #pragma unroll
           for (int part = 0; part < kParts; ++part) {
             const uint64_t pt = (uint64_t)(part * kKVBytes) >> 4;
@@ -758,10 +759,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             for (int k = 0; k < kTileKeys / 16; ++k) {
               const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
               const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
-              tc_mma_f16_ss(d, dV + so + pt + vo, dP + pb + po, id_pv, part > 0 || k > 0);
+              tc_mma_f16_ss(d, dV + so + pt + vo, dP + pb + po, id_pv, t > 0 || part > 0 || k > 0);
             }
           }
-          tc_commit(bar(BAR_OFULL + t % 2));
+          tc_commit(bar(BAR_OFULL));
           tc_commit(bar(Q8 ? BAR_CVEMPTY : BAR_VEMPTY + t % VS));
           npv = t + 1;
           if (t + 2 < t_count) {
@@ -874,7 +875,6 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       const int j = q4 * 32 + lane;
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
       float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
-      float* alpha_s = reinterpret_cast<float*>(smem + C::kAlpha);             // [4][32]
       float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
       float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
       const uint32_t bar_id = kBarGroup0 + g;
@@ -897,10 +897,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
       const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
 
-      float acc[RW], lpart[RW], bias[RW];
+      float lpart[RW], bias[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
-        acc[r] = lpart[r] = 0.f;
+        lpart[r] = 0.f;
         bias[r] = INFINITY;  // no reference yet: the row's first key forces one
       }
       // Reference max (raw score) of row row0 + lane % RW; -inf until the
@@ -908,80 +908,64 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       float m_lane = -INFINITY;
       bool ok = true;
       const int end_t = t_count;  // tiles of this CTA (local t -> tile t_first + t)
-
-      // Iteration t scores tile t and folds tile t-2's O^T (finished long
-      // ago) into the register accumulators; the two iterations after the
-      // last tile only fold.  Tile u's rescale factors live in alpha_s[u % 4].
-      // S(t) in TMEM implies O(t-2) (the issuer commits S(t) after issuing
-      // PV(t-2)), so one wait per tile suffices; the fold-only iterations
-      // wait for O itself.  With two P buffers, O(t-2) done also frees P
-      // buffer t % 2 (PV(t-2) read it).
-      for (int t = 0;; ++t) {
-        if (t - 2 >= end_t) break;  // the last tile (end_t - 1) was folded at end_t + 1
-        const bool has_s = t < end_t, has_o = t >= 2;
-        const int gt = t_first + t;  // tile number of local tile t (when has_s)
-        const int sb = t % 2, st = t % VS, ob = t % 2;  // O of tile t-2 sits in buffer t%2
-        if (has_s)
-          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
-        else if (has_o)
-          ok = __all_sync(0xffffffffu,
-                          ok && mbar_wait(bar(BAR_OFULL + ob), ((t - 2) / 2) & 1, abort));
-        float sv[RW], oh[RW], ol[RW];
+      // O^T accumulates in TMEM over every tile (columns 2NR.. : the high
+      // parts of the rows, then their residuals).  When a row's reference
+      // rises at tile t, its O column is scaled by alpha in place, after
+      // PV(t-1) has finished and before P(t) is published.  S(t) in TMEM
+      // implies that PV(t-2) has finished (the issuer commits S(t) after
+      // issuing PV(t-2)), so P buffer t % 2 is free again.
+      const uint32_t o_hi = tmem + lane_off + 2 * NR + row0, o_lo = o_hi + NR;
+      for (int t = 0; t < end_t; ++t) {
+        const int gt = t_first + t;  // tile number of local tile t
+        const int sb = t % 2, st = t % VS;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+        float sv[RW];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) sv[r] = oh[r] = ol[r] = 0.f;
+        for (int r = 0; r < RW; ++r) sv[r] = 0.f;
         if (ok) {
           tc_fence_after();
-          if (has_o) {
-            tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + row0, oh);
-            tmem_ld<RW>(tmem + lane_off + 2 * NR + ob * 2 * NR + NR + row0, ol);
-          }
-          if (has_s) tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
+          tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
           tmem_ld_wait();
           tc_fence_before();
         }
         __syncwarp();
-        if (ok && lane == 0) {
-          if (has_o) mbar_arrive(bar(BAR_OEMPTY + ob));
-          if (has_s) mbar_arrive(bar(BAR_SEMPTY + sb));
-        }
+        if (ok && lane == 0) mbar_arrive(bar(BAR_SEMPTY + sb));
 
         uint32_t rmask = 0;
-        bool all_vis = false;  // every key of this warp is seen by every row
-        float x[RW];           // cs * s + bias: log2 of the scaled weight
-        bool exceed = false;
-        if (has_s) {
-          // Which rows see this key?  Chunks that were not loaded lie wholly
-          // outside [lo_u, hi_u], so their keys see none.
-          const int key = base + gt * kTileKeys + j;
-          if (ok && key >= lo_u && key <= hi_u) {
-            if (key >= lo_all && key <= hi_all) {
-              rmask = all_rows;
-            } else {
-#pragma unroll
-              for (int i = 0; i < kMaxQuery; ++i)
-                if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
-            }
-          }
-          all_vis = __all_sync(0xffffffffu, rmask == all_rows);
-          // x = -inf for a row that does not see this key: its weight is
-          // exactly 0 and it cannot raise the row's reference.
-          float xmax = -INFINITY;
-          if (all_vis) {  // interior tiles: every row sees every key
-#pragma unroll
-            for (int r = 0; r < RW; ++r) {
-              x[r] = fmaf(sv[r], cs, bias[r]);
-              xmax = fmaxf(xmax, x[r]);
-            }
+        // Which rows see this key?  Chunks that were not loaded lie wholly
+        // outside [lo_u, hi_u], so their keys see none.
+        const int key = base + gt * kTileKeys + j;
+        if (ok && key >= lo_u && key <= hi_u) {
+          if (key >= lo_all && key <= hi_all) {
+            rmask = all_rows;
           } else {
-            const uint32_t rm = rmask >> row0;
 #pragma unroll
-            for (int r = 0; r < RW; ++r) {
-              x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
-              xmax = fmaxf(xmax, x[r]);
-            }
+            for (int i = 0; i < kMaxQuery; ++i)
+              if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
           }
-          exceed = xmax > (float)kPShift + kLazy;
         }
+        // every key of this warp is seen by every row: the interior fast path
+        const bool all_vis = __all_sync(0xffffffffu, rmask == all_rows);
+        // x = cs * s + bias, the log2 of the scaled weight; -inf for a row
+        // that does not see this key: its weight is exactly 0 and it cannot
+        // raise the row's reference.
+        float x[RW];
+        float xmax = -INFINITY;
+        if (all_vis) {
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            x[r] = fmaf(sv[r], cs, bias[r]);
+            xmax = fmaxf(xmax, x[r]);
+          }
+        } else {
+          const uint32_t rm = rmask >> row0;
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
+            xmax = fmaxf(xmax, x[r]);
+          }
+        }
+        const bool exceed = xmax > (float)kPShift + kLazy;
         // Reconverge before the group barrier: a warp that arrives diverged
         // (after lane-predicated code) makes the barrier several times slower
         // (measured: 61k verify 122 -> 67 us per call).
@@ -989,124 +973,146 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         // One barrier per tile: orders the shared-memory traffic of the group
         // and tells every thread whether any score passed its row's reference.
         const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
-        if (has_o && ok) {  // acc = acc * alpha_{t-2} + O_{t-2} (high + residual)
-          const float4* al = reinterpret_cast<const float4*>(alpha_s + ((t - 2) % 4) * 32 + row0);
+        if (rescale) {
+          // New reference max per row: warp transpose-reduction, then
+          // across the group's four warps.
+          const uint32_t rm = all_vis ? 0xffffffffu : (rmask >> row0);
+          float tmp[RW];
 #pragma unroll
-          for (int r = 0; r < RW; r += 4) {
-            const float4 a = al[r / 4];
-            acc[r] = fmaf(acc[r], a.x, oh[r] + ol[r]);
-            acc[r + 1] = fmaf(acc[r + 1], a.y, oh[r + 1] + ol[r + 1]);
-            acc[r + 2] = fmaf(acc[r + 2], a.z, oh[r + 2] + ol[r + 2]);
-            acc[r + 3] = fmaf(acc[r + 3], a.w, oh[r + 3] + ol[r + 3]);
-          }
-        }
-        if (has_s) {
-          float alpha = 1.f;
-          if (rescale) {
-            // New reference max per row: warp transpose-reduction, then
-            // across the group's four warps.
-            const uint32_t rm = all_vis ? 0xffffffffu : (rmask >> row0);
-            float tmp[RW];
-#pragma unroll
-            for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
-            const float wmax = warp_row_reduce<RW, true>(tmp, lane);
-            if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
-            __syncwarp();
-            named_bar_sync(bar_id, kSoftmaxThreads);
-            const int rl = lane % RW;
-            float tmax = red[(sb * 4 + 0) * 32 + rl];
-            tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
-            tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
-            tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
-            const float m_new = fmaxf(m_lane, tmax);
-            // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
-            // 2^(cs (s - m_new) + kPShift).
-            alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
-            const float bias_l =
-                (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
-            m_lane = m_new;
-            if (lane < RW) {
-              bc[lane] = bias_l;
-              bc[32 + lane] = alpha;
-            }
-            __syncwarp();
-            float av[RW];
-#pragma unroll
-            for (int r = 0; r < RW; r += 4) {
-              const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
-              const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
-              bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
-              av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
-            }
-#pragma unroll
-            for (int r = 0; r < RW; ++r) {
-              x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
-              lpart[r] *= av[r];
-            }
-          }
-          if (widx == 0 && lane < RW) alpha_s[(t % 4) * 32 + row0 + lane] = alpha;
-
-          // Scaled weights (2^-inf = 0 for keys a row does not see), split
-          // into an fp16 high part (the weight truncated to 11 significant
-          // bits: exact in fp16 over the weights' range) and an fp16 residual.
-          uint32_t phi[RW / 2], plo[RW / 2];
-#pragma unroll
-          for (int r = 0; r < RW; r += 2) {
-            const float p0 = fast_exp2(x[r]), p1 = fast_exp2(x[r + 1]);
-            lpart[r] += p0;
-            lpart[r + 1] += p1;
-            const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-            const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-            const __half2 h = __floats2half2_rn(h0, h1);
-            const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
-            phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-            plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-          }
-
-          // A key no row can see must not reach the PV product: zero its V
-          // row (after its V tile has landed).
-          if (!Q8 && g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
-            ok = __all_sync(0xffffffffu,
-                            ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
-            if (ok && rmask == 0) {
-              const uint4 z = make_uint4(0, 0, 0, 0);
-              const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                sts_v4(vrow + c * 16, z);
-                sts_v4(vrow + kAtomBytes + c * 16, z);
-              }
-            }
-          }
-          if (PB == 1 && t >= 1)  // the single P buffer: PV(t-1) must have read it
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL + (t - 1) % 2),
-                                                         ((t - 1) / 2) & 1, abort));
-          if (ok) {
-            // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
-            // [row'%8] with row' < NR the high parts and row' >= NR the
-            // residuals, in P buffer t % PB.
-            const uint32_t pbuf = sP + (t % PB) * C::kPBytes;
-            const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
-            constexpr uint32_t lo_off = (NR / 8) * 128;
-            if constexpr (RW >= 8) {
-#pragma unroll
-              for (int r8 = 0; r8 < RW / 8; ++r8) {
-                const uint32_t off = kb + ((row0 / 8) + r8) * 128;
-                sts_v4(pbuf + off,
-                       make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
-                sts_v4(pbuf + lo_off + off,
-                       make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
-              }
-            } else {  // four rows: half of one 16-byte core-matrix row
-              const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
-              sts_v2(pbuf + off, phi[0], phi[1]);
-              sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
-            }
-            fence_proxy_async_smem();
+          for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
+          const float wmax = warp_row_reduce<RW, true>(tmp, lane);
+          if (lane < RW) red[(sb * 4 + widx) * 32 + lane] = wmax;
+          __syncwarp();
+          named_bar_sync(bar_id, kSoftmaxThreads);
+          const int rl = lane % RW;
+          float tmax = red[(sb * 4 + 0) * 32 + rl];
+          tmax = fmaxf(tmax, red[(sb * 4 + 1) * 32 + rl]);
+          tmax = fmaxf(tmax, red[(sb * 4 + 2) * 32 + rl]);
+          tmax = fmaxf(tmax, red[(sb * 4 + 3) * 32 + rl]);
+          const float m_new = fmaxf(m_lane, tmax);
+          // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
+          // 2^(cs (s - m_new) + kPShift).
+          const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
+          const float bias_l =
+              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
+          m_lane = m_new;
+          if (lane < RW) {
+            bc[lane] = bias_l;
+            bc[32 + lane] = alpha;
           }
           __syncwarp();
-          if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % PB));
+          float av[RW];
+#pragma unroll
+          for (int r = 0; r < RW; r += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
+            const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
+            bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
+            av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
+          }
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
+            lpart[r] *= av[r];
+          }
+          if (t > 0) {  // rescale the accumulated O columns of this group's rows
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (t - 1) & 1, abort));
+            if (ok) {
+              tc_fence_after();
+              float oh[RW], ol[RW];
+              tmem_ld<RW>(o_hi, oh);
+              tmem_ld<RW>(o_lo, ol);
+              tmem_ld_wait();
+#pragma unroll
+              for (int r = 0; r < RW; ++r) {
+                oh[r] *= av[r];
+                ol[r] *= av[r];
+              }
+              tmem_st<RW>(o_hi, oh);
+              tmem_st<RW>(o_lo, ol);
+              tmem_st_wait();
+              tc_fence_before();  // ordered before the PFULL arrive below
+            }
+          }
         }
+
+        // Scaled weights (2^-inf = 0 for keys a row does not see), split
+        // into an fp16 high part (the weight truncated to 11 significant
+        // bits: exact in fp16 over the weights' range) and an fp16 residual.
+        uint32_t phi[RW / 2], plo[RW / 2];
+#pragma unroll
+        for (int r = 0; r < RW; r += 2) {
+          const float p0 = fast_exp2(x[r]), p1 = fast_exp2(x[r + 1]);
+          lpart[r] += p0;
+          lpart[r + 1] += p1;
+          const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+          const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+          const __half2 h = __floats2half2_rn(h0, h1);
+          const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
+          phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+          plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+
+        // A key no row can see must not reach the PV product: zero its V
+        // row (after its V tile has landed).  (q8_0: the converter does.)
+        if (!Q8 && g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
+          ok = __all_sync(0xffffffffu,
+                          ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
+          if (ok && rmask == 0) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              sts_v4(vrow + c * 16, z);
+              sts_v4(vrow + kAtomBytes + c * 16, z);
+            }
+          }
+        }
+        if (ok) {
+          // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
+          // [row'%8] with row' < NR the high parts and row' >= NR the
+          // residuals, in P buffer t % PB.
+          const uint32_t pbuf = sP + (t % PB) * C::kPBytes;
+          const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
+          constexpr uint32_t lo_off = (NR / 8) * 128;
+          if constexpr (RW >= 8) {
+#pragma unroll
+            for (int r8 = 0; r8 < RW / 8; ++r8) {
+              const uint32_t off = kb + ((row0 / 8) + r8) * 128;
+              sts_v4(pbuf + off,
+                     make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
+              sts_v4(pbuf + lo_off + off,
+                     make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
+            }
+          } else {  // four rows: half of one 16-byte core-matrix row
+            const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
+            sts_v2(pbuf + off, phi[0], phi[1]);
+            sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % PB));
+      }
+
+      // The accumulated O^T once PV(end_t - 1) has finished: high + residual.
+      // A parity wait is only exact while the barrier is at most one phase
+      // behind: with two tiles, S(1) says nothing about PV(0), so wait for
+      // phase end_t - 2 first.
+      float acc[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) acc[r] = 0.f;
+      if (end_t >= 2)
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (end_t - 2) & 1, abort));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (end_t - 1) & 1, abort));
+      if (ok) {
+        tc_fence_after();
+        float oh[RW], ol[RW];
+        tmem_ld<RW>(o_hi, oh);
+        tmem_ld<RW>(o_lo, ol);
+        tmem_ld_wait();
+#pragma unroll
+        for (int r = 0; r < RW; ++r) acc[r] = oh[r] + ol[r];
+        tc_fence_before();
       }
 
       // Row sums: per-thread partials -> per-warp (lane r) -> across warps.

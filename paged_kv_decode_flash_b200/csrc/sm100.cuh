@@ -269,6 +269,38 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[M]) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Each thread of the warp writes v[OFF .. OFF+N-1] to N consecutive 32-bit
+// columns of its own TMEM lane (N = 4, 8 or 16).
+template <int N, int OFF = 0, int M>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&v)[M]) {
+  static_assert(OFF + N <= M, "tmem_st out of range");
+  uint32_t r[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) r[i] = __float_as_uint(v[OFF + i]);
+  if constexpr (N == 16) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+  } else if constexpr (N == 8) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                     taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+                 : "memory");
+  } else {
+    static_assert(N == 4, "tmem_st: 4, 8 or 16 columns");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+  }
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // ------------------------------------------------------------- descriptors
 // Swizzle codes of the shared-memory matrix descriptor.

@@ -90,6 +90,26 @@ def test_random_sweep(B, orc, case):
     assert_parity(out, ref, "sweep")
 
 
+@pytest.mark.parametrize("tiles_per_cta,dt,nq,G", [(2, gen.KV_FP16, 8, 4), (3, gen.KV_FP16, 1, 8),
+                                                  (5, gen.KV_FP16, 4, 4), (2, gen.KV_Q8_0, 4, 4),
+                                                  (4, gen.KV_Q8_0, 1, 8)])
+def test_several_tiles_per_split(B, orc, tiles_per_cta, dt, nq, G):
+    """Splits of 2-5 tiles of 128 keys, with key spikes so that rows raise
+    their running maximum after the first tile (the accumulated output is
+    then rescaled in place); every row against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    L = sms * 128 * tiles_per_cta - 37  # one split per SM, ragged last tile
+    case = gen.make_case(seed=40 + tiles_per_cta, context_lens=(L,), n_query=nq, num_q_heads=G,
+                         num_kv_heads=1, causal=1, kv_dtype=dt, spike_frac=0.003,
+                         spike_gain=6.0, max_blocks_per_seq=(L + 15) // 16)
+    dec = B.PagedDecode.for_case(case)
+    S = dec.num_splits(dt)
+    assert -(-((L + 127) // 128) // S) == tiles_per_cta, (S, L)
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, f"{tiles_per_cta} tiles per split")
+
+
 def test_sliding_window_config_and_nan_invariance(B, orc):
     case = gen.sliding_window(0)
     out, _ = run(B, case)
