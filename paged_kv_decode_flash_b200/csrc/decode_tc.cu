@@ -184,6 +184,13 @@ struct TileInfo {
 };
 static_assert(sizeof(TileInfo) == 48, "TileInfo layout");
 
+// 32-bit load through the non-coherent path, issued in program order with
+// the other volatile loads (so that two independent loads are in flight).
+__device__ __forceinline__ int ld_nc_s32(const int* p) {
+  int r;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -474,7 +481,22 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // partition depends only on the context length and S, so every call on the
   // same inputs adds the same tiles in the same order: results are
   // bit-reproducible.
-  const int L = p.context_lens[s];
+  const int L = ld_nc_s32(p.context_lens + s);
+  // While L is in flight, the K producer lanes read the block-table entries
+  // of this split's first tile on the guess that the whole table is visible
+  // (no window, full length); used below only if the guess was right.  This
+  // takes one memory latency off the time to the first tile.
+  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
+  int spec_key0 = -1, spec_phys = 0;
+  if (warp == 0 && lane < kChunksPerTile) {
+    const int ntg = (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
+    const int tfg = split * (ntg / S) + min(split, ntg % S);
+    const int key0 = tfg * kTileKeys + lane * kChunk;
+    if (ntg / S + (split < ntg % S ? 1 : 0) > 0 && key0 / p.block_size < p.max_blocks_per_seq) {
+      spec_key0 = key0;
+      spec_phys = ld_nc_s32(table + key0 / p.block_size);
+    }
+  }
   int lo_u = 0, hi_u = -1;
   if (context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size)) {
     union_range(L, nq, p.causal, p.window, lo_u, hi_u);
@@ -486,7 +508,6 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
   const int t_first = split * t_per + min(split, t_rem);
   const int t_count = t_per + (split < t_rem ? 1 : 0);
-  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
 
   const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
   const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
@@ -562,7 +583,13 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       const int key0 = base + tile_of(t) * kTileKeys + c * kChunk;
       return (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
     };
-    int row_cur = to_row8(lookup_raw(0), 0);
+    long long raw0 = kNone;
+    if (c < kChunksPerTile && t_count > 0) {
+      const int key0 = base + t_first * kTileKeys + c * kChunk;
+      if (key0 <= hi_u && key0 + kChunk - 1 >= lo_u)
+        raw0 = key0 == spec_key0 ? (long long)spec_phys : (long long)table[key0 / p.block_size];
+    }
+    int row_cur = to_row8(raw0, 0);
     long long raw_nxt = lookup_raw(1);
     int issued = 0;
     for (int t = 0;; ++t) {
