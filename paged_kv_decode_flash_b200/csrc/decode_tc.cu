@@ -481,6 +481,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // partition depends only on the context length and S, so every call on the
   // same inputs adds the same tiles in the same order: results are
   // bit-reproducible.
+  // Launched as a programmatic dependent of whatever precedes it on the
+  // stream: set-up above touched only registers; nothing global is read
+  // before that grid has completed and flushed.  Dependents of this grid
+  // may launch at once (they wait the same way).
+  griddep_wait();
+  griddep_launch_dependents();
   const int L = ld_nc_s32(p.context_lens + s);
   // While L is in flight, the K producer lanes read the block-table entries
   // of this split's first tile on the guess that the whole table is visible
@@ -1288,11 +1294,15 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   cfg.blockDim = dim3(Cfg<RW, NG, Q8>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  // Programmatic stream serialization lets this grid's CTAs be scheduled
+  // while the previous kernel drains (they wait in griddepcontrol.wait).
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.coop ? 1 : 0;
+  cfg.numAttrs = p.coop ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW, NG, Q8>, mk, mv, p);
 }
 
