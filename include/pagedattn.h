@@ -100,14 +100,15 @@ typedef struct {
 } pa_dims;
 
 /* Bytes of workspace paged_attn_decode needs for these shapes: a 256-byte
- * status header, one int32 arrival counter per (sequence, KV head) and the
+ * status header, two int32 arrival counters per (sequence, KV head) and the
  * split partials.  Host only, no device access.  Returns 0 for invalid
  * shapes. */
 size_t paged_attn_workspace_size(const pa_dims* dims, int32_t n_query);
 
 /* Zero the workspace status header and arrival counters (enqueued on
  * `stream`).  Call once after allocating a workspace, before its first
- * paged_attn_decode; every decode call leaves the counters at zero again. */
+ * paged_attn_decode; every decode call leaves the counters ready for the
+ * next (their low 31 bits at zero). */
 int paged_attn_workspace_init(const pa_dims* dims, void* stream);
 
 /* Decode attention (see the header comment for the exact definition).

@@ -34,7 +34,9 @@ struct DecodeParams {
   int num_seqs, num_q_heads, num_kv_heads, block_size, max_blocks_per_seq;
   int num_blocks, n_query, causal, window, kv_dtype, group, rows;
   float scale_log2;           // scale * log2(e): scores live in the log2 domain
-  int num_splits;             // key splits per (seq, kv head)
+  int num_splits;             // key splits per (seq, kv head) (CUDA-core kernel;
+                              // tensor-core kernel: ceil(num_ctas / groups))
+  int num_ctas;               // tensor-core kernel: CTAs of the (1-D) grid
   int blocks_per_split;       // logical blocks per split
   float* part_out;            // [B][S][nq*Hq][D]
   float* part_lse;            // [B][S][nq*Hq], natural log

@@ -171,6 +171,7 @@ struct Misc {
   int k_consumed, v_consumed;
   int last;  // this CTA arrived last in its (sequence, KV head): it merges
   int bad;   // a block index of this CTA's keys was out of range
+  int g_s, g_kvh, g_split, g_splits, g_first;  // group_of() of this CTA
 };
 
 // What the K producer publishes for each local tile of a CTA: the tile's
@@ -207,6 +208,98 @@ __device__ __forceinline__ void sts_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
+// Visible 128-key tiles of a sequence of context length L (0 for a length
+// outside [n_query, max_blocks_per_seq * block_size]); also its first key
+// rounded down to a 16-key chunk and its visible range.
+struct SeqTiles {
+  int lo, hi, base, tiles;
+};
+__device__ __forceinline__ SeqTiles seq_tiles(const DecodeParams& p, int L) {
+  SeqTiles t{0, -1, 0, 0};
+  if (context_len_ok(L, p.n_query, p.max_blocks_per_seq, p.block_size)) {
+    union_range(L, p.n_query, p.causal, p.window, t.lo, t.hi);
+    t.base = (t.lo / kChunk) * kChunk;
+    if (t.hi >= t.lo) t.tiles = (t.hi + 1 - t.base + kTileKeys - 1) / kTileKeys;
+  }
+  return t;
+}
+
+// Which (sequence, KV head) group CTA c of the C CTAs works for.  Each of the
+// G = num_seqs * num_kv_heads groups gets one CTA plus a share of the other
+// C - G in proportion to its visible tiles: group g owns CTAs
+// [cum(g), cum(g+1)) with cum(g) = g + floor((C - G) * tiles before g / all
+// tiles).  A batch of equal lengths gets C / G CTAs per group in blockIdx
+// order; a mixed batch gives long sequences more splits.  Computed by one
+// warp from context_lens alone (device side, no host synchronisation).
+struct GroupOf {
+  int s, kvh, split, splits, first;  // first: the group's first CTA
+};
+__device__ GroupOf group_of(const DecodeParams& p, int c, int C, int lane) {
+  const int B = p.num_seqs, H = p.num_kv_heads;
+  const long long E = (long long)C - (long long)B * H;
+  if (B == 1) {  // the KV heads of one sequence weigh the same: cum(k) = k + floor(E k / H)
+    GroupOf r{0, 0, 0, 1, 0};
+    int k = (int)((long long)c * H / C);
+    auto cum = [&](int kk) { return kk + (int)(E * kk / H); };
+    while (k > 0 && cum(k) > c) --k;
+    while (k + 1 < H && cum(k + 1) <= c) ++k;
+    r.kvh = k;
+    r.first = cum(k);
+    r.splits = cum(k + 1) - cum(k);
+    r.split = c - r.first;
+    return r;
+  }
+  long long tot = 0;  // visible tiles of all sequences (per KV head)
+  for (int s0 = 0; s0 < B; s0 += 32) {
+    const int sq = s0 + lane;
+    int T = sq < B ? seq_tiles(p, __ldg(p.context_lens + sq)).tiles : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
+    tot += T;
+  }
+  const bool uniform_weights = tot == 0;  // nothing visible anywhere: equal shares
+  if (uniform_weights) tot = B;
+  GroupOf r{0, 0, 0, 1, 0};
+  long long run = 0;  // tiles of the sequences before this chunk
+  for (int s0 = 0; s0 < B; s0 += 32) {
+    const int sq = s0 + lane;
+    long long T = sq < B ? (uniform_weights ? 1 : seq_tiles(p, __ldg(p.context_lens + sq)).tiles) : 0;
+    long long incl = T;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const long long P = run + incl - T;  // tiles of sequences before sq
+    // cum at (sq, kvh) = sq*H + kvh + floor(E * (H*P + kvh*T) / (H*tot))
+    auto cum = [&](int kvh) {
+      return (long long)sq * H + kvh + (E * (H * P + kvh * T)) / (H * tot);
+    };
+    const bool mine = sq < B && cum(0) <= c && c < cum(H);
+    const unsigned m = __ballot_sync(0xffffffffu, mine);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      if (lane == src) {
+        int k = 0;
+        while (k + 1 < H && cum(k + 1) <= c) ++k;
+        r.s = sq;
+        r.kvh = k;
+        r.first = (int)cum(k);
+        r.splits = (int)(cum(k + 1) - cum(k));
+        r.split = c - r.first;
+      }
+      r.s = __shfl_sync(0xffffffffu, r.s, src);
+      r.kvh = __shfl_sync(0xffffffffu, r.kvh, src);
+      r.first = __shfl_sync(0xffffffffu, r.first, src);
+      r.splits = __shfl_sync(0xffffffffu, r.splits, src);
+      r.split = __shfl_sync(0xffffffffu, r.split, src);
+      break;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return r;
+}
+
 // q8_0 cache: byte offset of the qs rows of the 16-key chunk that starts at
 // key key0 of (block, head) tile `tile` (tiles are block_size * (128 + 8)
 // bytes: qs [block_size][128] then fp16 d [block_size][4]).
@@ -219,16 +312,16 @@ __device__ __forceinline__ long long q8_scale_offset(const DecodeParams& p, int 
   return (long long)(p.block_size - slot) * kHeadDim + slot * 8;
 }
 
-// Eight signed bytes -> eight exact floats: byte b becomes the low mantissa
-// byte of 2^23 + (b + 128) (a float whose value is that integer), minus
-// 2^23 + 128.
-__device__ __forceinline__ void q8_to_float8(uint2 q, float (&x)[8]) {
+// Eight signed bytes -> eight exact fp16 values, two per half2: byte b
+// becomes the low mantissa byte of the fp16 1024 + (b + 128) (bits 0x6400 |
+// (b ^ 0x80)), minus 1152; every integer below 2048 is exact in fp16.
+__device__ __forceinline__ void q8_to_half8(uint2 q, __half2 (&x)[4]) {
   const uint32_t w0 = q.x ^ 0x80808080u, w1 = q.y ^ 0x80808080u;
+  const uint32_t u[4] = {__byte_perm(w0, 0x64646464u, 0x5140), __byte_perm(w0, 0x64646464u, 0x7362),
+                         __byte_perm(w1, 0x64646464u, 0x5140), __byte_perm(w1, 0x64646464u, 0x7362)};
+  const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    x[e] = __uint_as_float(__byte_perm(w0, 0x4B00u, 0x5440u | e)) - 8388736.f;
-    x[4 + e] = __uint_as_float(__byte_perm(w1, 0x4B00u, 0x5440u | e)) - 8388736.f;
-  }
+  for (int e = 0; e < 4; ++e) x[e] = __hsub2(*reinterpret_cast<const __half2*>(&u[e]), off);
 }
 
 // Warp transpose-reduction over the 32 lanes (= 32 keys): lane l ends with
@@ -262,14 +355,14 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
 // flight at once, so that the merge costs a few memory latencies rather than
 // one per split.
 template <int RW, int NG, bool Q8>
-__device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, uint8_t* smem,
-                                            uint32_t sbase) {
+__device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, int S, int first,
+                                            uint8_t* smem, uint32_t sbase) {
   using C = Cfg<RW, NG, Q8>;
   constexpr int kThreads = C::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;  // float4 per partial row
   constexpr int kWarps = kThreads / 32;
   constexpr int kPairsMax = (NG * RW * kRowF4 + kThreads - 1) / kThreads;  // rows <= NG * RW
-  const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
+  const int R = p.rows, G = p.group, Hq = p.num_q_heads;
   const long long rps = (long long)p.n_query * Hq;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   float* w = reinterpret_cast<float*>(smem);  // [S][R]
@@ -279,7 +372,7 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
   const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);
   const int per_round = max(1, (int)((C::kRed - stage_off) / (uint32_t)(R * kHeadDim * 4)));
   auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
-  const long long split0 = (long long)s * S * rps;  // row offset of split 0 of sequence s
+  const long long split0 = (long long)first * R;  // partial row of (split 0, row 0) of the group
 
   // Raw log-sum-exps, all loads in flight together.
   for (int i0 = 0; i0 < S * R; i0 += 8 * kThreads) {
@@ -287,8 +380,7 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int i = i0 + u * kThreads + threadIdx.x;
-      v[u] = i < S * R ? __ldcg(p.part_lse + split0 + (long long)(i / R) * rps + row_index(i % R))
-                       : 0.f;
+      v[u] = i < S * R ? __ldcg(p.part_lse + split0 + i) : 0.f;  // [split][row]
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -332,7 +424,7 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
     const int nrows = (k1 - k0) * R;
     for (int q = warp; q < nrows; q += kWarps) {
       const int k = k0 + q / R, r = q % R;
-      const float* src = p.part_out + (split0 + k * rps + row_index(r)) * kHeadDim + lane * 4;
+      const float* src = p.part_out + (split0 + (long long)k * R + r) * kHeadDim + lane * 4;
       cp_async_16(stage + (uint32_t)(q * kRowF4 + lane) * 16u, src);
     }
     cp_async_wait_all();
@@ -372,16 +464,18 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kv
 // Cooperative merge (every CTA of the grid resident): once its whole group
 // has written its partials, split k of a (sequence, KV head) merges pairs
 // [k*P/S, (k+1)*P/S) of the group's P = R*32 (row, float4 column) pairs.
-// Same arithmetic as merge_group (log-sum-exp weights, splits added in index
-// order), spread over all S CTAs of the group so that each stages only a
-// few kilobytes of partials with one round of 16-byte asynchronous copies.
+// The log-sum-exp weights of merge_group, spread over all S CTAs of the
+// group so that each stages only a few kilobytes of partials with one round
+// of 16-byte asynchronous copies; the weighted partials of a pair are added
+// in a fixed order (lane i of a pair's lanes takes splits i, i + tp, ...,
+// then a butterfly), so results stay reproducible.
 template <int RW, int NG, bool Q8>
-__device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split,
-                                            uint8_t* smem, uint32_t sbase) {
+__device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split, int S,
+                                            int first, uint8_t* smem, uint32_t sbase) {
   constexpr int kThreads = Cfg<RW, NG, Q8>::kThreads;
   constexpr int kRowF4 = kHeadDim / 4;
   constexpr int kWarps = kThreads / 32;
-  const int R = p.rows, S = p.num_splits, G = p.group, Hq = p.num_q_heads;
+  const int R = p.rows, G = p.group, Hq = p.num_q_heads;
   const long long rps = (long long)p.n_query * Hq;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int P = R * kRowF4;
@@ -389,7 +483,7 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   if (pa >= pb) return;  // uniform across the CTA
   const int r_lo = pa / kRowF4, nr = (pb - 1) / kRowF4 - r_lo + 1, np = pb - pa;
   auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
-  const long long split0 = (long long)s * S * rps;  // row offset of split 0 of sequence s
+  const long long split0 = (long long)first * R;  // partial row of (split 0, row 0) of the group
   float* w = reinterpret_cast<float*>(smem);  // [nr][S]
   float* inv = w + nr * S;                    // [nr]
   const uint32_t stage_off = ((uint32_t)(nr * S + nr) * 4u + 1023u) & ~1023u;
@@ -399,11 +493,11 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   for (int e = threadIdx.x; e < S * np; e += kThreads) {
     const int k = e / np, pr = pa + e % np;
     const float* src =
-        p.part_out + (split0 + k * rps + row_index(pr / kRowF4)) * kHeadDim + (pr % kRowF4) * 4;
+        p.part_out + (split0 + (long long)k * R + pr / kRowF4) * kHeadDim + (pr % kRowF4) * 4;
     cp_async_16(sbase + stage_off + (uint32_t)e * 16u, src);
   }
   for (int e = threadIdx.x; e < nr * S; e += kThreads)
-    w[e] = __ldcg(p.part_lse + split0 + (long long)(e % S) * rps + row_index(r_lo + e / S));
+    w[e] = __ldcg(p.part_lse + split0 + (long long)(e % S) * R + r_lo + e / S);
   __syncthreads();
   for (int j = warp; j < nr; j += kWarps) {
     float M = -INFINITY;
@@ -428,24 +522,42 @@ __device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kv
   }
   cp_async_wait_all();
   __syncthreads();
-  for (int q = threadIdx.x; q < np; q += kThreads) {
-    const int pr = pa + q, r = pr / kRowF4, c4 = pr % kRowF4, j = r - r_lo;
+  // tp threads (lanes of one warp) per pair, each adding every tp-th split;
+  // then a fixed butterfly over the tp lanes.  Loop bounds are uniform per
+  // warp, so every lane takes part in the shuffles.
+  int tp = 1;
+  while (tp < 32 && 2 * tp * np <= kThreads) tp *= 2;
+  const int per_warp = 32 / tp, sub = lane % tp;
+  for (int q0 = warp * per_warp; q0 < np; q0 += kWarps * per_warp) {
+    const int q = q0 + lane / tp;
+    const bool valid = q < np;
+    const int pr = pa + (valid ? q : 0), r = pr / kRowF4, c4 = pr % kRowF4, j = r - r_lo;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < S; ++k) {
-      const float wk = w[j * S + k];
-      const float4 v = stage4[k * np + q];
-      acc.x = fmaf(wk, v.x, acc.x);
-      acc.y = fmaf(wk, v.y, acc.y);
-      acc.z = fmaf(wk, v.z, acc.z);
-      acc.w = fmaf(wk, v.w, acc.w);
+    if (valid) {
+      for (int k = sub; k < S; k += tp) {
+        const float wk = w[j * S + k];
+        const float4 v = stage4[k * np + q];
+        acc.x = fmaf(wk, v.x, acc.x);
+        acc.y = fmaf(wk, v.y, acc.y);
+        acc.z = fmaf(wk, v.z, acc.z);
+        acc.w = fmaf(wk, v.w, acc.w);
+      }
     }
-    const float iv = inv[j];
-    const __half2 h0 = __floats2half2_rn(acc.x * iv, acc.y * iv);
-    const __half2 h1 = __floats2half2_rn(acc.z * iv, acc.w * iv);
-    uint2 u;
-    u.x = *reinterpret_cast<const uint32_t*>(&h0);
-    u.y = *reinterpret_cast<const uint32_t*>(&h1);
-    *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
+    for (int o = tp / 2; o > 0; o >>= 1) {
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    if (valid && sub == 0) {
+      const float iv = inv[j];
+      const __half2 h0 = __floats2half2_rn(acc.x * iv, acc.y * iv);
+      const __half2 h1 = __floats2half2_rn(acc.z * iv, acc.w * iv);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&h0);
+      u.y = *reinterpret_cast<const uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
+    }
   }
 }
 
@@ -466,51 +578,66 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   volatile int* abort = &misc->abort;
   auto bar = [&](int i) { return sbase + C::kBars + 8u * i; };
 
-  const int split = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
-  const int S = p.num_splits;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nq = p.n_query, G = p.group, Hq = p.num_q_heads, R = p.rows;
-  const int rps = nq * Hq;
-  const long long part_base = ((long long)s * S + split) * rps;
-  auto row_index = [&](int r) { return (r / G) * Hq + kvh * G + (r % G); };
+  const int C_all = gridDim.x, cta = blockIdx.x;
 
-  // ---- the head's visible keys and its tiles (uniform across the CTA) ------
-  // The keys of (sequence s, KV head kvh) that any query token sees form
-  // [lo_u, hi_u]; they are cut into 128-key tiles from `base`, and the S
-  // splits take contiguous runs of them, as even as whole tiles allow.  The
-  // partition depends only on the context length and S, so every call on the
-  // same inputs adds the same tiles in the same order: results are
-  // bit-reproducible.
   // Launched as a programmatic dependent of whatever precedes it on the
   // stream: set-up above touched only registers; nothing global is read
   // before that grid has completed and flushed.  Dependents of this grid
   // may launch at once (they wait the same way).
   griddep_wait();
   griddep_launch_dependents();
-  const int L = ld_nc_s32(p.context_lens + s);
-  // While L is in flight, the K producer lanes read the block-table entries
-  // of this split's first tile on the guess that the whole table is visible
-  // (no window, full length); used below only if the guess was right.  This
-  // takes one memory latency off the time to the first tile.
-  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
+  // Which (sequence, KV head) this CTA works for (warp 0).  With one
+  // sequence that needs no memory access, and the K producer lanes then read
+  // the block-table entries of this CTA's first tile on the guess that the
+  // whole table is visible (no window, full length) while the context length
+  // is in flight; used below only if the guess held.  This takes one memory
+  // latency off the time to the first tile.
   int spec_key0 = -1, spec_phys = 0;
-  if (warp == 0 && lane < kChunksPerTile) {
-    const int ntg = (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
-    const int tfg = split * (ntg / S) + min(split, ntg % S);
-    const int key0 = tfg * kTileKeys + lane * kChunk;
-    if (ntg / S + (split < ntg % S ? 1 : 0) > 0 && key0 / p.block_size < p.max_blocks_per_seq) {
-      spec_key0 = key0;
-      spec_phys = ld_nc_s32(table + key0 / p.block_size);
+  if (warp == 0) {
+    const GroupOf go = group_of(p, cta, C_all, lane);
+    if (lane == 0) {
+      misc->g_s = go.s;
+      misc->g_kvh = go.kvh;
+      misc->g_split = go.split;
+      misc->g_splits = go.splits;
+      misc->g_first = go.first;
+    }
+    if (p.num_seqs == 1 && lane < kChunksPerTile) {
+      const int ntg =
+          (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
+      const int tfg = go.split * (ntg / go.splits) + min(go.split, ntg % go.splits);
+      const int key0 = tfg * kTileKeys + lane * kChunk;
+      if (ntg / go.splits + (go.split < ntg % go.splits ? 1 : 0) > 0 &&
+          key0 / p.block_size < p.max_blocks_per_seq) {
+        spec_key0 = key0;
+        spec_phys = ld_nc_s32(p.block_table + key0 / p.block_size);
+      }
     }
   }
-  int lo_u = 0, hi_u = -1;
-  if (context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size)) {
-    union_range(L, nq, p.causal, p.window, lo_u, hi_u);
-  } else if (split == 0 && kvh == 0 && threadIdx.x == 0) {
+  __syncthreads();
+  const int s = misc->g_s, kvh = misc->g_kvh, split = misc->g_split;
+  const int S = misc->g_splits, first = misc->g_first;
+  // Partials: CTA c owns rows [c*R, c*R + R) of the partial outputs and
+  // log-sum-exps; the CTAs of one group are consecutive.
+  const long long part_base = (long long)cta * R;
+  auto row_index = [&](int r) { return (r / G) * Hq + kvh * G + (r % G); };
+
+  // ---- the head's visible keys and its tiles (uniform across the CTA) ------
+  // The keys of (sequence s, KV head kvh) that any query token sees form
+  // [lo_u, hi_u]; they are cut into 128-key tiles from `base`, and the S
+  // splits take contiguous runs of them, as even as whole tiles allow.  The
+  // partition depends only on the context lengths and the grid, so every
+  // call on the same inputs adds the same tiles in the same order: results
+  // are bit-reproducible.
+  const int L = ld_nc_s32(p.context_lens + s);
+  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
+  const SeqTiles st_ = seq_tiles(p, L);
+  const int lo_u = st_.lo, hi_u = st_.hi, base = st_.base, ntiles_h = st_.tiles;
+  if (!context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size) && split == 0 && kvh == 0 &&
+      threadIdx.x == 0)
     atomicOr(p.flags, kFlagBadLen);
-  }
-  const int base = (lo_u / kChunk) * kChunk;
-  const int ntiles_h = hi_u >= lo_u ? (hi_u + 1 - base + kTileKeys - 1) / kTileKeys : 0;
   const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
   const int t_first = split * t_per + min(split, t_rem);
   const int t_count = t_per + (split < t_rem ? 1 : 0);
@@ -522,8 +649,8 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     // Every tile is another CTA's: an empty partial (weight 0 in the merge).
     for (int t = threadIdx.x; t < R * kHeadDim; t += kThreads) {
       const int r = t / kHeadDim;
-      p.part_out[(part_base + row_index(r)) * kHeadDim + t % kHeadDim] = 0.f;
-      if (t % kHeadDim == 0) p.part_lse[part_base + row_index(r)] = -INFINITY;
+      p.part_out[(part_base + r) * kHeadDim + t % kHeadDim] = 0.f;
+      if (t % kHeadDim == 0) p.part_lse[part_base + r] = -INFINITY;
     }
   } else if (warp == 0) {
     // ======================= K producer (also sets up the barriers) ========
@@ -816,11 +943,11 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     } else if (Q8 && warp >= C::kConvWarp) {
       // ===================== q8_0 converter (4 warps) ========================
       // Raw tile t (int8 qs, fp16 scales d per 32 elements) -> the fp16 K and
-      // V operand tiles.  Each element is x = qs * d, exact in fp32 (an 8-bit
-      // integer times an 11-bit significand); the operand holds its high part
-      // (x truncated to 11 significant bits, exact in fp16) and, kKVBytes
-      // further, the fp16 residual x - high, so that the tensor core sees x to
-      // about 2^-22.  Layout as the fp16 TMA boxes: [key/8][half][key%8]
+      // V operand tiles.  Each element is x = qs * d; the operand holds its
+      // high part (x rounded to fp16) and, kKVBytes further, the residual
+      // x - high, which is an fp16 value as well, so that the tensor core
+      // sees x exactly.  The arithmetic is packed fp16 (two elements per
+      // instruction, no conversions).  Layout as the fp16 TMA boxes: [key/8][half][key%8]
       // [64 dims], 128-byte swizzle.  V rows of keys outside [lo_u, hi_u]
       // (masked or never loaded) are written as zeros: they must not reach
       // the PV product.
@@ -844,25 +971,26 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       int n = 0;
       bool ok = true;
       // One 8-element item: x = qs * d split into an fp16 high part and an
-      // fp16 residual (zeros for a V row no query row may see).
+      // fp16 residual (zeros for a V row no query row may see).  The high
+      // part is x rounded to fp16; qs * d has at most 18 significant bits
+      // and is a multiple of 2^-24 (the smallest fp16 step), so the residual
+      // x - high is an fp16 value too and the fused multiply-add gives it
+      // exactly: high + residual = x.
       auto convert = [&](const uint8_t* raw, int r, uint32_t off, bool live) {
         uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
         if (live) {
           const uint2 q = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
-          const float d = __half2float(
+          const __half2 d2 = __half2half2(
               *reinterpret_cast<const __half*>(raw + kRawQsBytes + r * 8 + (cc >> 2) * 2));
-          float x[8];
-          q8_to_float8(q, x);
+          __half2 x[4];
+          q8_to_half8(q, x);
           uint32_t h[4], l[4];
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const float x0 = x[e] * d, x1 = x[e + 1] * d;
-            const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffffe000u);
-            const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffffe000u);
-            const __half2 hh = __floats2half2_rn(h0, h1);
-            const __half2 ll = __floats2half2_rn(x0 - h0, x1 - h1);
-            h[e / 2] = *reinterpret_cast<const uint32_t*>(&hh);
-            l[e / 2] = *reinterpret_cast<const uint32_t*>(&ll);
+          for (int e = 0; e < 4; ++e) {
+            const __half2 hh = __hmul2(x[e], d2);
+            const __half2 ll = __hfma2(x[e], d2, __hneg2(hh));
+            h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            l[e] = *reinterpret_cast<const uint32_t*>(&ll);
           }
           hi = make_uint4(h[0], h[1], h[2], h[3]);
           lo = make_uint4(l[0], l[1], l[2], l[3]);
@@ -1160,7 +1288,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       for (int r = 0; r < RW; ++r) {
         if (row0 + r < R) {
           const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
-          const long long pr = part_base + row_index(row0 + r);
+          const long long pr = part_base + row0 + r;
           p.part_out[pr * kHeadDim + j] = (!aborted && !bad && l > 0.f) ? acc[r] / l : 0.f;
         }
       }
@@ -1168,7 +1296,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
         // NaN marks a partial that read a stand-in for an out-of-range block.
         const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
-        p.part_lse[part_base + row_index(row0 + lane)] =
+        p.part_lse[part_base + row0 + lane] =
             bad ? __int_as_float(0x7fc00000)
             : (!aborted && l > 0.f)
                 ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
@@ -1185,53 +1313,53 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   }
 
   // ---- arrival and merge --------------------------------------------------------
-  // Writers make their partials visible device-wide before they are counted.
-  // Counters (two per group) are zero at the start of a call and are reset
-  // by the call itself once no CTA of the group needs them any more (the
-  // next launch on the stream starts after this grid ends).
   if (t_count == 0 && threadIdx.x == 0) misc->abort = 0;  // set by the K producer otherwise
-  __threadfence();
   __syncthreads();  // (B) partials written, copies drained, TMEM freed
+  // Two counters per (sequence, KV head) group.  After (B), one thread makes
+  // the CTA's partials visible device-wide (its fence covers the stores the
+  // barrier ordered before it) and then counts the CTA in.
   int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
   if (p.coop) {
-    // Every CTA of the grid is resident: wait (bounded) until the whole group
-    // has written its partials, then merge this CTA's share of the group.
+    // Every CTA of the grid is resident: a barrier over the group's S CTAs,
+    // then each merges its share of the group.  The barrier needs no reset:
+    // the group's first CTA adds 2^31 - (S - 1) and the others 1, so the top
+    // bit of counter 0 flips once all S have arrived and its low bits return
+    // to their value (zero).  The wait is bounded.
     if (threadIdx.x == 0) {
-      atomicAdd(cnt, 1);
+      __threadfence();
+      const unsigned int add = split == 0 ? 0x80000000u - (unsigned int)(S - 1) : 1u;
+      const unsigned int old = atomicAdd(reinterpret_cast<unsigned int*>(cnt), add);
       const unsigned long long t0 = globaltimer();
       int ok = 1;
-      while (ld_acquire_gpu(cnt) < S) {
+      while ((((unsigned int)ld_acquire_gpu(cnt) ^ old) & 0x80000000u) == 0u) {
         if (globaltimer() - t0 > kWaitLimitNs) {
           ok = 0;
           break;
         }
         __nanosleep(32);
       }
+      __threadfence();
       misc->last = ok;
     }
     __syncthreads();
-    __threadfence();
     if (misc->last) {
-      merge_slice<RW, NG, Q8>(p, s, kvh, split, smem, sbase);
+      merge_slice<RW, NG, Q8>(p, s, kvh, split, S, first, smem, sbase);
     } else if (threadIdx.x == 0) {
       atomicOr(p.flags, kFlagTimeout);
     }
-    __syncthreads();
-    // The last CTA of the group to finish merging: every CTA of the group
-    // has passed its wait, so both counters can return to zero.
-    if (threadIdx.x == 0 && atomicAdd(cnt + 1, 1) == S - 1) {
-      atomicExch(cnt, 0);
-      atomicExch(cnt + 1, 0);
-    }
     return;
   }
-  // Otherwise the last CTA of the group to arrive merges all of it.
-  if (threadIdx.x == 0) misc->last = (atomicAdd(cnt, 1) == S - 1);
+  // Otherwise the last CTA of the group to arrive (counter 1) merges all of
+  // it and sets the counter back to zero.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    misc->last = (atomicAdd(cnt + 1, 1) == S - 1);
+  }
   __syncthreads();
   if (!misc->last) return;
   __threadfence();  // the other CTAs' partials, published before their counts
-  merge_group<RW, NG, Q8>(p, s, kvh, smem, sbase);
-  if (threadIdx.x == 0) *cnt = 0;
+  merge_group<RW, NG, Q8>(p, s, kvh, S, first, smem, sbase);
+  if (threadIdx.x == 0) cnt[1] = 0;
 }
 
 // ---- host side ----------------------------------------------------------------
@@ -1285,12 +1413,12 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) resident[dev] = per_sm * sms;
   }
-  const long long ctas = (long long)p.num_splits * p.num_kv_heads * p.num_seqs;
+  const long long ctas = p.num_ctas;
   // A cooperative launch guarantees that every CTA is resident at once, which
   // the group-wide merge waits rely on; larger grids merge in their last CTA.
   p.coop = (dev >= 0 && dev < 64 && ctas <= resident[dev]) ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.num_splits, p.num_kv_heads, p.num_seqs);
+  cfg.gridDim = dim3(p.num_ctas);
   cfg.blockDim = dim3(Cfg<RW, NG, Q8>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;

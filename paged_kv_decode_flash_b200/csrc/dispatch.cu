@@ -79,9 +79,19 @@ Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
   const int rows = n_query * (d->num_q_heads / d->num_kv_heads);
   pl.tensor_cores =
       decode_tc_supported(kv_dtype, rows, d->num_blocks, d->num_kv_heads, d->block_size);
-  pl.splits = pl.tensor_cores ? plan_splits(d, sms, false, &pl.blocks_per_split)
-                              : plan_splits(d, (long long)sms * kCtasPerSm, true,
-                                            &pl.blocks_per_split);
+  if (pl.tensor_cores) {
+    // One CTA per SM (one per group at least, and no more than the table's
+    // 128-key tiles could keep busy); the kernel shares them out among the
+    // groups in proportion to each group's visible tiles.
+    const long long groups = (long long)d->num_seqs * d->num_kv_heads;
+    const long long max_split = ceil_div((long long)d->max_blocks_per_seq * d->block_size, 128);
+    pl.ctas = (int)std::max(groups, std::min<long long>(sms, groups * max_split));
+    pl.splits = (int)ceil_div(pl.ctas, groups);
+    pl.blocks_per_split = (int)ceil_div(d->max_blocks_per_seq, pl.splits);
+  } else {
+    pl.splits = plan_splits(d, (long long)sms * kCtasPerSm, true, &pl.blocks_per_split);
+    pl.ctas = pl.splits * d->num_kv_heads * d->num_seqs;
+  }
   return pl;
 }
 
@@ -143,6 +153,7 @@ int enqueue_decode(const pa_dims* d, const Plan& plan, const void* q, const void
   p.rows = n_query * p.group;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_splits = plan.splits;
+  p.num_ctas = plan.ctas;
   p.blocks_per_split = plan.blocks_per_split;
   p.part_out = reinterpret_cast<float*>(ws + w.part_out);
   p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);

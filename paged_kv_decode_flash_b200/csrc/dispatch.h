@@ -15,6 +15,8 @@ namespace pa {
 struct Plan {
   bool tensor_cores;
   int splits, blocks_per_split;
+  int ctas;  // tensor-core kernel: CTAs of the grid (the device shares them out
+             // among the (sequence, KV head) groups); splits = ceil(ctas / groups)
 };
 
 // Workspace: status header | arrival counters | split partial outputs |
