@@ -225,78 +225,28 @@ __device__ __forceinline__ SeqTiles seq_tiles(const DecodeParams& p, int L) {
 }
 
 // Which (sequence, KV head) group CTA c of the C CTAs works for.  Each of the
-// G = num_seqs * num_kv_heads groups gets one CTA plus a share of the other
-// C - G in proportion to its visible tiles: group g owns CTAs
-// [cum(g), cum(g+1)) with cum(g) = g + floor((C - G) * tiles before g / all
-// tiles).  A batch of equal lengths gets C / G CTAs per group in blockIdx
-// order; a mixed batch gives long sequences more splits.  Computed by one
-// warp from context_lens alone (device side, no host synchronisation).
+// G = num_seqs * num_kv_heads groups gets C / G CTAs, as even as whole CTAs
+// allow: group g owns CTAs [cum(g), cum(g+1)) with cum(g) = g + floor((C -
+// G) g / G), in blockIdx order.  The grid and this mapping depend on the
+// shapes alone, never on the context lengths, so a sequence's splits, and
+// with them every bit of its output, do not depend on the other sequences
+// of the batch.
 struct GroupOf {
   int s, kvh, split, splits, first;  // first: the group's first CTA
 };
-__device__ GroupOf group_of(const DecodeParams& p, int c, int C, int lane) {
-  const int B = p.num_seqs, H = p.num_kv_heads;
-  const long long E = (long long)C - (long long)B * H;
-  if (B == 1) {  // the KV heads of one sequence weigh the same: cum(k) = k + floor(E k / H)
-    GroupOf r{0, 0, 0, 1, 0};
-    int k = (int)((long long)c * H / C);
-    auto cum = [&](int kk) { return kk + (int)(E * kk / H); };
-    while (k > 0 && cum(k) > c) --k;
-    while (k + 1 < H && cum(k + 1) <= c) ++k;
-    r.kvh = k;
-    r.first = cum(k);
-    r.splits = cum(k + 1) - cum(k);
-    r.split = c - r.first;
-    return r;
-  }
-  long long tot = 0;  // visible tiles of all sequences (per KV head)
-  for (int s0 = 0; s0 < B; s0 += 32) {
-    const int sq = s0 + lane;
-    int T = sq < B ? seq_tiles(p, __ldg(p.context_lens + sq)).tiles : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
-    tot += T;
-  }
-  const bool uniform_weights = tot == 0;  // nothing visible anywhere: equal shares
-  if (uniform_weights) tot = B;
-  GroupOf r{0, 0, 0, 1, 0};
-  long long run = 0;  // tiles of the sequences before this chunk
-  for (int s0 = 0; s0 < B; s0 += 32) {
-    const int sq = s0 + lane;
-    long long T = sq < B ? (uniform_weights ? 1 : seq_tiles(p, __ldg(p.context_lens + sq)).tiles) : 0;
-    long long incl = T;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const long long P = run + incl - T;  // tiles of sequences before sq
-    // cum at (sq, kvh) = sq*H + kvh + floor(E * (H*P + kvh*T) / (H*tot))
-    auto cum = [&](int kvh) {
-      return (long long)sq * H + kvh + (E * (H * P + kvh * T)) / (H * tot);
-    };
-    const bool mine = sq < B && cum(0) <= c && c < cum(H);
-    const unsigned m = __ballot_sync(0xffffffffu, mine);
-    if (m) {
-      const int src = __ffs(m) - 1;
-      if (lane == src) {
-        int k = 0;
-        while (k + 1 < H && cum(k + 1) <= c) ++k;
-        r.s = sq;
-        r.kvh = k;
-        r.first = (int)cum(k);
-        r.splits = (int)(cum(k + 1) - cum(k));
-        r.split = c - r.first;
-      }
-      r.s = __shfl_sync(0xffffffffu, r.s, src);
-      r.kvh = __shfl_sync(0xffffffffu, r.kvh, src);
-      r.first = __shfl_sync(0xffffffffu, r.first, src);
-      r.splits = __shfl_sync(0xffffffffu, r.splits, src);
-      r.split = __shfl_sync(0xffffffffu, r.split, src);
-      break;
-    }
-    run += __shfl_sync(0xffffffffu, incl, 31);
-  }
+__device__ __forceinline__ GroupOf group_of(const DecodeParams& p, int c, int C) {
+  const int G = p.num_seqs * p.num_kv_heads;
+  const long long E = (long long)C - G;
+  auto cum = [&](int g) { return g + (int)(E * g / G); };
+  int g = (int)((long long)c * G / C);
+  while (g > 0 && cum(g) > c) --g;
+  while (g + 1 < G && cum(g + 1) <= c) ++g;
+  GroupOf r;
+  r.s = g / p.num_kv_heads;
+  r.kvh = g % p.num_kv_heads;
+  r.first = cum(g);
+  r.splits = cum(g + 1) - r.first;
+  r.split = c - r.first;
   return r;
 }
 
@@ -588,15 +538,15 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // may launch at once (they wait the same way).
   griddep_wait();
   griddep_launch_dependents();
-  // Which (sequence, KV head) this CTA works for (warp 0).  With one
-  // sequence that needs no memory access, and the K producer lanes then read
-  // the block-table entries of this CTA's first tile on the guess that the
-  // whole table is visible (no window, full length) while the context length
-  // is in flight; used below only if the guess held.  This takes one memory
-  // latency off the time to the first tile.
+  // Which (sequence, KV head) this CTA works for (warp 0, no memory access).
+  // With one sequence, the K producer lanes then read the block-table entries
+  // of this CTA's first tile on the guess that the whole table is visible
+  // (no window, full length) while the context length is in flight; used
+  // below only if the guess held.  This takes one memory latency off the
+  // time to the first tile.
   int spec_key0 = -1, spec_phys = 0;
   if (warp == 0) {
-    const GroupOf go = group_of(p, cta, C_all, lane);
+    const GroupOf go = group_of(p, cta, C_all);
     if (lane == 0) {
       misc->g_s = go.s;
       misc->g_kvh = go.kvh;
@@ -976,27 +926,19 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       // and is a multiple of 2^-24 (the smallest fp16 step), so the residual
       // x - high is an fp16 value too and the fused multiply-add gives it
       // exactly: high + residual = x.
-      auto convert = [&](const uint8_t* raw, int r, uint32_t off, bool live) {
-        uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
-        if (live) {
-          const uint2 q = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
-          const __half2 d2 = __half2half2(
-              *reinterpret_cast<const __half*>(raw + kRawQsBytes + r * 8 + (cc >> 2) * 2));
-          __half2 x[4];
-          q8_to_half8(q, x);
-          uint32_t h[4], l[4];
+      auto convert = [&](uint2 q, __half2 d2, uint4& hi, uint4& lo) {
+        __half2 x[4];
+        q8_to_half8(q, x);
+        uint32_t h[4], l[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __half2 hh = __hmul2(x[e], d2);
-            const __half2 ll = __hfma2(x[e], d2, __hneg2(hh));
-            h[e] = *reinterpret_cast<const uint32_t*>(&hh);
-            l[e] = *reinterpret_cast<const uint32_t*>(&ll);
-          }
-          hi = make_uint4(h[0], h[1], h[2], h[3]);
-          lo = make_uint4(l[0], l[1], l[2], l[3]);
+        for (int e = 0; e < 4; ++e) {
+          const __half2 hh = __hmul2(x[e], d2);
+          const __half2 ll = __hfma2(x[e], d2, __hneg2(hh));
+          h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+          l[e] = *reinterpret_cast<const uint32_t*>(&ll);
         }
-        sts_v4(dst + off, hi);
-        sts_v4(dst + kKVBytes + off, lo);
+        hi = make_uint4(h[0], h[1], h[2], h[3]);
+        lo = make_uint4(l[0], l[1], l[2], l[3]);
       };
       for (int t = 0; t < t_count && ok; ++t) {
         const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
@@ -1005,13 +947,28 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
                                          mbar_wait(bar(bar_cempty), (t & 1) ^ 1, abort));
         if (!ok) break;
         const uint8_t* raw = smem + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
-#pragma unroll 2
-        for (int grp = 0; grp < kTileKeys / 8; ++grp) {
-          const int ra = grp * 8 + r0, rb = ra + 4;
-          convert(raw, ra, grp * kGroupBytes + off_a,
-                  kv == 0 || (key_t + ra >= lo_u && key_t + ra <= hi_u));
-          convert(raw, rb, grp * kGroupBytes + off_b,
-                  kv == 0 || (key_t + rb >= lo_u && key_t + rb <= hi_u));
+        const __half* rawd = reinterpret_cast<const __half*>(raw + kRawQsBytes);
+        // Eight items at a time: every load first, so that one shared-memory
+        // latency covers all eight (the stores below are compiler barriers).
+#pragma unroll 1
+        for (int g0 = 0; g0 < kTileKeys / 8; g0 += 4) {
+          uint2 qv[8];
+          __half2 dv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
+            qv[i] = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
+            dv[i] = __half2half2(rawd[r * 4 + (cc >> 2)]);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
+            uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+            if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) convert(qv[i], dv[i], hi, lo);
+            const uint32_t off = (g0 + i / 2) * kGroupBytes + ((i & 1) ? off_b : off_a);
+            sts_v4(dst + off, hi);
+            sts_v4(dst + kKVBytes + off, lo);
+          }
         }
         fence_proxy_async_smem();  // generic writes -> the tensor core's reads
         __syncwarp();

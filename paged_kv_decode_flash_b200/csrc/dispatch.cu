@@ -81,8 +81,8 @@ Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
       decode_tc_supported(kv_dtype, rows, d->num_blocks, d->num_kv_heads, d->block_size);
   if (pl.tensor_cores) {
     // One CTA per SM (one per group at least, and no more than the table's
-    // 128-key tiles could keep busy); the kernel shares them out among the
-    // groups in proportion to each group's visible tiles.
+    // 128-key tiles could keep busy); the kernel shares them out evenly
+    // among the (sequence, KV head) groups.
     const long long groups = (long long)d->num_seqs * d->num_kv_heads;
     const long long max_split = ceil_div((long long)d->max_blocks_per_seq * d->block_size, 128);
     pl.ctas = (int)std::max(groups, std::min<long long>(sms, groups * max_split));
