@@ -39,7 +39,10 @@
  *                 PA_KV_Q8_0: bytes [num_blocks][num_kv_heads][tile] with one
  *                   tile = int8 qs[block_size][head_dim] followed by
  *                   fp16 d[block_size][head_dim/32]; element value = qs * d of
- *                   its group of 32 consecutive head_dim elements
+ *                   its group of 32 consecutive head_dim elements; scales of
+ *                   keys that a query can see must be finite with |d| < 1024
+ *                   (true of any cache quantised from fp16 data, where
+ *                   d = amax / 127 <= 516): larger ones give non-finite rows
  *   block_table   int32 [num_seqs][max_blocks_per_seq]
  *   context_lens  int32 [num_seqs]
  * Supported: head_dim 128; block_size a multiple of 16 up to 128; n_query

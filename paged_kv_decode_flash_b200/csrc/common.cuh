@@ -37,6 +37,11 @@ struct DecodeParams {
   int num_splits;             // key splits per (seq, kv head) (CUDA-core kernel;
                               // tensor-core kernel: ceil(num_ctas / groups))
   int num_ctas;               // tensor-core kernel: CTAs of the (1-D) grid
+  int tiles_per_item;         // tensor-core kernel: 0 = the CTAs are shared
+                              // evenly among the (sequence, KV head) groups
+                              // (one wave); T > 0 = each group's 128-key tiles
+                              // are cut into items of T tiles, CTA c taking
+                              // item c % num_splits of group c / num_splits
   int blocks_per_split;       // logical blocks per split
   float* part_out;            // [B][S][nq*Hq][D]
   float* part_lse;            // [B][S][nq*Hq], natural log

@@ -10,7 +10,7 @@
 // left for the log-sum-exp merge.  Masks and block-table resolution follow
 // section "Bug 2: the drafter read freed memory".
 //
-// Hardware mapping (one CTA per SM, 12 warps):
+// Hardware mapping (one CTA per SM, 11 warps; 15 for the q8_0 cache):
 //   warps 0, 10 TMA producers for K and for V: resolve the block table and
 //               load whole 16-key chunks (two 64-column halves each, 128-byte
 //               swizzle) into separate rings of 128-key tiles (2-3 slots);
@@ -28,8 +28,8 @@
 //               plus one named barrier per group); when a row's reference
 //               maximum rises, its O column is rescaled in TMEM in place
 //               (thread = head_dim lane) before the tile's P is published.
-//   warps 11-14 (q8_0 cache only) converters: raw int8 tiles -> fp16 operand
-//               tiles (see below).
+//   warps 11-14 (q8_0 cache only) converters: raw int8 tiles -> exact fp16
+//               operand tiles (see below).
 // Putting keys and head_dim on the MMA's M side keeps the tensor core free of
 // padding even at 4-32 query rows.
 //
@@ -43,15 +43,27 @@
 // zero-filled in shared memory before the PV product (the NaN-poisoned
 // out-of-window blocks of the pages' regression test must not leak).
 //
-// Merge: every CTA counts itself in the arrival counter of its (sequence,
-// KV head) once its partial is written; the last one to arrive merges the
-// group's partials into the fp16 output rows (log-sum-exp weights, splits in
-// a fixed order) and resets the counter.  No CTA ever waits for another, and
-// a call is one launch.
+// q8_0 cache (int8 qs with one fp16 scale d per 32 head_dim elements): the
+// scale stays out of the operands, so that they remain exact without a
+// high/residual split.  K's operand is qs; S^T gets one TMEM accumulator per
+// scale group, and the softmax forms each score as the sum over the groups of
+// K's scale times the group's partial product, in fp32.  V's operand is
+// qs * 2^e, with d = m * 2^e split into its power of two and its mantissa m;
+// P gets one copy per scale group with the weights multiplied by that
+// group's m (then split into fp16 parts as above), and each group has its
+// own O^T accumulator, of which a head_dim lane reads only its own group's.
+// The softmax reads the scales of its keys from the cache (L2) a tile ahead.
 //
-// Every wait is bounded (sm100::mbar_wait): on a timeout the kernel raises
-// kFlagTimeout, drains its own copies and MMAs, frees TMEM and still takes
-// part in the merge (its rows count as empty).
+// Merge: every CTA writes its fp32 partial (O, lse).  With a cooperative
+// launch (every CTA resident) the CTAs of one (sequence, KV head) meet at a
+// bounded counter barrier and each merges a slice of the group's rows;
+// otherwise the last CTA of the group to arrive merges all of it.  Splits
+// are added in a fixed order (log-sum-exp weights), so results are
+// bit-reproducible.  A call is one launch.
+//
+// Every wait is bounded (sm100::mbar_wait and the group barrier): on a
+// timeout the kernel raises kFlagTimeout, drains its own copies and MMAs,
+// frees TMEM and still takes part in the merge (its rows count as empty).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -89,10 +101,9 @@ constexpr uint32_t kQ8ChunkBytes = kChunk * (kHeadDim + 8);         // 2176 B
 constexpr int kSoftmaxThreads = 128;           // per softmax warpgroup
 constexpr uint32_t kBarSetup = 1;              // named barrier: set-up done
 constexpr uint32_t kBarGroup0 = 2;             // named barriers 2.. : softmax groups
-constexpr int kPShift = 14;                    // weights scaled by 2^14 before fp16
 // A row's reference max is only raised when a score passes it by more than
-// kLazy (log2 units); scaled weights then stay below 2^(kPShift + kLazy),
-// inside fp16 range.
+// kLazy (log2 units); weights scaled by 2^kPShift (see Cfg) then stay below
+// 2^(kPShift + kLazy), inside fp16 range.
 constexpr float kLazy = 1.5f;
 
 enum : int {
@@ -108,21 +119,22 @@ enum : int {
   BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
   BAR_CKFULL = 31,  // q8_0: converted K tile written
   BAR_CKEMPTY = 32, // q8_0: converted K tile read by QK^T
-  BAR_CVFULL = 33,  // q8_0: converted V tile written
-  BAR_CVEMPTY = 34, // q8_0: converted V tile read by PV
-  BAR_COUNT = 35
+  BAR_CVFULL = 33,  // [2] q8_0: converted V tile written
+  BAR_CVEMPTY = 35, // [2] q8_0: converted V tile read by PV
+  BAR_COUNT = 37
 };
 constexpr int kBarSlots = 40;
 constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
 // NG softmax warpgroups of RW query rows each; NR = the MMA's N for S
 // (>= 16).  Warps: 0 K producer, 1 MMA issuer, 2 .. 4*NG+1 softmax, then the
-// V producer.
-// KS / VS slots in the K / V rings, PB buffers for P (two, so that the
-// softmax of tile t+1 never waits for PV(t)).  At 32 rows the two P buffers
-// take 32 KB and the V ring keeps two slots (measured: three V slots with
-// one P buffer is slower).  With one P buffer the softmax of tile t waits
-// for PV(t-1) before it stores P(t).
+// V producer (and, q8_0 only, four converter warps).
+// KS / VS slots in the K / V rings, PB buffers for P.  fp16: two P buffers,
+// so that the softmax of tile t+1 never waits for PV(t); at 32 rows they take
+// 32 KB and the V ring keeps two slots (measured: three V slots with one P
+// buffer is slower).  q8_0: raw rings of two slots each, one converted K tile,
+// two converted V tiles, and one P buffer that holds a P per scale group
+// (the softmax of tile t waits for PV(t-1) before it stores P(t)).
 template <int RW, int NG, bool Q8>
 struct Cfg {
   static constexpr int kGroups = NG;
@@ -130,24 +142,31 @@ struct Cfg {
   static constexpr int kConvWarp = kVWarp + 1;   // q8_0: first of 4 converter warps
   static constexpr int kThreads = 32 * (kVWarp + 1 + (Q8 ? 4 : 0));
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
-  // fp16: K/V rings of TMA-loaded tiles.  q8_0: rings of raw tiles (2 slots
-  // of kRawBytes) plus one converted K and one converted V tile, each an
-  // fp16 high part and an fp16 residual (2 * kKVBytes).
+  // q8_0: one S^T accumulator, one P and one O^T accumulator per group of 32
+  // head_dim elements that shares a scale; fp16: one of each.
+  static constexpr int kSG = Q8 ? kHeadDim / 32 : 1;
   static constexpr int KS = Q8 ? 2 : 3;
   static constexpr int VS = Q8 ? 2 : (NR > 16 ? 2 : 3);
-  static constexpr int PB = 2;
+  static constexpr int PB = Q8 ? 1 : 2;
+  static constexpr int CVS = 2;                  // q8_0: converted V slots
+  // Weights are scaled by 2^kPShift before they are split into fp16 parts.
+  // q8_0 multiplies them by a scale mantissa in [1, 2) as well, so it keeps
+  // one bit of headroom more.
+  static constexpr int kPShift = Q8 ? 13 : 14;
   static constexpr uint32_t kSlotBytes = Q8 ? kRawBytes : kKVBytes;
   static constexpr uint32_t kK = 0;                                 // K ring
   static constexpr uint32_t kV = KS * kSlotBytes;                   // V ring
-  static constexpr uint32_t kConvK = (KS + VS) * kSlotBytes;        // q8_0: K hi | K lo
-  static constexpr uint32_t kConvV = kConvK + (Q8 ? 2 * kKVBytes : 0);  // q8_0: V hi | V lo
-  static constexpr uint32_t kQ = kConvV + (Q8 ? 2 * kKVBytes : 0);
+  static constexpr uint32_t kConvK = (KS + VS) * kSlotBytes;        // q8_0: converted K
+  static constexpr uint32_t kConvV = kConvK + (Q8 ? kKVBytes : 0);  // q8_0: CVS converted V
+  static constexpr uint32_t kQ = kConvV + (Q8 ? CVS * kKVBytes : 0);
   static constexpr uint32_t kQHalf = NR * 128;
-  // P^T of one tile: 2*NR "rows" (the fp16 high parts of the NR query rows,
-  // then their residuals), so one MMA with N = 2*NR multiplies both.  Tile t
-  // uses buffer t % PB.
+  // P^T of one tile: per scale group 2*NR "rows" (the fp16 high parts of the
+  // NR query rows, then their residuals), the groups side by side, so that
+  // one MMA with N = kSG * 2 * NR multiplies all of them with each V step
+  // (V is read once).  Tile t uses buffer t % PB.
+  static constexpr int kPN = kSG * 2 * NR;  // N of the PV product
   static constexpr uint32_t kP = kQ + 2 * kQHalf;
-  static constexpr uint32_t kPBytes = kTileKeys * 2 * NR * 2;
+  static constexpr uint32_t kPBytes = kTileKeys * kPN * 2;
   static constexpr uint32_t kRed = kP + PB * kPBytes;               // float [2 grp][2][4][32]
   static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4 tiles][32 rows]
   static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
@@ -156,13 +175,16 @@ struct Cfg {
   static constexpr uint32_t kInfo = kBars + kBarSlots * 8;          // TileInfo [8]
   static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
   static constexpr uint32_t kTotal = kMisc + 64;
-  // TMEM columns: S^T[2] (NR each) then O^T (2*NR: high | residual).
-  static constexpr uint32_t kTmemUsed = 4 * NR;
+  // TMEM columns: S^T[2] (kSG accumulators of NR columns each), then O^T
+  // from column kTmemS (kSG accumulators of 2*NR: high | residual).
+  static constexpr uint32_t kTmemS = 2 * kSG * NR;
+  static constexpr uint32_t kTmemUsed = kTmemS + kSG * 2 * NR;
   static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
-                                        : kTmemUsed <= 128 ? 128 : 256;
+                                        : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
   static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
   static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
   static_assert(kConvK % 1024 == 0, "converted tiles sit on 1 KB swizzle atoms");
+  static_assert(kTmemUsed <= 512, "TMEM columns");
 };
 
 struct Misc {
@@ -197,6 +219,11 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
   return r;
 }
 __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
@@ -235,13 +262,22 @@ struct GroupOf {
   int s, kvh, split, splits, first;  // first: the group's first CTA
 };
 __device__ __forceinline__ GroupOf group_of(const DecodeParams& p, int c, int C) {
+  GroupOf r;
+  if (p.tiles_per_item > 0) {  // items: num_splits consecutive CTAs per group
+    const int g = c / p.num_splits;
+    r.s = g / p.num_kv_heads;
+    r.kvh = g % p.num_kv_heads;
+    r.splits = p.num_splits;
+    r.first = g * p.num_splits;
+    r.split = c - r.first;
+    return r;
+  }
   const int G = p.num_seqs * p.num_kv_heads;
   const long long E = (long long)C - G;
   auto cum = [&](int g) { return g + (int)(E * g / G); };
   int g = (int)((long long)c * G / C);
   while (g > 0 && cum(g) > c) --g;
   while (g + 1 < G && cum(g + 1) <= c) ++g;
-  GroupOf r;
   r.s = g / p.num_kv_heads;
   r.kvh = g % p.num_kv_heads;
   r.first = cum(g);
@@ -260,6 +296,26 @@ __device__ __forceinline__ long long q8_chunk_offset(const DecodeParams& p, int 
 __device__ __forceinline__ long long q8_scale_offset(const DecodeParams& p, int key0) {
   const int slot = key0 % p.block_size;
   return (long long)(p.block_size - slot) * kHeadDim + slot * 8;
+}
+
+// ... and of the four scales of one key (slot `slot` of its block) of q8_0
+// (block, head) tile `tile`.
+__device__ __forceinline__ long long q8_key_scales_offset(const DecodeParams& p, int tile, int slot) {
+  return (long long)tile * p.block_size * (kHeadDim + 8) + (long long)p.block_size * kHeadDim +
+         (long long)slot * 8;
+}
+
+// A q8_0 scale d (fp16 bits) as d = m * 2^e with 2^e the power of two of its
+// exponent field (2^-14 for zero and subnormal scales): 2^e as fp16 bits, and
+// the factor 2^-e that turns d into m (|m| in [1, 2), below 1 for subnormal
+// scales).  Both are exact.
+__device__ __forceinline__ uint16_t q8_scale_pow2_bits(uint16_t d) {
+  const uint16_t e = d & 0x7C00u;
+  return e != 0 ? e : (uint16_t)0x0400u;
+}
+__device__ __forceinline__ float q8_scale_mantissa(uint16_t d) {
+  const int E = max((int)((d >> 10) & 31u), 1);
+  return __half2float(__ushort_as_half(d)) * __int_as_float((127 + 15 - E) << 23);
 }
 
 // Eight signed bytes -> eight exact fp16 values, two per half2: byte b
@@ -554,7 +610,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       misc->g_splits = go.splits;
       misc->g_first = go.first;
     }
-    if (p.num_seqs == 1 && lane < kChunksPerTile) {
+    if (p.num_seqs == 1 && p.tiles_per_item == 0 && lane < kChunksPerTile) {
       const int ntg =
           (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
       const int tfg = go.split * (ntg / go.splits) + min(go.split, ntg % go.splits);
@@ -577,10 +633,11 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // ---- the head's visible keys and its tiles (uniform across the CTA) ------
   // The keys of (sequence s, KV head kvh) that any query token sees form
   // [lo_u, hi_u]; they are cut into 128-key tiles from `base`, and the S
-  // splits take contiguous runs of them, as even as whole tiles allow.  The
-  // partition depends only on the context lengths and the grid, so every
-  // call on the same inputs adds the same tiles in the same order: results
-  // are bit-reproducible.
+  // splits take contiguous runs of them (as even as whole tiles allow, or
+  // items of tiles_per_item tiles).  The partition depends only on the
+  // sequence's own context length and the shapes, so every call on the same
+  // inputs adds the same tiles in the same order: results are
+  // bit-reproducible.
   const int L = ld_nc_s32(p.context_lens + s);
   const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
   const SeqTiles st_ = seq_tiles(p, L);
@@ -588,9 +645,15 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   if (!context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size) && split == 0 && kvh == 0 &&
       threadIdx.x == 0)
     atomicOr(p.flags, kFlagBadLen);
-  const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
-  const int t_first = split * t_per + min(split, t_rem);
-  const int t_count = t_per + (split < t_rem ? 1 : 0);
+  int t_first, t_count;
+  if (p.tiles_per_item > 0) {  // item `split` of T tiles
+    t_first = split * p.tiles_per_item;
+    t_count = max(0, min(p.tiles_per_item, ntiles_h - t_first));
+  } else {  // the S CTAs of the group take contiguous runs, as even as whole tiles allow
+    const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
+    t_first = split * t_per + min(split, t_rem);
+    t_count = t_per + (split < t_rem ? 1 : 0);
+  }
 
   const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
   const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
@@ -615,8 +678,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       if (Q8) {
         mbar_init(bar(BAR_CKFULL), 2);
         mbar_init(bar(BAR_CKEMPTY), 1);
-        mbar_init(bar(BAR_CVFULL), 2);
-        mbar_init(bar(BAR_CVEMPTY), 1);
+        for (int i = 0; i < C::CVS; ++i) {
+          mbar_init(bar(BAR_CVFULL + i), 2);
+          mbar_init(bar(BAR_CVEMPTY + i), 1);
+        }
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(bar(BAR_SFULL + i), 1);
@@ -708,6 +773,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
                     src + off + q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk), kChunk * 8,
                     fb);
           bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off, kChunk * kHeadDim);
+          bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off +
+                               q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk),
+                           kChunk * 8);
         } else {
           tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
           tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
@@ -811,18 +879,21 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       // t_count (uniform), so the issuer reads no published tile information.
       if (lane == 0) {
         const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
-        const uint32_t id_pv = idesc_f16_f32(128, 2 * NR, true, true);
+        const uint32_t id_pv = idesc_f16_f32(128, C::kPN, true, true);
         // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
         // start-address field is the low 14 bits, addresses stay < 256 KB).
-        // q8_0: K and V are the converted tiles (fp16 high part, then the
-        // fp16 residual kKVBytes further), each multiplied and accumulated in
-        // turn into the same TMEM accumulator.
+        // q8_0: K and V are the converted tiles (exact fp16 images of the
+        // int8 values; V's rows also carry the power of two of their scales).
+        // S^T gets one accumulator per scale group g (head_dim 32g .. 32g+31,
+        // two steps of 16), which the softmax combines with K's scales; PV
+        // multiplies V with each group's P (the weights times V's scale
+        // mantissas) into that group's O^T accumulator.
         const uint64_t dK = smem_desc(Q8 ? sbase + C::kConvK : sKr, 16, kGroupBytes, kSwizzle128B);
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
         const uint64_t dV =
             smem_desc(Q8 ? sbase + C::kConvV : sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
-        const uint64_t dP = smem_desc(sP, 2 * NR * 16, 128, kSwizzleNone);
-        constexpr int kParts = Q8 ? 2 : 1;  // operand parts per product (high, residual)
+        const uint64_t dP = smem_desc(sP, C::kPN * 16, 128, kSwizzleNone);
+        constexpr int kSG = C::kSG;
         // QK(u) once K(u) is ready and the softmax took S(u-2) from its buffer.
         auto issue_qk = [&](int u) -> bool {
           const bool ready = Q8 ? mbar_wait(bar(BAR_CKFULL), u & 1, abort)
@@ -831,16 +902,13 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             return false;
           tc_fence_after();
           const uint64_t so = Q8 ? 0 : (uint64_t)((u % KS) * kKVBytes) >> 4;
-          const uint32_t d = tmem + (u % 2) * NR;
+          const uint32_t d = tmem + (u % 2) * kSG * NR;
+          constexpr int kSteps = kHeadDim / 16 / kSG;  // steps of 16 per accumulator
 #pragma unroll
-          for (int part = 0; part < kParts; ++part) {
-            const uint64_t po = (uint64_t)(part * kKVBytes) >> 4;
-#pragma unroll
-            for (int k = 0; k < kHeadDim / 16; ++k) {
-              const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
-              const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
-              tc_mma_f16_ss(d, dK + so + po + ko, dQ + qo, id_qk, part > 0 || k > 0);
-            }
+          for (int k = 0; k < kHeadDim / 16; ++k) {
+            const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
+            const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
+            tc_mma_f16_ss(d + (k / kSteps) * NR, dK + so + ko, dQ + qo, id_qk, k % kSteps != 0);
           }
           tc_commit(bar(BAR_SFULL + u % 2));
           tc_commit(bar(Q8 ? BAR_CKEMPTY : BAR_KEMPTY + u % KS));
@@ -855,25 +923,23 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         for (int t = 0; ok && t < t_count; ++t) {
           // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
           ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
-               (Q8 ? mbar_wait(bar(BAR_CVFULL), t & 1, abort)
+               (Q8 ? mbar_wait(bar(BAR_CVFULL + t % C::CVS), (t / C::CVS) & 1, abort)
                    : mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort));
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = Q8 ? 0 : (uint64_t)((t % VS) * kKVBytes) >> 4;
+          const uint64_t so = (uint64_t)((t % (Q8 ? C::CVS : VS)) * kKVBytes) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
-          const uint32_t d = tmem + 2 * NR;  // O^T accumulates over all tiles
+          // O^T accumulates over all tiles; q8_0: the kSG group accumulators
+          // are the consecutive column ranges of one N = kPN product.
+          const uint32_t d = tmem + C::kTmemS;
 #pragma unroll
-          for (int part = 0; part < kParts; ++part) {
-            const uint64_t pt = (uint64_t)(part * kKVBytes) >> 4;
-#pragma unroll
-            for (int k = 0; k < kTileKeys / 16; ++k) {
-              const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
-              const uint64_t po = (k * 2 * 2 * NR * 16) >> 4;
-              tc_mma_f16_ss(d, dV + so + pt + vo, dP + pb + po, id_pv, t > 0 || part > 0 || k > 0);
-            }
+          for (int k = 0; k < kTileKeys / 16; ++k) {
+            const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
+            const uint64_t po = (k * 2 * C::kPN * 16) >> 4;
+            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, t > 0 || k > 0);
           }
           tc_commit(bar(BAR_OFULL));
-          tc_commit(bar(Q8 ? BAR_CVEMPTY : BAR_VEMPTY + t % VS));
+          tc_commit(bar(Q8 ? BAR_CVEMPTY + t % C::CVS : BAR_VEMPTY + t % VS));
           npv = t + 1;
           if (t + 2 < t_count) {
             ok = issue_qk(t + 2);
@@ -893,87 +959,85 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     } else if (Q8 && warp >= C::kConvWarp) {
       // ===================== q8_0 converter (4 warps) ========================
       // Raw tile t (int8 qs, fp16 scales d per 32 elements) -> the fp16 K and
-      // V operand tiles.  Each element is x = qs * d; the operand holds its
-      // high part (x rounded to fp16) and, kKVBytes further, the residual
-      // x - high, which is an fp16 value as well, so that the tensor core
-      // sees x exactly.  The arithmetic is packed fp16 (two elements per
-      // instruction, no conversions).  Layout as the fp16 TMA boxes: [key/8][half][key%8]
-      // [64 dims], 128-byte swizzle.  V rows of keys outside [lo_u, hi_u]
-      // (masked or never loaded) are written as zeros: they must not reach
-      // the PV product.
-      // Warps kConvWarp, +1 convert K; warps +2, +3 convert V, so that K is
-      // never held up by V waiting for its operand buffer.  Thread = one
-      // 8-element column cc of every other 4th key: with 64 threads per
-      // stream, key r = 8 * group + rr with rr in {r0, r0 + 4}, so that the
-      // swizzled destination offset is constant up to the key group.
+      // V operand tiles, exactly: K's operand is qs itself (every integer
+      // below 2048 is an fp16 value; K's scales are applied to the per-group
+      // scores in the softmax), V's is qs * 2^e with 2^e the power of two of
+      // the element's scale d = m * 2^e (exact for |d| < 1024: at most 7
+      // significant bits above 2^-24); the mantissa m goes into that group's
+      // P.  The arithmetic is packed fp16 (two elements per instruction).
+      // Layout as the fp16 TMA boxes: [key/8][half][key%8][64 dims], 128-byte
+      // swizzle.  V rows of keys outside [lo_u, hi_u] (masked or never
+      // loaded) are written as zeros: they must not reach the PV product.
+      // Warps kConvWarp, +1 convert K (one operand tile); warps +2, +3
+      // convert V (two operand tiles), so that K is never held up by V
+      // waiting for its operand buffer.  Thread = one 8-element column cc of
+      // every other 4th key: with 64 threads per stream, key r = 8 * group +
+      // rr with rr in {r0, r0 + 4}, so that the swizzled destination offset is
+      // constant up to the key group.
       const int kv = (warp - C::kConvWarp) >> 1;  // 0: K, 1: V
       const int ct = threadIdx.x - 32 * (C::kConvWarp + 2 * kv);  // 0 .. 63
       const int cc = ct & 15, r0 = ct >> 4;      // column, first key (0 .. 3)
       const uint32_t col_off = (cc >> 3) * kAtomBytes;
       const uint32_t off_a = col_off + r0 * 128 + (((cc & 7) ^ r0) << 4);
       const uint32_t off_b = col_off + (r0 + 4) * 128 + (((cc & 7) ^ (r0 + 4)) << 4);
-      const int NSl = kv == 0 ? KS : VS;
+      const int NSl = kv == 0 ? KS : VS;        // raw slots
+      const int NCs = kv == 0 ? 1 : C::CVS;     // operand slots
       const uint32_t bar_full = kv == 0 ? BAR_KFULL : BAR_VFULL;
       const uint32_t bar_raw_empty = kv == 0 ? BAR_KEMPTY : BAR_VEMPTY;
       const uint32_t bar_cfull = kv == 0 ? BAR_CKFULL : BAR_CVFULL;
       const uint32_t bar_cempty = kv == 0 ? BAR_CKEMPTY : BAR_CVEMPTY;
-      const uint32_t dst = sbase + (kv == 0 ? C::kConvK : C::kConvV);
       int n = 0;
       bool ok = true;
-      // One 8-element item: x = qs * d split into an fp16 high part and an
-      // fp16 residual (zeros for a V row no query row may see).  The high
-      // part is x rounded to fp16; qs * d has at most 18 significant bits
-      // and is a multiple of 2^-24 (the smallest fp16 step), so the residual
-      // x - high is an fp16 value too and the fused multiply-add gives it
-      // exactly: high + residual = x.
-      auto convert = [&](uint2 q, __half2 d2, uint4& hi, uint4& lo) {
+      // Eight int8 -> eight fp16 values times the power of two p2 (1 for K).
+      auto convert = [&](uint2 q, __half2 p2) -> uint4 {
         __half2 x[4];
         q8_to_half8(q, x);
-        uint32_t h[4], l[4];
+        uint32_t h[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const __half2 hh = __hmul2(x[e], d2);
-          const __half2 ll = __hfma2(x[e], d2, __hneg2(hh));
-          h[e] = *reinterpret_cast<const uint32_t*>(&hh);
-          l[e] = *reinterpret_cast<const uint32_t*>(&ll);
+          const __half2 y = kv == 0 ? x[e] : __hmul2(x[e], p2);
+          h[e] = *reinterpret_cast<const uint32_t*>(&y);
         }
-        hi = make_uint4(h[0], h[1], h[2], h[3]);
-        lo = make_uint4(l[0], l[1], l[2], l[3]);
+        return make_uint4(h[0], h[1], h[2], h[3]);
       };
       for (int t = 0; t < t_count && ok; ++t) {
         const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
-        const int rs = t % NSl;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort) &&
-                                         mbar_wait(bar(bar_cempty), (t & 1) ^ 1, abort));
+        const int rs = t % NSl, cs_ = t % NCs;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort) &&
+                            mbar_wait(bar(bar_cempty + cs_), ((t / NCs) & 1) ^ 1, abort));
         if (!ok) break;
         const uint8_t* raw = smem + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
-        const __half* rawd = reinterpret_cast<const __half*>(raw + kRawQsBytes);
+        const uint16_t* rawd = reinterpret_cast<const uint16_t*>(raw + kRawQsBytes);
+        const uint32_t dst = sbase + (kv == 0 ? C::kConvK : C::kConvV + cs_ * kKVBytes);
         // Eight items at a time: every load first, so that one shared-memory
         // latency covers all eight (the stores below are compiler barriers).
 #pragma unroll 1
         for (int g0 = 0; g0 < kTileKeys / 8; g0 += 4) {
           uint2 qv[8];
-          __half2 dv[8];
+          uint16_t dv[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
             qv[i] = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
-            dv[i] = __half2half2(rawd[r * 4 + (cc >> 2)]);
+            dv[i] = kv == 0 ? (uint16_t)0 : rawd[r * 4 + (cc >> 2)];
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
-            uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
-            if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) convert(qv[i], dv[i], hi, lo);
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) {
+              const __half p2 = __ushort_as_half(q8_scale_pow2_bits(dv[i]));
+              x = convert(qv[i], __halves2half2(p2, p2));
+            }
             const uint32_t off = (g0 + i / 2) * kGroupBytes + ((i & 1) ? off_b : off_a);
-            sts_v4(dst + off, hi);
-            sts_v4(dst + kKVBytes + off, lo);
+            sts_v4(dst + off, x);
           }
         }
         fence_proxy_async_smem();  // generic writes -> the tensor core's reads
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(bar(bar_cfull));
+          mbar_arrive(bar(bar_cfull + cs_));
           mbar_arrive(bar(bar_raw_empty + rs));
         }
         n = t + 1;
@@ -1026,25 +1090,87 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       float m_lane = -INFINITY;
       bool ok = true;
       const int end_t = t_count;  // tiles of this CTA (local t -> tile t_first + t)
-      // O^T accumulates in TMEM over every tile (columns 2NR.. : the high
-      // parts of the rows, then their residuals).  When a row's reference
-      // rises at tile t, its O column is scaled by alpha in place, after
-      // PV(t-1) has finished and before P(t) is published.  S(t) in TMEM
-      // implies that PV(t-2) has finished (the issuer commits S(t) after
-      // issuing PV(t-2)), so P buffer t % 2 is free again.
-      const uint32_t o_hi = tmem + lane_off + 2 * NR + row0, o_lo = o_hi + NR;
+      // O^T accumulates in TMEM over every tile (from column kTmemS: the
+      // high parts of the rows, then their residuals).  When a row's
+      // reference rises at tile t, its O column is scaled by alpha in place,
+      // after PV(t-1) has finished and before P(t) is published.  S(t) in
+      // TMEM implies that PV(t-2) has finished (the issuer commits S(t) after
+      // issuing PV(t-2)), so with two P buffers buffer t % 2 is free again;
+      // with one (q8_0) the softmax waits for PV(t-1) before storing P(t).
+      // q8_0: this thread's lanes of O^T are head_dim elements 32*q4 ..
+      // 32*q4 + 31, i.e. scale group q4: only that group's accumulator is
+      // read (and rescaled) here.
+      const uint32_t o_hi = tmem + lane_off + C::kTmemS + (Q8 ? q4 * 2 * NR : 0) + row0;
+      const uint32_t o_lo = o_hi + NR;
+      constexpr int kSG = C::kSG;
+      // q8_0: the K and V scales of this thread's key (4 fp16 each), read
+      // from the cache (an L2 hit: the tile's bulk copies brought them) one
+      // tile ahead; zeros for a key no row sees.
+      auto fetch_scales = [&](int u) -> uint4 {
+        uint4 sc = make_uint4(0, 0, 0, 0);
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_INFO + u % kInfoSlots),
+                                                     (u / kInfoSlots) & 1, abort));
+        if (ok) {
+          const int key = base + (t_first + u) * kTileKeys + j;
+          const int tix = info[u % kInfoSlots].row8[j / kChunk];  // (block, head) tile, -1: not loaded
+          if (tix >= 0 && key >= lo_u && key <= hi_u) {
+            const long long off = q8_key_scales_offset(p, tix, key % p.block_size);
+            const uint2 a = ldg_nc_v2(static_cast<const uint8_t*>(p.k) + off);
+            const uint2 b = ldg_nc_v2(static_cast<const uint8_t*>(p.v) + off);
+            sc = make_uint4(a.x, a.y, b.x, b.y);
+          }
+        }
+        return sc;
+      };
+      uint4 sc_next = make_uint4(0, 0, 0, 0);
+      if constexpr (Q8) {
+        if (end_t > 0) sc_next = fetch_scales(0);
+      }
       for (int t = 0; t < end_t; ++t) {
         const int gt = t_first + t;  // tile number of local tile t
         const int sb = t % 2, st = t % VS;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+        float mv[kSG];  // q8_0: V's scale mantissas of this key, per group
         float sv[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) sv[r] = 0.f;
-        if (ok) {
-          tc_fence_after();
-          tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
-          tmem_ld_wait();
-          tc_fence_before();
+        if constexpr (Q8) {
+          const uint4 sc = sc_next;
+          if (t + 1 < end_t) sc_next = fetch_scales(t + 1);
+          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+          // Score = sum over the scale groups of K's scale times the group's
+          // partial product (fp32, groups in order).
+          float sg[kSG][RW];
+#pragma unroll
+          for (int q = 0; q < kSG; ++q)
+#pragma unroll
+            for (int r = 0; r < RW; ++r) sg[q][r] = 0.f;
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int q = 0; q < kSG; ++q)
+              tmem_ld<RW>(tmem + lane_off + sb * kSG * NR + q * NR + row0, sg[q]);
+            tmem_ld_wait();
+            tc_fence_before();
+          }
+          const uint32_t kw[2] = {sc.x, sc.y}, vw[2] = {sc.z, sc.w};
+#pragma unroll
+          for (int q = 0; q < kSG; ++q) {
+            const uint16_t kd = (uint16_t)(kw[q / 2] >> (16 * (q % 2)));
+            const uint16_t vd = (uint16_t)(vw[q / 2] >> (16 * (q % 2)));
+            const float dk = __half2float(__ushort_as_half(kd));
+            mv[q] = q8_scale_mantissa(vd);
+#pragma unroll
+            for (int r = 0; r < RW; ++r) sv[r] = q == 0 ? dk * sg[0][r] : fmaf(dk, sg[q][r], sv[r]);
+          }
+        } else {
+          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
+          mv[0] = 1.f;
+          if (ok) {
+            tc_fence_after();
+            tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
+            tmem_ld_wait();
+            tc_fence_before();
+          }
         }
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(bar(BAR_SEMPTY + sb));
@@ -1083,7 +1209,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             xmax = fmaxf(xmax, x[r]);
           }
         }
-        const bool exceed = xmax > (float)kPShift + kLazy;
+        const bool exceed = xmax > (float)C::kPShift + kLazy;
         // Reconverge before the group barrier: a warp that arrives diverged
         // (after lane-predicated code) makes the barrier several times slower
         // (measured: 61k verify 122 -> 67 us per call).
@@ -1112,7 +1238,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           // 2^(cs (s - m_new) + kPShift).
           const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
           const float bias_l =
-              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
+              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)C::kPShift);
           m_lane = m_new;
           if (lane < RW) {
             bc[lane] = bias_l;
@@ -1153,21 +1279,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           }
         }
 
-        // Scaled weights (2^-inf = 0 for keys a row does not see), split
-        // into an fp16 high part (the weight truncated to 11 significant
-        // bits: exact in fp16 over the weights' range) and an fp16 residual.
-        uint32_t phi[RW / 2], plo[RW / 2];
+        // Scaled weights (2^-inf = 0 for keys a row does not see).
+        float pw[RW];
 #pragma unroll
-        for (int r = 0; r < RW; r += 2) {
-          const float p0 = fast_exp2(x[r]), p1 = fast_exp2(x[r + 1]);
-          lpart[r] += p0;
-          lpart[r + 1] += p1;
-          const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-          const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-          const __half2 h = __floats2half2_rn(h0, h1);
-          const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
-          phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-          plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+        for (int r = 0; r < RW; ++r) {
+          pw[r] = fast_exp2(x[r]);
+          lpart[r] += pw[r];
         }
 
         // A key no row can see must not reach the PV product: zero its V
@@ -1185,26 +1302,49 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             }
           }
         }
+        // One P buffer: PV(t-1) must have read it before P(t) goes in.
+        if (PB == 1 && t > 0) {
+          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (t - 1) & 1, abort));
+          if (ok) tc_fence_after();
+        }
         if (ok) {
-          // P^T as no-swizzle MN-major core matrices [key/8][row'/8][key%8]
-          // [row'%8] with row' < NR the high parts and row' >= NR the
-          // residuals, in P buffer t % PB.
-          const uint32_t pbuf = sP + (t % PB) * C::kPBytes;
-          const uint32_t kb = (j >> 3) * (2 * NR / 8) * 128 + (j & 7) * 16;
+          // P^T as no-swizzle MN-major core matrices [key/8][n/8][key%8]
+          // [n%8], n = group * 2NR + row' with row' < NR the high parts and
+          // row' >= NR the residuals, in P buffer t % PB.  Each weight (times
+          // V's scale mantissa of the group, q8_0) is split into an fp16 high
+          // part (truncated to 11 significant bits: exact in fp16 over the
+          // weights' range) and an fp16 residual.
+          const uint32_t kb = (j >> 3) * (C::kPN / 8) * 128 + (j & 7) * 16;
           constexpr uint32_t lo_off = (NR / 8) * 128;
-          if constexpr (RW >= 8) {
 #pragma unroll
-            for (int r8 = 0; r8 < RW / 8; ++r8) {
-              const uint32_t off = kb + ((row0 / 8) + r8) * 128;
-              sts_v4(pbuf + off,
-                     make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
-              sts_v4(pbuf + lo_off + off,
-                     make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
+          for (int q = 0; q < kSG; ++q) {
+            const uint32_t pbuf = sP + (t % PB) * C::kPBytes + q * (2 * NR / 8) * 128;
+            uint32_t phi[RW / 2], plo[RW / 2];
+#pragma unroll
+            for (int r = 0; r < RW; r += 2) {
+              const float p0 = Q8 ? pw[r] * mv[q] : pw[r];
+              const float p1 = Q8 ? pw[r + 1] * mv[q] : pw[r + 1];
+              const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+              const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+              const __half2 h = __floats2half2_rn(h0, h1);
+              const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
+              phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
+              plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
             }
-          } else {  // four rows: half of one 16-byte core-matrix row
-            const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
-            sts_v2(pbuf + off, phi[0], phi[1]);
-            sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
+            if constexpr (RW >= 8) {
+#pragma unroll
+              for (int r8 = 0; r8 < RW / 8; ++r8) {
+                const uint32_t off = kb + ((row0 / 8) + r8) * 128;
+                sts_v4(pbuf + off,
+                       make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
+                sts_v4(pbuf + lo_off + off,
+                       make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
+              }
+            } else {  // four rows: half of one 16-byte core-matrix row
+              const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
+              sts_v2(pbuf + off, phi[0], phi[1]);
+              sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
+            }
           }
           fence_proxy_async_smem();
         }
@@ -1256,7 +1396,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         p.part_lse[part_base + row0 + lane] =
             bad ? __int_as_float(0x7fc00000)
             : (!aborted && l > 0.f)
-                ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
+                ? (fmaf(cs, m_lane, -(float)C::kPShift) + log2f(l)) * 0.69314718055994531f
                 : -INFINITY;
       }
     }

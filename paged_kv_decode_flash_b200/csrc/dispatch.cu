@@ -23,6 +23,10 @@ namespace {
 constexpr int kCtasPerSm = 2;           // CUDA-core kernel: resident CTAs per SM aimed for
 constexpr int kMaxTargetCtas = 4096;    // device-independent bound used to size workspaces
 constexpr int kMinKeysPerSplit = 128;   // a split below this is all overhead
+// Tensor-core kernel, many (sequence, KV head) groups: items of at least this
+// many 128-key tiles, sized for about kItemWaves waves of CTAs.
+constexpr int kMinItemTiles = 16;
+constexpr int kItemWaves = 4;
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -80,13 +84,29 @@ Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
   pl.tensor_cores =
       decode_tc_supported(kv_dtype, rows, d->num_blocks, d->num_kv_heads, d->block_size);
   if (pl.tensor_cores) {
-    // One CTA per SM (one per group at least, and no more than the table's
-    // 128-key tiles could keep busy); the kernel shares them out evenly
-    // among the (sequence, KV head) groups.
     const long long groups = (long long)d->num_seqs * d->num_kv_heads;
     const long long max_split = ceil_div((long long)d->max_blocks_per_seq * d->block_size, 128);
-    pl.ctas = (int)std::max(groups, std::min<long long>(sms, groups * max_split));
-    pl.splits = (int)ceil_div(pl.ctas, groups);
+    if (groups * 4 > sms) {
+      // Many groups (a batch): an even share of the SMs would give a long
+      // sequence no more CTAs than a short one.  Instead every group's tiles
+      // are cut into items of T tiles, T from the shapes alone (so that a
+      // sequence's split, and every bit of its output, depends only on its
+      // own length), one CTA per item over about kItemWaves waves; the
+      // hardware hands each free SM the next item, and a group's items past
+      // its length leave at once.
+      const long long T = std::max<long long>(
+          kMinItemTiles, ceil_div(max_split * groups, (long long)kItemWaves * sms));
+      pl.splits = (int)ceil_div(max_split, T);
+      pl.ctas = (int)(groups * pl.splits);
+      pl.tiles_per_item = (int)T;
+    } else {
+      // One CTA per SM (one per group at least, and no more than the
+      // table's 128-key tiles could keep busy); the kernel shares them out
+      // evenly among the (sequence, KV head) groups.
+      pl.ctas = (int)std::max(groups, std::min<long long>(sms, groups * max_split));
+      pl.splits = (int)ceil_div(pl.ctas, groups);
+      pl.tiles_per_item = 0;
+    }
     pl.blocks_per_split = (int)ceil_div(d->max_blocks_per_seq, pl.splits);
   } else {
     pl.splits = plan_splits(d, (long long)sms * kCtasPerSm, true, &pl.blocks_per_split);
@@ -154,6 +174,7 @@ int enqueue_decode(const pa_dims* d, const Plan& plan, const void* q, const void
   p.scale_log2 = scale * 1.4426950408889634f;
   p.num_splits = plan.splits;
   p.num_ctas = plan.ctas;
+  p.tiles_per_item = plan.tiles_per_item;
   p.blocks_per_split = plan.blocks_per_split;
   p.part_out = reinterpret_cast<float*>(ws + w.part_out);
   p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);

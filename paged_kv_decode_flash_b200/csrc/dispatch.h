@@ -17,6 +17,7 @@ struct Plan {
   int splits, blocks_per_split;
   int ctas;  // tensor-core kernel: CTAs of the grid (the device shares them out
              // among the (sequence, KV head) groups); splits = ceil(ctas / groups)
+  int tiles_per_item;  // tensor-core kernel: 0, or the item size of a batched grid
 };
 
 // Workspace: status header | arrival counters | split partial outputs |

@@ -185,6 +185,39 @@ def test_sequence_independent_of_neighbours(B):
     assert np.array_equal(out_a[1].view(np.uint16), out_b[1].view(np.uint16))
 
 
+@pytest.mark.parametrize("dt", [gen.KV_FP16, gen.KV_Q8_0])
+def test_batched_items_every_row(B, orc, dt):
+    """Many (sequence, KV head) groups: each group's tiles are cut into
+    fixed-size items over several waves of CTAs, and the last CTA of a group
+    to finish merges it.  Ragged lengths (one shorter than a tile, one with
+    an item boundary inside), every row against the oracle."""
+    lens = (3000, 77, 2049, 1, 2500, 640)
+    case = gen.make_case(seed=60 + dt, context_lens=tuple(max(l, 2) for l in lens), n_query=2,
+                         num_q_heads=32, num_kv_heads=8, causal=1, kv_dtype=dt, spike_frac=0.002,
+                         spike_gain=5.0)
+    dec = B.PagedDecode.for_case(case)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert case.num_seqs * case.num_kv_heads * 4 > sms  # the item grid
+    assert dec.num_splits(dt) > 1
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, f"batched items dt={dt}")
+
+
+def test_batched_items_sequence_independent_of_neighbours(B):
+    """The item size comes from the shapes alone: other sequences' lengths
+    and data do not change a sequence's output by a bit."""
+    a = gen.make_case(seed=61, context_lens=(2500, 3900, 300, 4000, 10), n_query=4,
+                      num_q_heads=32, num_kv_heads=8, causal=1, max_blocks_per_seq=260)
+    out_a, _ = run(B, a)
+    b = gen.Case(**a.__dict__)
+    b.context_lens = a.context_lens.copy()
+    b.context_lens[0], b.context_lens[2], b.context_lens[4] = 4100, 9, 3333
+    b.q = a.q.copy(); b.q[3] = -a.q[3]
+    out_b, _ = run(B, b)
+    assert np.array_equal(out_a[1].view(np.uint16), out_b[1].view(np.uint16))
+
+
 def test_batch_matches_each_sequence_alone(B, orc):
     case = gen.make_case(seed=11, context_lens=(900, 33, 2500, 8), n_query=2,
                          num_q_heads=8, num_kv_heads=2, causal=1)
