@@ -10,7 +10,7 @@
 // left for the log-sum-exp merge.  Masks and block-table resolution follow
 // section "Bug 2: the drafter read freed memory".
 //
-// Hardware mapping (one CTA per SM, 11 warps; 15 for the q8_0 cache):
+// Hardware mapping (one CTA per SM, 11 warps; 19 for the q8_0 cache):
 //   warps 0, 10 TMA producers for K and for V: resolve the block table and
 //               load whole 16-key chunks (two 64-column halves each, 128-byte
 //               swizzle) into separate rings of 128-key tiles (2-3 slots);
@@ -28,7 +28,7 @@
 //               plus one named barrier per group); when a row's reference
 //               maximum rises, its O column is rescaled in TMEM in place
 //               (thread = head_dim lane) before the tile's P is published.
-//   warps 11-14 (q8_0 cache only) converters: raw int8 tiles -> exact fp16
+//   warps 11-18 (q8_0 cache only) converters: raw int8 tiles -> exact fp16
 //               operand tiles (see below).
 // Putting keys and head_dim on the MMA's M side keeps the tensor core free of
 // padding even at 4-32 query rows.
@@ -139,8 +139,9 @@ template <int RW, int NG, bool Q8>
 struct Cfg {
   static constexpr int kGroups = NG;
   static constexpr int kVWarp = 2 + NG * 4;      // the V producer's warp
-  static constexpr int kConvWarp = kVWarp + 1;   // q8_0: first of 4 converter warps
-  static constexpr int kThreads = 32 * (kVWarp + 1 + (Q8 ? 4 : 0));
+  static constexpr int kConvWarp = kVWarp + 1;   // q8_0: first converter warp
+  static constexpr int kConvWarps = 4;           // q8_0: converter warps per stream (K, V)
+  static constexpr int kThreads = 32 * (kVWarp + 1 + (Q8 ? 2 * kConvWarps : 0));
   static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
   // q8_0: one S^T accumulator, one P and one O^T accumulator per group of 32
   // head_dim elements that shares a scale; fp16: one of each.
@@ -230,6 +231,20 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
+}
+// Shared-memory loads by 32-bit shared address (issued in program order with
+// the other volatile shared-memory accesses).
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t r;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
+  return r;
 }
 __device__ __forceinline__ void sts_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
@@ -668,18 +683,18 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   } else if (warp == 0) {
     // ======================= K producer (also sets up the barriers) ========
     if (lane == 0) {
-      // q8_0: the raw K (V) slots are released by the 2 K (V) converter warps.
+      // q8_0: the raw K (V) slots are released by the K (V) converter warps.
       for (int i = 0; i < kMaxStages; ++i) {
         mbar_init(bar(BAR_KFULL + i), 1);
-        mbar_init(bar(BAR_KEMPTY + i), Q8 ? 2 : 1);
+        mbar_init(bar(BAR_KEMPTY + i), Q8 ? C::kConvWarps : 1);
         mbar_init(bar(BAR_VFULL + i), 1);
-        mbar_init(bar(BAR_VEMPTY + i), Q8 ? 2 : 1);
+        mbar_init(bar(BAR_VEMPTY + i), Q8 ? C::kConvWarps : 1);
       }
       if (Q8) {
-        mbar_init(bar(BAR_CKFULL), 2);
+        mbar_init(bar(BAR_CKFULL), C::kConvWarps);
         mbar_init(bar(BAR_CKEMPTY), 1);
         for (int i = 0; i < C::CVS; ++i) {
-          mbar_init(bar(BAR_CVFULL + i), 2);
+          mbar_init(bar(BAR_CVFULL + i), C::kConvWarps);
           mbar_init(bar(BAR_CVEMPTY + i), 1);
         }
       }
@@ -874,9 +889,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       // ===================== MMA issuer ======================================
       // One thread, in a fixed order: QK(0), QK(1), then PV(t), QK(t+2) for
       // t = 0, 1, ...  A commit completes once every MMA this thread issued
-      // before it has finished, so S(t) in TMEM also means that O(t-2) is:
-      // the softmax waits for one barrier per tile.  The number of tiles is
-      // t_count (uniform), so the issuer reads no published tile information.
+      // before it has finished, so S(t) in TMEM also means that O(t-2) is.
+      // The number of tiles is t_count (uniform), so the issuer reads no
+      // published tile information.
       if (lane == 0) {
         const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
         const uint32_t id_pv = idesc_f16_f32(128, C::kPN, true, true);
@@ -957,7 +972,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       __syncwarp();
       __syncthreads();  // (A)
     } else if (Q8 && warp >= C::kConvWarp) {
-      // ===================== q8_0 converter (4 warps) ========================
+      // ===================== q8_0 converters =================================
       // Raw tile t (int8 qs, fp16 scales d per 32 elements) -> the fp16 K and
       // V operand tiles, exactly: K's operand is qs itself (every integer
       // below 2048 is an fp16 value; K's scales are applied to the per-group
@@ -968,18 +983,27 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       // Layout as the fp16 TMA boxes: [key/8][half][key%8][64 dims], 128-byte
       // swizzle.  V rows of keys outside [lo_u, hi_u] (masked or never
       // loaded) are written as zeros: they must not reach the PV product.
-      // Warps kConvWarp, +1 convert K (one operand tile); warps +2, +3
-      // convert V (two operand tiles), so that K is never held up by V
-      // waiting for its operand buffer.  Thread = one 8-element column cc of
-      // every other 4th key: with 64 threads per stream, key r = 8 * group +
-      // rr with rr in {r0, r0 + 4}, so that the swizzled destination offset is
-      // constant up to the key group.
-      const int kv = (warp - C::kConvWarp) >> 1;  // 0: K, 1: V
-      const int ct = threadIdx.x - 32 * (C::kConvWarp + 2 * kv);  // 0 .. 63
-      const int cc = ct & 15, r0 = ct >> 4;      // column, first key (0 .. 3)
-      const uint32_t col_off = (cc >> 3) * kAtomBytes;
-      const uint32_t off_a = col_off + r0 * 128 + (((cc & 7) ^ r0) << 4);
-      const uint32_t off_b = col_off + (r0 + 4) * 128 + (((cc & 7) ^ (r0 + 4)) << 4);
+      // The first kConvWarps converter warps convert K (one operand tile),
+      // the next kConvWarps convert V (two operand tiles), so that K is never
+      // held up by V waiting for its operand buffer.  Thread ct of a
+      // stream's kCT takes the 16-byte column chunk c16 = ct % 8 (head_dim
+      // 16*c16 .. +15, half of one scale group) of keys r = ct / 8 + kRS*k:
+      // one 16-byte load and two 16-byte stores per key, the swizzled
+      // destination offset constant up to the key group, no bank conflicts on
+      // either side.
+      constexpr int kCT = 32 * C::kConvWarps;   // threads per stream
+      constexpr int kRS = kCT / 8;              // key stride between a thread's keys
+      constexpr int kKeysPer = kTileKeys / kRS; // keys per thread per tile
+      const int kv = (warp - C::kConvWarp) / C::kConvWarps;  // 0: K, 1: V
+      const int ct = threadIdx.x - 32 * (C::kConvWarp + C::kConvWarps * kv);  // 0 .. kCT-1
+      const int c16 = ct & 7, r0 = ct >> 3;      // column chunk, first key
+      const int r08 = r0 & 7;                    // its row within a key group
+      // destination of the two 8-element halves: chunk cc = 2*c16 + e of the
+      // key's 256-byte row, i.e. half cc / 8, 16-byte slot (cc % 8) ^ (key % 8)
+      const uint32_t dst_a = (r0 >> 3) * kGroupBytes + ((2 * c16) >> 3) * kAtomBytes + r08 * 128 +
+                             ((((2 * c16) & 7) ^ r08) << 4);
+      const uint32_t dst_b = (r0 >> 3) * kGroupBytes + ((2 * c16 + 1) >> 3) * kAtomBytes +
+                             r08 * 128 + ((((2 * c16 + 1) & 7) ^ r08) << 4);
       const int NSl = kv == 0 ? KS : VS;        // raw slots
       const int NCs = kv == 0 ? 1 : C::CVS;     // operand slots
       const uint32_t bar_full = kv == 0 ? BAR_KFULL : BAR_VFULL;
@@ -989,9 +1013,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       int n = 0;
       bool ok = true;
       // Eight int8 -> eight fp16 values times the power of two p2 (1 for K).
-      auto convert = [&](uint2 q, __half2 p2) -> uint4 {
+      auto convert = [&](uint32_t w0, uint32_t w1, __half2 p2) -> uint4 {
         __half2 x[4];
-        q8_to_half8(q, x);
+        q8_to_half8(make_uint2(w0, w1), x);
         uint32_t h[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -1007,31 +1031,33 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
                         mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort) &&
                             mbar_wait(bar(bar_cempty + cs_), ((t / NCs) & 1) ^ 1, abort));
         if (!ok) break;
-        const uint8_t* raw = smem + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
-        const uint16_t* rawd = reinterpret_cast<const uint16_t*>(raw + kRawQsBytes);
+        const uint32_t raw = sbase + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
+        const uint32_t src = raw + r0 * kHeadDim + c16 * 16;                 // key r0, chunk c16
+        const uint32_t srcd = raw + kRawQsBytes + r0 * 8 + (c16 >> 1) * 2;  // its scale
         const uint32_t dst = sbase + (kv == 0 ? C::kConvK : C::kConvV + cs_ * kKVBytes);
-        // Eight items at a time: every load first, so that one shared-memory
-        // latency covers all eight (the stores below are compiler barriers).
+        // Four keys at a time: every load first, so that one shared-memory
+        // latency covers all four.
 #pragma unroll 1
-        for (int g0 = 0; g0 < kTileKeys / 8; g0 += 4) {
-          uint2 qv[8];
-          uint16_t dv[8];
+        for (int k0 = 0; k0 < kKeysPer; k0 += 4) {
+          uint4 qv[4];
+          uint16_t dv[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
-            qv[i] = *reinterpret_cast<const uint2*>(raw + r * kHeadDim + cc * 8);
-            dv[i] = kv == 0 ? (uint16_t)0 : rawd[r * 4 + (cc >> 2)];
+          for (int i = 0; i < 4; ++i) {
+            qv[i] = lds_v4(src + (k0 + i) * kRS * kHeadDim);
+            dv[i] = kv == 0 ? (uint16_t)0 : lds_u16(srcd + (k0 + i) * kRS * 8);
           }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = (g0 + i / 2) * 8 + r0 + (i & 1) * 4;
-            uint4 x = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < 4; ++i) {
+            const int r = (k0 + i) * kRS + r0;
+            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
             if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) {
               const __half p2 = __ushort_as_half(q8_scale_pow2_bits(dv[i]));
-              x = convert(qv[i], __halves2half2(p2, p2));
+              const __half2 p22 = __halves2half2(p2, p2);
+              xa = convert(qv[i].x, qv[i].y, p22);
+              xb = convert(qv[i].z, qv[i].w, p22);
             }
-            const uint32_t off = (g0 + i / 2) * kGroupBytes + ((i & 1) ? off_b : off_a);
-            sts_v4(dst + off, x);
+            sts_v4(dst + (k0 + i) * (kRS / 8) * kGroupBytes + dst_a, xa);
+            sts_v4(dst + (k0 + i) * (kRS / 8) * kGroupBytes + dst_b, xb);
           }
         }
         fence_proxy_async_smem();  // generic writes -> the tensor core's reads
@@ -1093,10 +1119,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       // O^T accumulates in TMEM over every tile (from column kTmemS: the
       // high parts of the rows, then their residuals).  When a row's
       // reference rises at tile t, its O column is scaled by alpha in place,
-      // after PV(t-1) has finished and before P(t) is published.  S(t) in
-      // TMEM implies that PV(t-2) has finished (the issuer commits S(t) after
-      // issuing PV(t-2)), so with two P buffers buffer t % 2 is free again;
-      // with one (q8_0) the softmax waits for PV(t-1) before storing P(t).
+      // after PV(t-1) has finished and before P(t) is published.  fp16: S(t)
+      // in TMEM implies that PV(t-2) has finished (the issuer commits S(t)
+      // after issuing PV(t-2)), so P buffer t % 2 is free again; q8_0 (one P
+      // buffer) waits for PV(t-1) before storing P(t).
       // q8_0: this thread's lanes of O^T are head_dim elements 32*q4 ..
       // 32*q4 + 31, i.e. scale group q4: only that group's accumulator is
       // read (and rescaled) here.
@@ -1121,6 +1147,20 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           }
         }
         return sc;
+      };
+      // Wait until PV(k) has finished.  A parity wait for phase k of the
+      // O barrier is exact only when phases < k have completed and phase k+1
+      // cannot have (P(k+1) not yet published): k = t-1 before P(t) goes
+      // out, where phases < t-1 are complete because S(t) implies PV(t-2).
+      // A wait after the last P went out would not be exact for PV(end_t-2),
+      // so that one is waited for before.  o_seen counts the phases known to
+      // be complete.
+      int o_seen = 0;
+      auto wait_o_done = [&](int k) -> bool {
+        if (o_seen > k) return true;
+        if (!mbar_wait(bar(BAR_OFULL), k & 1, abort)) return false;
+        o_seen = k + 1;
+        return true;
       };
       uint4 sc_next = make_uint4(0, 0, 0, 0);
       if constexpr (Q8) {
@@ -1259,7 +1299,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             lpart[r] *= av[r];
           }
           if (t > 0) {  // rescale the accumulated O columns of this group's rows
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (t - 1) & 1, abort));
+            ok = __all_sync(0xffffffffu, ok && wait_o_done(t - 1));
             if (ok) {
               tc_fence_after();
               float oh[RW], ol[RW];
@@ -1302,9 +1342,11 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             }
           }
         }
-        // One P buffer: PV(t-1) must have read it before P(t) goes in.
-        if (PB == 1 && t > 0) {
-          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (t - 1) & 1, abort));
+        // One P buffer: PV(t-1) must have read it before P(t) goes in.  The
+        // last tile waits for PV(t-1) in any case, so that the final wait
+        // below is for one phase only.
+        if ((PB == 1 || t == end_t - 1) && t > 0) {
+          ok = __all_sync(0xffffffffu, ok && wait_o_done(t - 1));
           if (ok) tc_fence_after();
         }
         if (ok) {
@@ -1352,16 +1394,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % PB));
       }
 
-      // The accumulated O^T once PV(end_t - 1) has finished: high + residual.
-      // A parity wait is only exact while the barrier is at most one phase
-      // behind: with two tiles, S(1) says nothing about PV(0), so wait for
-      // phase end_t - 2 first.
+      // The accumulated O^T once PV(end_t - 1) has finished: high + residual
+      // (PV(end_t - 2) was waited for before the last P went out).
       float acc[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) acc[r] = 0.f;
-      if (end_t >= 2)
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (end_t - 2) & 1, abort));
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_OFULL), (end_t - 1) & 1, abort));
+      if (end_t >= 1) ok = __all_sync(0xffffffffu, ok && wait_o_done(end_t - 1));
       if (ok) {
         tc_fence_after();
         float oh[RW], ol[RW];
