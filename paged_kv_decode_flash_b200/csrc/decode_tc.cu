@@ -194,7 +194,6 @@ struct Misc {
   int k_consumed, v_consumed;
   int last;  // this CTA arrived last in its (sequence, KV head): it merges
   int bad;   // a block index of this CTA's keys was out of range
-  int g_s, g_kvh, g_split, g_splits, g_first;  // group_of() of this CTA
 };
 
 // What the K producer publishes for each local tile of a CTA: the tile's
@@ -609,37 +608,33 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // may launch at once (they wait the same way).
   griddep_wait();
   griddep_launch_dependents();
-  // Which (sequence, KV head) this CTA works for (warp 0, no memory access).
-  // With one sequence, the K producer lanes then read the block-table entries
-  // of this CTA's first tile on the guess that the whole table is visible
-  // (no window, full length) while the context length is in flight; used
-  // below only if the guess held.  This takes one memory latency off the
-  // time to the first tile.
+  // Which (sequence, KV head) this CTA works for: every thread computes it
+  // (arithmetic only), so that no barrier stands between the grid
+  // dependency and the first memory reads.  The context length is read at
+  // once; with one sequence, the K producer lanes read the block-table
+  // entries of this CTA's first tile at the same time, on the guess that the
+  // whole table is visible (no window, full length), used below only if the
+  // guess held.  Both latencies overlap.
+  const GroupOf go = group_of(p, cta, C_all);
+  const int s = go.s, kvh = go.kvh, split = go.split, S = go.splits, first = go.first;
+  const int L = ld_nc_s32(p.context_lens + s);
   int spec_key0 = -1, spec_phys = 0;
-  if (warp == 0) {
-    const GroupOf go = group_of(p, cta, C_all);
-    if (lane == 0) {
-      misc->g_s = go.s;
-      misc->g_kvh = go.kvh;
-      misc->g_split = go.split;
-      misc->g_splits = go.splits;
-      misc->g_first = go.first;
-    }
-    if (p.num_seqs == 1 && p.tiles_per_item == 0 && lane < kChunksPerTile) {
-      const int ntg =
-          (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
-      const int tfg = go.split * (ntg / go.splits) + min(go.split, ntg % go.splits);
-      const int key0 = tfg * kTileKeys + lane * kChunk;
-      if (ntg / go.splits + (go.split < ntg % go.splits ? 1 : 0) > 0 &&
-          key0 / p.block_size < p.max_blocks_per_seq) {
-        spec_key0 = key0;
-        spec_phys = ld_nc_s32(p.block_table + key0 / p.block_size);
-      }
+  if (warp == 0 && p.num_seqs == 1 && p.tiles_per_item == 0 && lane < kChunksPerTile) {
+    const int ntg =
+        (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
+    const int tfg = go.split * (ntg / go.splits) + min(go.split, ntg % go.splits);
+    const int key0 = tfg * kTileKeys + lane * kChunk;
+    if (ntg / go.splits + (go.split < ntg % go.splits ? 1 : 0) > 0 &&
+        key0 / p.block_size < p.max_blocks_per_seq) {
+      spec_key0 = key0;
+      spec_phys = ld_nc_s32(p.block_table + key0 / p.block_size);
     }
   }
-  __syncthreads();
-  const int s = misc->g_s, kvh = misc->g_kvh, split = misc->g_split;
-  const int S = misc->g_splits, first = misc->g_first;
+  // Group barrier of the cooperative merge (below): its phase bit, read
+  // before this CTA arrives (it cannot flip before then).
+  int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
+  unsigned int bar_phase = 0;
+  if (p.coop && threadIdx.x == 0) bar_phase = (unsigned int)ld_acquire_gpu(cnt) & 0x80000000u;
   // Partials: CTA c owns rows [c*R, c*R + R) of the partial outputs and
   // log-sum-exps; the CTAs of one group are consecutive.
   const long long part_base = (long long)cta * R;
@@ -653,7 +648,6 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // sequence's own context length and the shapes, so every call on the same
   // inputs adds the same tiles in the same order: results are
   // bit-reproducible.
-  const int L = ld_nc_s32(p.context_lens + s);
   const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
   const SeqTiles st_ = seq_tiles(p, L);
   const int lo_u = st_.lo, hi_u = st_.hi, base = st_.base, ntiles_h = st_.tiles;
@@ -1450,30 +1444,28 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   // ---- arrival and merge --------------------------------------------------------
   if (t_count == 0 && threadIdx.x == 0) misc->abort = 0;  // set by the K producer otherwise
   __syncthreads();  // (B) partials written, copies drained, TMEM freed
-  // Two counters per (sequence, KV head) group.  After (B), one thread makes
-  // the CTA's partials visible device-wide (its fence covers the stores the
-  // barrier ordered before it) and then counts the CTA in.
-  int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
+  // Two counters per (sequence, KV head) group (cnt, above).  After (B), one
+  // thread counts the CTA in with release semantics, which publish the
+  // CTA's partials (the barrier ordered their stores before it).
   if (p.coop) {
     // Every CTA of the grid is resident: a barrier over the group's S CTAs,
     // then each merges its share of the group.  The barrier needs no reset:
     // the group's first CTA adds 2^31 - (S - 1) and the others 1, so the top
     // bit of counter 0 flips once all S have arrived and its low bits return
-    // to their value (zero).  The wait is bounded.
+    // to their value (zero).  The arrival does not wait for a reply; the
+    // wait (acquire loads) is bounded.
     if (threadIdx.x == 0) {
-      __threadfence();
       const unsigned int add = split == 0 ? 0x80000000u - (unsigned int)(S - 1) : 1u;
-      const unsigned int old = atomicAdd(reinterpret_cast<unsigned int*>(cnt), add);
+      red_release_add_gpu(cnt, add);
       const unsigned long long t0 = globaltimer();
       int ok = 1;
-      while ((((unsigned int)ld_acquire_gpu(cnt) ^ old) & 0x80000000u) == 0u) {
+      while (((unsigned int)ld_acquire_gpu(cnt) & 0x80000000u) == bar_phase) {
         if (globaltimer() - t0 > kWaitLimitNs) {
           ok = 0;
           break;
         }
-        __nanosleep(32);
+        __nanosleep(20);
       }
-      __threadfence();
       misc->last = ok;
     }
     __syncthreads();

@@ -106,6 +106,11 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   return v;
 }
 
+// Atomic add at GPU scope with release semantics, no value returned.
+__device__ __forceinline__ void red_release_add_gpu(int* p, unsigned int v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // ----------------------------------------------- programmatic dependent launch
 // Allow the next kernel on the stream (launched with programmatic stream
 // serialization) to be scheduled before this grid finishes.
