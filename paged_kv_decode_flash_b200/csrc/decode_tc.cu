@@ -95,12 +95,13 @@ constexpr uint32_t kChunkBytes = kChunk * 256;     // one 16-key chunk (TMA box)
 // q8_0: a raw 128-key tile in shared memory is qs [128 keys][128 int8] then
 // d [128 keys][4 fp16]; a 16-key chunk arrives as two bulk copies (2048 B of
 // qs, 128 B of scales).
-constexpr uint32_t kRawQsBytes = kTileKeys * kHeadDim;              // 16 KB
-constexpr uint32_t kRawBytes = kRawQsBytes + kTileKeys * 8;         // 17 KB
-constexpr uint32_t kQ8ChunkBytes = kChunk * (kHeadDim + 8);         // 2176 B
+constexpr uint32_t kRawOff = kKVBytes / 2;          // q8_0: raw qs in the slot's upper half
+constexpr uint32_t kQ8QsChunk = kChunk * kHeadDim;    // 2048 B of qs per 16-key chunk
+constexpr uint32_t kQ8DChunk = kChunk * 8;            // 128 B of scales per 16-key chunk
 constexpr int kSoftmaxThreads = 128;           // per softmax warpgroup
 constexpr uint32_t kBarSetup = 1;              // named barrier: set-up done
-constexpr uint32_t kBarGroup0 = 2;             // named barriers 2.. : softmax groups
+constexpr uint32_t kBarGroup0 = 2;             // named barriers 2, 3: softmax groups
+constexpr uint32_t kBarConv0 = 4;              // named barriers 4, 5: q8_0 K / V converters
 // A row's reference max is only raised when a score passes it by more than
 // kLazy (log2 units); weights scaled by 2^kPShift (see Cfg) then stay below
 // 2^(kPShift + kLazy), inside fp16 range.
@@ -117,10 +118,8 @@ enum : int {
   BAR_OFULL = 18,   // PV of one more tile accumulated into O^T
   BAR_DONE = 22,    // every MMA finished
   BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
-  BAR_CKFULL = 31,  // q8_0: converted K tile written
-  BAR_CKEMPTY = 32, // q8_0: converted K tile read by QK^T
-  BAR_CVFULL = 33,  // [2] q8_0: converted V tile written
-  BAR_CVEMPTY = 35, // [2] q8_0: converted V tile read by PV
+  BAR_CKFULL = 31,  // [3] q8_0: K slot converted to fp16
+  BAR_CVFULL = 34,  // [3] q8_0: V slot converted to fp16
   BAR_COUNT = 37
 };
 constexpr int kBarSlots = 40;
@@ -132,9 +131,11 @@ constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 // KS / VS slots in the K / V rings, PB buffers for P.  fp16: two P buffers,
 // so that the softmax of tile t+1 never waits for PV(t); at 32 rows they take
 // 32 KB and the V ring keeps two slots (measured: three V slots with one P
-// buffer is slower).  q8_0: raw rings of two slots each, one converted K tile,
-// two converted V tiles, and one P buffer that holds a P per scale group
-// (the softmax of tile t waits for PV(t-1) before it stores P(t)).
+// buffer is slower).  q8_0: a slot is the fp16 operand tile; the raw int8
+// tile lands in its upper half and the converters expand it in place (a V
+// slot also keeps the raw scales after the tile); two K slots, three V
+// slots, one P buffer that holds a P per scale group (the softmax of tile t
+// waits for PV(t-1) before it stores P(t)).
 template <int RW, int NG, bool Q8>
 struct Cfg {
   static constexpr int kGroups = NG;
@@ -147,19 +148,17 @@ struct Cfg {
   // head_dim elements that shares a scale; fp16: one of each.
   static constexpr int kSG = Q8 ? kHeadDim / 32 : 1;
   static constexpr int KS = Q8 ? 2 : 3;
-  static constexpr int VS = Q8 ? 2 : (NR > 16 ? 2 : 3);
-  static constexpr int PB = Q8 ? 1 : 2;
-  static constexpr int CVS = 2;                  // q8_0: converted V slots
+  static constexpr int VS = Q8 ? 3 : (NR > 16 ? 2 : 3);
+  static constexpr int PB = Q8 ? 1 : 2;  // q8_0 measured: two V slots and two P buffers are slower
   // Weights are scaled by 2^kPShift before they are split into fp16 parts.
   // q8_0 multiplies them by a scale mantissa in [1, 2) as well, so it keeps
   // one bit of headroom more.
   static constexpr int kPShift = Q8 ? 13 : 14;
-  static constexpr uint32_t kSlotBytes = Q8 ? kRawBytes : kKVBytes;
-  static constexpr uint32_t kK = 0;                                 // K ring
-  static constexpr uint32_t kV = KS * kSlotBytes;                   // V ring
-  static constexpr uint32_t kConvK = (KS + VS) * kSlotBytes;        // q8_0: converted K
-  static constexpr uint32_t kConvV = kConvK + (Q8 ? kKVBytes : 0);  // q8_0: CVS converted V
-  static constexpr uint32_t kQ = kConvV + (Q8 ? CVS * kKVBytes : 0);
+  static constexpr uint32_t kKSlot = kKVBytes;                           // K slot
+  static constexpr uint32_t kVSlot = kKVBytes + (Q8 ? kTileKeys * 8 : 0);  // V slot (+ scales)
+  static constexpr uint32_t kK = 0;                                      // K ring
+  static constexpr uint32_t kV = KS * kKSlot;                            // V ring
+  static constexpr uint32_t kQ = kV + VS * kVSlot;
   static constexpr uint32_t kQHalf = NR * 128;
   // P^T of one tile: per scale group 2*NR "rows" (the fp16 high parts of the
   // NR query rows, then their residuals), the groups side by side, so that
@@ -184,7 +183,7 @@ struct Cfg {
                                         : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
   static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
   static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
-  static_assert(kConvK % 1024 == 0, "converted tiles sit on 1 KB swizzle atoms");
+  static_assert(kV % 1024 == 0 && kVSlot % 1024 == 0, "tiles sit on 1 KB swizzle atoms");
   static_assert(kTmemUsed <= 512, "TMEM columns");
 };
 
@@ -677,19 +676,14 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   } else if (warp == 0) {
     // ======================= K producer (also sets up the barriers) ========
     if (lane == 0) {
-      // q8_0: the raw K (V) slots are released by the K (V) converter warps.
       for (int i = 0; i < kMaxStages; ++i) {
         mbar_init(bar(BAR_KFULL + i), 1);
-        mbar_init(bar(BAR_KEMPTY + i), Q8 ? C::kConvWarps : 1);
+        mbar_init(bar(BAR_KEMPTY + i), 1);
         mbar_init(bar(BAR_VFULL + i), 1);
-        mbar_init(bar(BAR_VEMPTY + i), Q8 ? C::kConvWarps : 1);
-      }
-      if (Q8) {
-        mbar_init(bar(BAR_CKFULL), C::kConvWarps);
-        mbar_init(bar(BAR_CKEMPTY), 1);
-        for (int i = 0; i < C::CVS; ++i) {
+        mbar_init(bar(BAR_VEMPTY + i), 1);
+        if (Q8) {  // q8_0: a slot's fp16 tile is ready once every converter warp arrived
+          mbar_init(bar(BAR_CKFULL + i), C::kConvWarps);
           mbar_init(bar(BAR_CVFULL + i), C::kConvWarps);
-          mbar_init(bar(BAR_CVEMPTY + i), 1);
         }
       }
       for (int i = 0; i < 2; ++i) {
@@ -770,17 +764,14 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       const uint32_t fb = bar(BAR_KFULL + st);
-      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8ChunkBytes : kChunkBytes));
+      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8QsChunk : kChunkBytes));
       __syncwarp();
       if (w_cur) {
         if constexpr (Q8) {
+          // K's scales are read by the softmax (from L2), not staged here.
           const long long off = q8_chunk_offset(p, row_cur, base + g_cur * kTileKeys + c * kChunk);
-          const uint32_t dst = sKr + st * kRawBytes;
           const uint8_t* src = static_cast<const uint8_t*>(p.k);
-          bulk_load(dst + c * kChunk * kHeadDim, src + off, kChunk * kHeadDim, fb);
-          bulk_load(dst + kRawQsBytes + c * kChunk * 8,
-                    src + off + q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk), kChunk * 8,
-                    fb);
+          bulk_load(sKr + st * C::kKSlot + kRawOff + c * kQ8QsChunk, src + off, kQ8QsChunk, fb);
           bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off, kChunk * kHeadDim);
           bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off +
                                q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk),
@@ -855,17 +846,18 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const uint32_t fb = bar(BAR_VFULL + st);
-        if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8ChunkBytes : kChunkBytes));
+        if (lane == 0)
+          mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8QsChunk + kQ8DChunk : kChunkBytes));
         __syncwarp();
         if (c < kChunksPerTile && ((mask >> c) & 1u)) {
           if constexpr (Q8) {
             const long long off = q8_chunk_offset(p, row8, base + ti.tile * kTileKeys + c * kChunk);
-            const uint32_t dst = sVr + st * kRawBytes;
+            const uint32_t dst = sVr + st * C::kVSlot;
             const uint8_t* src = static_cast<const uint8_t*>(p.v);
-            bulk_load(dst + c * kChunk * kHeadDim, src + off, kChunk * kHeadDim, fb);
-            bulk_load(dst + kRawQsBytes + c * kChunk * 8,
+            bulk_load(dst + kRawOff + c * kQ8QsChunk, src + off, kQ8QsChunk, fb);
+            bulk_load(dst + kKVBytes + c * kQ8DChunk,
                       src + off + q8_scale_offset(p, base + ti.tile * kTileKeys + c * kChunk),
-                      kChunk * 8, fb);
+                      kQ8DChunk, fb);
           } else {
             tma_load_4d(sVr + st * kKVBytes + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
           }
@@ -891,26 +883,25 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         const uint32_t id_pv = idesc_f16_f32(128, C::kPN, true, true);
         // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
         // start-address field is the low 14 bits, addresses stay < 256 KB).
-        // q8_0: K and V are the converted tiles (exact fp16 images of the
+        // q8_0: K and V are the converted slots (exact fp16 images of the
         // int8 values; V's rows also carry the power of two of their scales).
         // S^T gets one accumulator per scale group g (head_dim 32g .. 32g+31,
         // two steps of 16), which the softmax combines with K's scales; PV
         // multiplies V with each group's P (the weights times V's scale
         // mantissas) into that group's O^T accumulator.
-        const uint64_t dK = smem_desc(Q8 ? sbase + C::kConvK : sKr, 16, kGroupBytes, kSwizzle128B);
+        const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
-        const uint64_t dV =
-            smem_desc(Q8 ? sbase + C::kConvV : sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
+        const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
         const uint64_t dP = smem_desc(sP, C::kPN * 16, 128, kSwizzleNone);
         constexpr int kSG = C::kSG;
         // QK(u) once K(u) is ready and the softmax took S(u-2) from its buffer.
         auto issue_qk = [&](int u) -> bool {
-          const bool ready = Q8 ? mbar_wait(bar(BAR_CKFULL), u & 1, abort)
-                                : mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, abort);
+          const bool ready =
+              mbar_wait(bar((Q8 ? BAR_CKFULL : BAR_KFULL) + u % KS), (u / KS) & 1, abort);
           if (!(ready && mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
             return false;
           tc_fence_after();
-          const uint64_t so = Q8 ? 0 : (uint64_t)((u % KS) * kKVBytes) >> 4;
+          const uint64_t so = (uint64_t)((u % KS) * C::kKSlot) >> 4;
           const uint32_t d = tmem + (u % 2) * kSG * NR;
           constexpr int kSteps = kHeadDim / 16 / kSG;  // steps of 16 per accumulator
 #pragma unroll
@@ -920,7 +911,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             tc_mma_f16_ss(d + (k / kSteps) * NR, dK + so + ko, dQ + qo, id_qk, k % kSteps != 0);
           }
           tc_commit(bar(BAR_SFULL + u % 2));
-          tc_commit(bar(Q8 ? BAR_CKEMPTY : BAR_KEMPTY + u % KS));
+          tc_commit(bar(BAR_KEMPTY + u % KS));
           return true;
         };
         int nqk = 0, npv = 0;
@@ -932,11 +923,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
         for (int t = 0; ok && t < t_count; ++t) {
           // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
           ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
-               (Q8 ? mbar_wait(bar(BAR_CVFULL + t % C::CVS), (t / C::CVS) & 1, abort)
-                   : mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, abort));
+               mbar_wait(bar((Q8 ? BAR_CVFULL : BAR_VFULL) + t % VS), (t / VS) & 1, abort);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((t % (Q8 ? C::CVS : VS)) * kKVBytes) >> 4;
+          const uint64_t so = (uint64_t)((t % VS) * C::kVSlot) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
           // O^T accumulates over all tiles; q8_0: the kSG group accumulators
           // are the consecutive column ranges of one N = kPN product.
@@ -948,17 +938,15 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
             tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, t > 0 || k > 0);
           }
           tc_commit(bar(BAR_OFULL));
-          tc_commit(bar(Q8 ? BAR_CVEMPTY + t % C::CVS : BAR_VEMPTY + t % VS));
+          tc_commit(bar(BAR_VEMPTY + t % VS));
           npv = t + 1;
           if (t + 2 < t_count) {
             ok = issue_qk(t + 2);
             if (ok) nqk = t + 3;
           }
         }
-        if (!Q8) {  // q8_0: the converter consumes the raw rings
-          misc->k_consumed = nqk;
-          misc->v_consumed = npv;
-        }
+        misc->k_consumed = nqk;
+        misc->v_consumed = npv;
         tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
         volatile int no_abort = 0;
         mbar_wait(bar(BAR_DONE), 0, &no_abort);
@@ -967,27 +955,31 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       __syncthreads();  // (A)
     } else if (Q8 && warp >= C::kConvWarp) {
       // ===================== q8_0 converters =================================
-      // Raw tile t (int8 qs, fp16 scales d per 32 elements) -> the fp16 K and
-      // V operand tiles, exactly: K's operand is qs itself (every integer
-      // below 2048 is an fp16 value; K's scales are applied to the per-group
-      // scores in the softmax), V's is qs * 2^e with 2^e the power of two of
-      // the element's scale d = m * 2^e (exact for |d| < 1024: at most 7
-      // significant bits above 2^-24); the mantissa m goes into that group's
-      // P.  The arithmetic is packed fp16 (two elements per instruction).
-      // Layout as the fp16 TMA boxes: [key/8][half][key%8][64 dims], 128-byte
-      // swizzle.  V rows of keys outside [lo_u, hi_u] (masked or never
-      // loaded) are written as zeros: they must not reach the PV product.
-      // The first kConvWarps converter warps convert K (one operand tile),
-      // the next kConvWarps convert V (two operand tiles), so that K is never
-      // held up by V waiting for its operand buffer.  Thread ct of a
-      // stream's kCT takes the 16-byte column chunk c16 = ct % 8 (head_dim
-      // 16*c16 .. +15, half of one scale group) of keys r = ct / 8 + kRS*k:
-      // one 16-byte load and two 16-byte stores per key, the swizzled
-      // destination offset constant up to the key group, no bank conflicts on
-      // either side.
+      // Raw tile t (int8 qs in the upper half of its slot; V: fp16 scales d
+      // per 32 elements after the tile) -> the fp16 operand in the same slot,
+      // exactly: K's operand is qs itself (every integer below 2048 is an
+      // fp16 value; K's scales are applied to the per-group scores in the
+      // softmax), V's is qs * 2^e with 2^e the power of two of the element's
+      // scale d = m * 2^e (exact for |d| < 1024: at most 7 significant bits
+      // above 2^-24); the mantissa m goes into that group's P.  The
+      // arithmetic is packed fp16 (two elements per instruction).  Layout as
+      // the fp16 TMA boxes: [key/8][half][key%8][64 dims], 128-byte swizzle.
+      // V rows of keys outside [lo_u, hi_u] (masked or never loaded) are
+      // written as zeros: they must not reach the PV product.
+      // The first kConvWarps converter warps convert K, the next kConvWarps
+      // V.  Thread ct of a stream's kCT takes the 16-byte column chunk
+      // c16 = ct % 8 (head_dim 16*c16 .. +15, half of one scale group) of keys
+      // r = ct / 8 + kRS*k: one 16-byte load and two 16-byte stores per key,
+      // the swizzled destination offset constant up to the key group, no bank
+      // conflicts on either side.  In place: keys 0 .. 63 land below the raw
+      // data; keys 64 .. 127 are stored only after every thread of the stream
+      // has read (and converted into registers) all its raw rows.
       constexpr int kCT = 32 * C::kConvWarps;   // threads per stream
       constexpr int kRS = kCT / 8;              // key stride between a thread's keys
       constexpr int kKeysPer = kTileKeys / kRS; // keys per thread per tile
+      constexpr int kHalfKeys = kKeysPer / 2;   // per half tile
+      static_assert(kKeysPer % 2 == 0 && (kTileKeys / 2) * 256 <= kRawOff,
+                    "the lower half of the keys is stored below the raw tile");
       const int kv = (warp - C::kConvWarp) / C::kConvWarps;  // 0: K, 1: V
       const int ct = threadIdx.x - 32 * (C::kConvWarp + C::kConvWarps * kv);  // 0 .. kCT-1
       const int c16 = ct & 7, r0 = ct >> 3;      // column chunk, first key
@@ -998,13 +990,11 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
                              ((((2 * c16) & 7) ^ r08) << 4);
       const uint32_t dst_b = (r0 >> 3) * kGroupBytes + ((2 * c16 + 1) >> 3) * kAtomBytes +
                              r08 * 128 + ((((2 * c16 + 1) & 7) ^ r08) << 4);
-      const int NSl = kv == 0 ? KS : VS;        // raw slots
-      const int NCs = kv == 0 ? 1 : C::CVS;     // operand slots
+      const int NSl = kv == 0 ? KS : VS;
       const uint32_t bar_full = kv == 0 ? BAR_KFULL : BAR_VFULL;
-      const uint32_t bar_raw_empty = kv == 0 ? BAR_KEMPTY : BAR_VEMPTY;
-      const uint32_t bar_cfull = kv == 0 ? BAR_CKFULL : BAR_CVFULL;
-      const uint32_t bar_cempty = kv == 0 ? BAR_CKEMPTY : BAR_CVEMPTY;
-      int n = 0;
+      const uint32_t bar_conv = kv == 0 ? BAR_CKFULL : BAR_CVFULL;
+      const uint32_t ring = sbase + (kv == 0 ? C::kK : C::kV);
+      const uint32_t slot_bytes = kv == 0 ? C::kKSlot : C::kVSlot;
       bool ok = true;
       // Eight int8 -> eight fp16 values times the power of two p2 (1 for K).
       auto convert = [&](uint32_t w0, uint32_t w1, __half2 p2) -> uint4 {
@@ -1020,51 +1010,48 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       };
       for (int t = 0; t < t_count && ok; ++t) {
         const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
-        const int rs = t % NSl, cs_ = t % NCs;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort) &&
-                            mbar_wait(bar(bar_cempty + cs_), ((t / NCs) & 1) ^ 1, abort));
+        const int rs = t % NSl;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort));
         if (!ok) break;
-        const uint32_t raw = sbase + (kv == 0 ? C::kK : C::kV) + rs * kRawBytes;
-        const uint32_t src = raw + r0 * kHeadDim + c16 * 16;                 // key r0, chunk c16
-        const uint32_t srcd = raw + kRawQsBytes + r0 * 8 + (c16 >> 1) * 2;  // its scale
-        const uint32_t dst = sbase + (kv == 0 ? C::kConvK : C::kConvV + cs_ * kKVBytes);
-        // Four keys at a time: every load first, so that one shared-memory
-        // latency covers all four.
-#pragma unroll 1
-        for (int k0 = 0; k0 < kKeysPer; k0 += 4) {
-          uint4 qv[4];
-          uint16_t dv[4];
+        const uint32_t slot = ring + rs * slot_bytes;
+        const uint32_t src = slot + kRawOff + r0 * kHeadDim + c16 * 16;       // key r0, chunk c16
+        const uint32_t srcd = slot + kKVBytes + r0 * 8 + (c16 >> 1) * 2;     // its scale (V)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            qv[i] = lds_v4(src + (k0 + i) * kRS * kHeadDim);
-            dv[i] = kv == 0 ? (uint16_t)0 : lds_u16(srcd + (k0 + i) * kRS * 8);
+        for (int h = 0; h < 2; ++h) {
+          uint4 qv[kHalfKeys];
+          uint16_t dv[kHalfKeys];
+#pragma unroll
+          for (int i = 0; i < kHalfKeys; ++i) {
+            const int k = h * kHalfKeys + i;
+            qv[i] = lds_v4(src + k * kRS * kHeadDim);
+            dv[i] = kv == 0 ? (uint16_t)0 : lds_u16(srcd + k * kRS * 8);
           }
+          uint4 xa[kHalfKeys], xb[kHalfKeys];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = (k0 + i) * kRS + r0;
-            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+          for (int i = 0; i < kHalfKeys; ++i) {
+            const int r = (h * kHalfKeys + i) * kRS + r0;
+            xa[i] = make_uint4(0, 0, 0, 0);
+            xb[i] = xa[i];
             if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) {
               const __half p2 = __ushort_as_half(q8_scale_pow2_bits(dv[i]));
               const __half2 p22 = __halves2half2(p2, p2);
-              xa = convert(qv[i].x, qv[i].y, p22);
-              xb = convert(qv[i].z, qv[i].w, p22);
+              xa[i] = convert(qv[i].x, qv[i].y, p22);
+              xb[i] = convert(qv[i].z, qv[i].w, p22);
             }
-            sts_v4(dst + (k0 + i) * (kRS / 8) * kGroupBytes + dst_a, xa);
-            sts_v4(dst + (k0 + i) * (kRS / 8) * kGroupBytes + dst_b, xb);
+          }
+          // The upper half overwrites raw rows: every thread of the stream
+          // has read all of its rows once it is past this barrier.
+          if (h == 1) named_bar_sync(kBarConv0 + kv, kCT);
+#pragma unroll
+          for (int i = 0; i < kHalfKeys; ++i) {
+            const uint32_t g8 = (h * kHalfKeys + i) * (kRS / 8) * kGroupBytes;
+            sts_v4(slot + g8 + dst_a, xa[i]);
+            sts_v4(slot + g8 + dst_b, xb[i]);
           }
         }
         fence_proxy_async_smem();  // generic writes -> the tensor core's reads
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(bar_cfull + cs_));
-          mbar_arrive(bar(bar_raw_empty + rs));
-        }
-        n = t + 1;
-      }
-      if (ct == 0) {
-        if (kv == 0) misc->k_consumed = n;
-        else misc->v_consumed = n;
+        if (lane == 0) mbar_arrive(bar(bar_conv + rs));
       }
       __syncthreads();  // (A)
     } else {
