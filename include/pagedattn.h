@@ -191,8 +191,8 @@ int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_
                               int32_t kv_dtype, void* out, void* stream);
 
 /* Kernel launches one paged_attn_decode call makes for these shapes and
- * cache type on the current device: 1 where the tensor-core kernel runs (the
- * last CTA of each (sequence, KV head) merges that group's partials), 2 for
+ * cache type on the current device: 1 where the tensor-core kernel runs (its
+ * CTAs also merge the split partials of each (sequence, KV head)), 2 for
  * the CUDA-core kernel followed by the merge kernel (launched as a
  * programmatic dependent so that it starts as soon as the split-KV kernel
  * ends).  Host only; negative pa_status on error. */

@@ -12,9 +12,11 @@
 //
 // Hardware mapping (one CTA per SM, 11 warps; 19 for the q8_0 cache):
 //   warps 0, 10 TMA producers for K and for V: resolve the block table and
-//               load whole 16-key chunks (two 64-column halves each, 128-byte
-//               swizzle) into separate rings of 128-key tiles (2-3 slots);
-//               K slots are released as soon as QK^T has read them, so K runs
+//               load whole 16-key chunks into separate rings of 128-key tiles
+//               (fp16: 4-D boxes of two 64-column halves with the 128-byte
+//               swizzle, 2-3 slots; q8_0: untiled bulk copies of the raw
+//               chunk into the upper half of a slot, 2 K and 3 V slots).  K
+//               slots are released as soon as QK^T has read them, so K runs
 //               ahead.  With each K copy the same chunk of V is prefetched
 //               into L2, so that V's own copy a tile later is short.
 //   warp 1      MMA issuer (one thread), fixed order QK(0), QK(1), then
@@ -22,20 +24,21 @@
 //               query rows (double-buffered in TMEM), O^T += V^T
 //               [P_hi | P_lo]^T with M = 128 head_dim lanes (one TMEM
 //               accumulator over all tiles); P is double-buffered in shared
-//               memory so that the softmax of tile t+1 overlaps PV(t).
+//               memory (fp16) so that the softmax of tile t+1 overlaps PV(t).
 //   warps 2-9   two softmax warpgroups, each owning half of the query rows:
 //               thread = key for S (row max by a warp transpose-reduction
 //               plus one named barrier per group); when a row's reference
 //               maximum rises, its O column is rescaled in TMEM in place
 //               (thread = head_dim lane) before the tile's P is published.
-//   warps 11-18 (q8_0 cache only) converters: raw int8 tiles -> exact fp16
-//               operand tiles (see below).
+//   warps 11-18 (q8_0 cache only) converters, four for K and four for V:
+//               each raw int8 tile is expanded in place into its exact fp16
+//               operand tile (see below).
 // Putting keys and head_dim on the MMA's M side keeps the tensor core free of
 // padding even at 4-32 query rows.
 //
 // Exactness: Q, K and V are fed to the tensor core as the exact fp16 inputs.
-// The softmax weights are scaled by 2^14 (so that weights down to ~4e-12 of
-// the row maximum stay representable) and split into an fp16 high part and
+// The softmax weights are scaled by 2^14 (2^13 for q8_0, so that weights
+// down to ~4e-12 of the row maximum stay representable) and split into an fp16 high part and
 // an fp16 residual; both are multiplied with V and accumulated in fp32, which
 // keeps the weights to about 2^-22 relative.  Keys no query row can see are
 // never multiplied: their chunks are not loaded when wholly outside the
@@ -53,6 +56,9 @@
 // group's m (then split into fp16 parts as above), and each group has its
 // own O^T accumulator, of which a head_dim lane reads only its own group's.
 // The softmax reads the scales of its keys from the cache (L2) a tile ahead.
+// Batches with many (sequence, KV head) groups cut every group's tiles into
+// fixed-size items, one CTA each, over several waves; the size depends on
+// the shapes only, so a sequence's output does not depend on the others.
 //
 // Merge: every CTA writes its fp32 partial (O, lse).  With a cooperative
 // launch (every CTA resident) the CTAs of one (sequence, KV head) meet at a

@@ -218,6 +218,38 @@ def test_batched_items_sequence_independent_of_neighbours(B):
     assert np.array_equal(out_a[1].view(np.uint16), out_b[1].view(np.uint16))
 
 
+def _q8_scales(cache, bs):
+    """The fp16 scales [NB][Hkv][bs][4] of a q8_0 cache held as bytes
+    [NB][Hkv][bs * 136] (a view: writing it edits the cache)."""
+    nb, h = cache.shape[0], cache.shape[1]
+    return cache[:, :, bs * 128:].view(np.float16).reshape(nb, h, bs, 4)
+
+
+def test_q8_0_extreme_scales(B, orc):
+    """q8_0 scales across the fp16 range the kernel supports: V groups
+    scaled by 2^14 (scales near 500, operand exponent at its limit), 2^-10
+    (subnormal scales), 3 (a new mantissa) and 1; K groups by 1, 2^5, 2^-6
+    and 1.5.  Every row against the oracle, each V group's output dims
+    rescaled back by the same factor on both sides before the comparison."""
+    case = gen.make_case(seed=70, context_lens=(1500, 333, 2600), n_query=4, num_q_heads=16,
+                         num_kv_heads=4, causal=1, kv_dtype=gen.KV_Q8_0, spare_blocks=2)
+    vf = np.array([2.0 ** 14, 2.0 ** -10, 3.0, 1.0])
+    kf = np.array([1.0, 2.0 ** 5, 2.0 ** -6, 1.5])
+    for cache, f in ((case.k_cache, kf), (case.v_cache, vf)):
+        d = _q8_scales(cache, case.block_size)
+        d[...] = (d.astype(np.float64) * f).astype(np.float16)
+    dv = _q8_scales(case.v_cache, case.block_size).astype(np.float64)
+    assert np.nanmax(np.abs(dv)) < 1024 and np.nanmax(np.abs(dv[..., 0])) > 256
+    assert np.nanmin(np.abs(dv[..., 1][dv[..., 1] != 0])) < 2.0 ** -14  # subnormal scales
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    # Back to unit size; the subnormal group only by 2^4, since outputs below
+    # fp16's normal range carry a rounding error that a larger factor would
+    # blow past the relative tolerance.
+    back = np.repeat([2.0 ** -14, 2.0 ** 4, 1.0 / 3.0, 1.0], 32)  # per head_dim element
+    assert_parity(out.astype(np.float64) * back, ref * back, "q8_0 extreme scales")
+
+
 def test_batch_matches_each_sequence_alone(B, orc):
     case = gen.make_case(seed=11, context_lens=(900, 33, 2500, 8), n_query=2,
                          num_q_heads=8, num_kv_heads=2, causal=1)
