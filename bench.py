@@ -300,6 +300,8 @@ def bench_ours(args, rank, world, dist):
         return {"s_per_step": dt, "h2d": h2d, "d2h": hout.nbytes}
 
     primary = args.workload
+    if primary not in WORKLOAD_TEXT and not args.primary_only:
+        raise SystemExit("--workload " + primary + " is timed alone: add --primary-only")
     secondary = SECONDARY if primary == PRIMARY else PRIMARY
     prim = measure(primary, args.steps, args.warmup, with_e2e=True)
     sec = measure(secondary, max(1, args.steps // 2), args.warmup, with_e2e=False) \
@@ -333,7 +335,7 @@ def bench_ours(args, rank, world, dist):
         "data": "synthetic (seeded N(0,1) fp16 KV, random block permutation)",
         "impl": "ours",
         "config": {
-            "workload": WORKLOAD_TEXT[primary],
+            "workload": WORKLOAD_TEXT.get(primary) or CONFIG_TEXT[primary],
             "kv_bytes_per_step": kv,
             "num_splits": prim["splits"],
             "l2": f"inputs larger than L2: {prim['copies']} KV pools of "
@@ -455,8 +457,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--primary-only", action="store_true")
-    ap.add_argument("--workload", choices=[PRIMARY, SECONDARY], default=PRIMARY,
-                    help="workload of the headline line (the other is reported under 'also')")
+    ap.add_argument("--workload", choices=[PRIMARY, SECONDARY, *OTHER_CONFIGS], default=PRIMARY,
+                    help="workload of the headline line (the other of the two headline "
+                         "workloads is reported under 'also'; the other configurations only "
+                         "with --primary-only, e.g. for a profiler run)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
