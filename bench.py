@@ -352,9 +352,9 @@ def bench_ours(args, rank, world, dist):
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": recorded_traffic(primary),
-            "kernel": "one paged_attn_decode call: one cooperative launch of the split-KV "
-                      "decode kernel, whose CTAs also merge the split partials; "
-                      "time = timed region / steps",
+            "kernel": "one paged_attn_decode call: one launch of the split-KV decode kernel "
+                      "(cooperative when its grid fits on the device at once), whose CTAs "
+                      "also merge the split partials; time = timed region / steps",
         },
         "clocks": prim["clocks"],
         "gpu_launches": prim["launches"] * args.steps,
