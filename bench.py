@@ -97,6 +97,23 @@ def recorded_traffic(workload):
     return float(ent["dram_bytes_per_launch"])
 
 
+def max_over_ranks(x, dist, device):
+    """The largest of the ranks' x (every rank gets it); x itself without a
+    process group.  Times of a multi-GPU run are the slowest rank's."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(kv_bytes_per_rank, world, seconds_per_step):
+    """Whole-job KV-read rate: every rank reads its own replica's bytes each
+    step (weak scaling), over the slowest rank's time per step."""
+    return world * kv_bytes_per_rank / seconds_per_step / 1e9
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled while running."""
 
@@ -234,10 +251,7 @@ def bench_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         eager_us = ea.elapsed_time(eb) * 1e3 / n_eager
         del graph
-        if dist:
-            t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, device)
         # Per-call spread (outside the timed region): events around each call.
         n_ev = min(steps, 300)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -292,10 +306,7 @@ def bench_ours(args, rank, world, dist):
         for _ in range(steps):
             one()
         dt = (time.perf_counter() - t) / steps
-        if dist:
-            tt = torch.tensor([dt], dtype=torch.float64, device=device)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            dt = float(tt.item())
+        dt = max_over_ranks(dt, dist, device)
         h2d = hq.nbytes + hbt.nbytes + hcl.nbytes
         return {"s_per_step": dt, "h2d": h2d, "d2h": hout.nbytes}
 
@@ -316,7 +327,7 @@ def bench_ours(args, rank, world, dist):
 
     peak, peak_kind = measured_peaks()
     kv = prim["kv_bytes"]
-    value = world * kv / (prim["ms_per_step"] * 1e-3) / 1e9
+    value = job_gbs(kv, world, prim["ms_per_step"] * 1e-3)
     achieved = kv / (prim["ms_per_step"] * 1e-3) / 1e9  # per launch pair, timed region
     line = {
         "metric": METRIC,
@@ -360,7 +371,7 @@ def bench_ours(args, rank, world, dist):
         "gpu_launches": prim["launches"] * args.steps,
     }
     e = prim["e2e"]
-    line["e2e"] = {"value": round(world * kv / e["s_per_step"] / 1e9, 1), "unit": "GB/s",
+    line["e2e"] = {"value": round(job_gbs(kv, world, e["s_per_step"]), 1), "unit": "GB/s",
                    "us_per_call": round(e["s_per_step"] * 1e6, 2),
                    "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
     if sec is not None:
@@ -369,7 +380,7 @@ def bench_ours(args, rank, world, dist):
             "workload": WORKLOAD_TEXT[secondary],
             "us_per_call": round(sec["ms_per_step"] * 1e3, 2),
             "eager_us_per_call": round(sec["eager_us"], 2),
-            "value": round(world * kv2 / (sec["ms_per_step"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "value": round(job_gbs(kv2, world, sec["ms_per_step"] * 1e-3), 1), "unit": "GB/s",
             "pct_of_8TBps": round(100 * kv2 / (sec["ms_per_step"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 1),
             "roofline_frac": round(kv2 / (sec["ms_per_step"] * 1e-3) / 1e9 / peak, 4),
             "per_call_us": {"median": round(sec["us_median"], 2), "min": round(sec["us_min"], 2),
