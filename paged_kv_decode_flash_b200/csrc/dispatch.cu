@@ -119,6 +119,14 @@ Plan max_plan(const pa_dims* d) {
   Plan pl{};
   pl.tensor_cores = false;
   pl.splits = plan_splits(d, kMaxTargetCtas, true, &pl.blocks_per_split);
+  // The tensor-core planner cuts the table into 128-key tiles, which for a
+  // block_size that does not divide 128 allows more splits than whole
+  // blocks do: at most one per tile, and no more than kMaxTargetCtas CTAs
+  // over the groups (one wave, or items of >= 16 tiles over a few waves).
+  const long long groups = (long long)d->num_seqs * d->num_kv_heads;
+  const long long tiles = ceil_div((long long)d->max_blocks_per_seq * d->block_size, 128);
+  const long long tc = std::min(tiles, std::max(1LL, ceil_div(kMaxTargetCtas, groups)));
+  pl.splits = std::max<int>(pl.splits, (int)tc);
   return pl;
 }
 

@@ -110,6 +110,21 @@ def test_several_tiles_per_split(B, orc, tiles_per_cta, dt, nq, G):
     assert_parity(out, ref, f"{tiles_per_cta} tiles per split")
 
 
+@pytest.mark.parametrize("bs,dt", [(48, gen.KV_FP16), (80, gen.KV_Q8_0), (112, gen.KV_FP16),
+                                   (96, gen.KV_Q8_0)])
+def test_block_sizes_that_do_not_divide_a_tile(B, orc, bs, dt):
+    """Blocks of 48-112 keys: a 128-key tile spans parts of two blocks and a
+    single sequence is split into as many CTAs as it has tiles; the
+    workspace from paged_attn_workspace_size must hold that plan.  Every
+    row against the oracle."""
+    case = gen.make_case(seed=80 + bs, context_lens=(bs * 100 - 5,), n_query=4, num_q_heads=8,
+                         num_kv_heads=1, block_size=bs, causal=1, window=bs * 37, kv_dtype=dt,
+                         spare_blocks=3)
+    out, _ = run(B, case)
+    ref, _ = orc.attend(case)
+    assert_parity(out, ref, f"block_size {bs}")
+
+
 def test_sliding_window_config_and_nan_invariance(B, orc):
     case = gen.sliding_window(0)
     out, _ = run(B, case)
