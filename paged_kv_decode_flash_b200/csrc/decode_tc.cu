@@ -1017,7 +1017,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       for (int t = 0; t < t_count && ok; ++t) {
         const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
         const int rs = t % NSl;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort));
+        // The stream's threads decide together (one gave up: all stop), so
+        // that every one of them reaches the named barrier below.
+        ok = named_bar_and(kBarConv0 + kv, kCT,
+                           __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort)));
         if (!ok) break;
         const uint32_t slot = ring + rs * slot_bytes;
         const uint32_t src = slot + kRawOff + r0 * kHeadDim + c16 * 16;       // key r0, chunk c16

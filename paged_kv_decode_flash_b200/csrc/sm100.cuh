@@ -148,6 +148,20 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t threads, bool
   return r != 0;
 }
 
+// Named barrier that also ANDs a predicate over the participating threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %3, 0;\n\t"
+      "bar.red.and.pred po, %1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(threads), "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
 // --------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
