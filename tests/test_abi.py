@@ -112,3 +112,64 @@ def test_binding_refuses_to_run_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         b.lib()
+
+
+def _ceil(a, b):
+    return -(-a // b)
+
+
+def _align(x):
+    return (x + 255) & ~255
+
+
+def _plan_splits(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
+    """The splits paged_attn_decode plans on a device with `sms` SMs (the
+    planner in csrc/dispatch.cu, restated): the tensor-core kernel for up to
+    32 (fp16) or 16 (q8_0) rows per KV head, the CUDA-core kernel beyond."""
+    rows = nq * (Hq // Hkv)
+    groups = B * Hkv
+    if rows <= (32 if kv_dtype == 0 else 16):
+        max_split = _ceil(mbps * bs, 128)
+        if groups * 4 > sms:
+            T = max(16, _ceil(max_split * groups, 4 * sms))
+            return _ceil(max_split, T)
+        ctas = max(groups, min(sms, groups * max_split))
+        return _ceil(ctas, groups)
+    min_blocks = _ceil(128, bs)
+    max_splits = max(1, _ceil(mbps, min_blocks))
+    splits = max(1, min(_ceil(2 * sms, groups), max_splits))
+    bps = _ceil(mbps, splits)
+    return _ceil(mbps, bps)
+
+
+def _ws_needed(B, Hq, Hkv, nq, splits):
+    rows = B * splits * nq * Hq
+    prefix = 256 + _align(B * Hkv * 2 * 4)
+    return prefix + _align(rows * 128 * 4) + _align(rows * 4)
+
+
+def test_workspace_size_covers_every_plan(L):
+    """paged_attn_workspace_size needs no device, so it must cover the plan
+    of any device: every SM count up to 1024, both kernels, every block size
+    (a multiple of 16 up to 128; those that do not divide 128 let the
+    tensor-core kernel cut more splits than whole blocks would)."""
+    import numpy as np
+    rng = np.random.default_rng(7)
+    shapes = [(1, 32, 8, 16, 3841, 8), (1, 32, 4, 16, 12288, 1), (8, 32, 8, 16, 4096, 4),
+              (1, 8, 1, 48, 100, 4), (1, 8, 1, 112, 100, 4), (64, 64, 8, 16, 4096, 8)]
+    for _ in range(60):
+        Hkv = int(rng.choice([1, 2, 4, 8]))
+        shapes.append((int(rng.integers(1, 40)), Hkv * int(rng.choice([1, 2, 4, 8])), Hkv,
+                       16 * int(rng.integers(1, 9)), int(rng.integers(1, 5000)),
+                       int(rng.integers(1, 9))))
+    for B, Hq, Hkv, bs, mbps, nq in shapes:
+        if nq * (Hq // Hkv) > 64:
+            continue
+        d = dims(num_seqs=B, num_q_heads=Hq, num_kv_heads=Hkv, block_size=bs,
+                 max_blocks_per_seq=mbps, num_blocks=mbps * B + 1)
+        have = L.paged_attn_workspace_size(ctypes.byref(d), nq)
+        assert have > 0
+        for kv_dtype in (0, 1):
+            for sms in list(range(1, 300)) + [512, 1024]:
+                need = _ws_needed(B, Hq, Hkv, nq, _plan_splits(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms))
+                assert have >= need, (B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms, have, need)
