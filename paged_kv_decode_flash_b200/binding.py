@@ -112,6 +112,17 @@ def _dptr(t: torch.Tensor | None) -> int | None:
     return t.data_ptr()
 
 
+def _expect(t: torch.Tensor, name: str, dtype, shape) -> None:
+    """The C ABI takes bare pointers: a tensor of the wrong type or size
+    would be read out of bounds, so it is refused here."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def cache_block_size(k_cache: torch.Tensor, kv_dtype: int, head_dim: int) -> int:
     if kv_dtype == KV_FP16:
         return int(k_cache.shape[2])
@@ -166,8 +177,34 @@ class PagedDecode:
             raise PagedAttnError(n, "launches_per_call")
         return n
 
+    def check_args(self, q, k_cache, v_cache, block_table, context_lens, kv_dtype, out=None):
+        """dtype, shape and device of every tensor a decode call reads or
+        writes, against this configuration (include/pagedattn.h layouts)."""
+        d = self.dims
+        B, nq, Hq, Hkv, D = d.num_seqs, self.n_query, d.num_q_heads, d.num_kv_heads, d.head_dim
+        _expect(q, "q", torch.float16, (B, nq, Hq, D))
+        if out is not None:
+            _expect(out, "out", torch.float16, (B, nq, Hq, D))
+        _expect(block_table, "block_table", torch.int32, (B, d.max_blocks_per_seq))
+        _expect(context_lens, "context_lens", torch.int32, (B,))
+        if int(kv_dtype) == KV_FP16:
+            cache = (torch.float16, (d.num_blocks, Hkv, d.block_size, D))
+        elif int(kv_dtype) == KV_Q8_0:
+            cache = (torch.uint8, (d.num_blocks, Hkv, d.block_size * (D + 2 * (D // 32))))
+        else:
+            raise ValueError(f"kv_dtype {kv_dtype}: expected {KV_FP16} (fp16) or {KV_Q8_0} (q8_0)")
+        _expect(k_cache, "k_cache", *cache)
+        _expect(v_cache, "v_cache", *cache)
+        dev = self.workspace.device
+        for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache),
+                        ("block_table", block_table), ("context_lens", context_lens),
+                        ("out", out)):
+            if t is not None and t.device != dev:
+                raise ValueError(f"{name} is on {t.device}, the workspace on {dev}")
+
     def __call__(self, q, k_cache, v_cache, block_table, context_lens, *, causal: int,
                  window: int, scale: float, kv_dtype: int, out=None, stream=None):
+        self.check_args(q, k_cache, v_cache, block_table, context_lens, kv_dtype, out)
         if out is None:
             out = torch.empty_like(q)
         rc = lib().paged_attn_decode(
@@ -183,6 +220,8 @@ class PagedDecode:
 
     def trace(self, block_table, context_lens, *, causal: int, window: int, stream=None):
         B, nq, Hq = self.dims.num_seqs, self.n_query, self.dims.num_q_heads
+        _expect(block_table, "block_table", torch.int32, (B, self.dims.max_blocks_per_seq))
+        _expect(context_lens, "context_lens", torch.int32, (B,))
         t = torch.empty((B, nq, Hq, 5), dtype=torch.int32, device=block_table.device)
         rc = lib().paged_attn_trace(ctypes.byref(self.dims), _dptr(block_table),
                                     _dptr(context_lens), nq, int(causal), int(window),
@@ -196,6 +235,12 @@ def merge(partial_out: torch.Tensor, partial_lse: torch.Tensor, out=None, out_ls
     """partial_out fp32 [S][rows][D], partial_lse fp32 [S][rows] ->
     (out fp16 [rows][D], out_lse fp32 [rows])."""
     S, rows, D = partial_out.shape
+    _expect(partial_out, "partial_out", torch.float32, (S, rows, D))
+    _expect(partial_lse, "partial_lse", torch.float32, (S, rows))
+    if out is not None:
+        _expect(out, "out", torch.float16, (rows, D))
+    if out_lse is not None:
+        _expect(out_lse, "out_lse", torch.float32, (rows,))
     if out is None:
         out = torch.empty((rows, D), dtype=torch.float16, device=partial_out.device)
     if out_lse is None:

@@ -173,3 +173,37 @@ def test_workspace_size_covers_every_plan(L):
             for sms in list(range(1, 300)) + [512, 1024]:
                 need = _ws_needed(B, Hq, Hkv, nq, _plan_splits(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms))
                 assert have >= need, (B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms, have, need)
+
+
+def test_binding_refuses_tensors_the_kernel_would_read_out_of_bounds():
+    """The C ABI takes bare pointers, so the binding checks dtype, shape and
+    device of every tensor against the configuration before a call."""
+    import torch
+    from paged_kv_decode_flash_b200 import binding as b
+    dec = object.__new__(b.PagedDecode)  # no device: the checks only
+    dec.n_query = 4
+    dec.dims = b.Dims(2, 16, 4, 128, 16, 10, 25, None, 0)
+    dec.workspace = torch.empty(1024, dtype=torch.uint8)
+    f16, i32 = torch.float16, torch.int32
+    good = dict(q=torch.empty(2, 4, 16, 128, dtype=f16),
+                k_cache=torch.empty(25, 4, 16, 128, dtype=f16),
+                v_cache=torch.empty(25, 4, 16, 128, dtype=f16),
+                block_table=torch.empty(2, 10, dtype=i32),
+                context_lens=torch.empty(2, dtype=i32))
+    dec.check_args(kv_dtype=b.KV_FP16, out=None, **good)
+    q8 = torch.empty(25, 4, 16 * 136, dtype=torch.uint8)
+    dec.check_args(kv_dtype=b.KV_Q8_0, out=None, **{**good, "k_cache": q8, "v_cache": q8})
+    bad = [("q", torch.empty(2, 4, 16, 64, dtype=f16)),              # wrong head_dim
+           ("q", torch.empty(2, 4, 16, 128, dtype=torch.float32)),   # wrong dtype
+           ("k_cache", torch.empty(24, 4, 16, 128, dtype=f16)),      # fewer blocks than num_blocks
+           ("v_cache", q8),                                          # q8_0 bytes given as fp16
+           ("block_table", torch.empty(2, 9, dtype=i32)),            # short rows
+           ("block_table", torch.empty(2, 10, dtype=torch.int64)),
+           ("context_lens", torch.empty(3, dtype=i32))]
+    for name, t in bad:
+        with pytest.raises(ValueError, match=name):
+            dec.check_args(kv_dtype=b.KV_FP16, out=None, **{**good, name: t})
+    with pytest.raises(ValueError, match="out"):
+        dec.check_args(kv_dtype=b.KV_FP16, out=torch.empty(2, 4, 16, 127, dtype=f16), **good)
+    with pytest.raises(ValueError, match="kv_dtype"):
+        dec.check_args(kv_dtype=7, out=None, **good)
