@@ -27,7 +27,8 @@ def orc():
 def B():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from paged_kv_decode_flash_b200 import binding
+    from paged_kv_decode_flash_b200 import binding, build
+    build.build()  # no-op when the in-tree library is up to date
     binding.lib()
     return binding
 

@@ -27,7 +27,8 @@ pytestmark = pytest.mark.gpu
 def B():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from paged_kv_decode_flash_b200 import binding
+    from paged_kv_decode_flash_b200 import binding, build
+    build.build()  # no-op when the in-tree library is up to date
     L = binding.lib()
     f = L.paged_attn_decode_noalloc
     vp, i32 = ctypes.c_void_p, ctypes.c_int32
