@@ -45,8 +45,9 @@
  *                   d = amax / 127 <= 516): larger ones give non-finite rows
  *   block_table   int32 [num_seqs][max_blocks_per_seq]
  *   context_lens  int32 [num_seqs]
- * Supported: head_dim 128; block_size a multiple of 16 up to 128; n_query
- * 1..8; num_q_heads a multiple of num_kv_heads with
+ * Supported: head_dim 128; block_size a multiple of 16 (the kernels work in
+ * 16-key chunks; sizes 16 to 112 are exercised by the tests); n_query 1..8;
+ * num_q_heads a multiple of num_kv_heads with
  * n_query * num_q_heads / num_kv_heads <= 64.
  *
  * Ownership and synchronisation: the caller owns every buffer, including the
@@ -95,7 +96,7 @@ typedef struct {
   int32_t num_q_heads;        /* Hq */
   int32_t num_kv_heads;       /* Hkv; Hq % Hkv == 0 */
   int32_t head_dim;           /* 128 */
-  int32_t block_size;         /* tokens per KV block; multiple of 16, <= 128 */
+  int32_t block_size;         /* tokens per KV block; a multiple of 16 */
   int32_t max_blocks_per_seq; /* row stride of block_table */
   int32_t num_blocks;         /* physical blocks in the pool (bounds check) */
   void* workspace;            /* device, caller-owned, 256-byte aligned */
