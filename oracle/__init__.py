@@ -91,6 +91,16 @@ class Oracle:
         lib.oracle_merge.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_float_to_half.argtypes = [ctypes.c_float]
+        lib.oracle_float_to_half.restype = ctypes.c_uint16
+        lib.oracle_quantize_q8_0.argtypes = [vp, vp, vp]
+        lib.oracle_quantize_q8_0.restype = None
+        lib.oracle_quantize_row.argtypes = [vp, i32, vp, vp]
+        lib.oracle_quantize_row.restype = None
+        lib.oracle_cache_write.argtypes = [P, vp, vp, vp, vp]
+        lib.oracle_cache_write.restype = ctypes.c_int
         self.lib = lib
 
     # -- helpers -----------------------------------------------------------
@@ -115,6 +125,44 @@ class Oracle:
 
     def num_threads(self) -> int:
         return self.lib.oracle_num_threads()
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
+
+    # -- quantise on write ---------------------------------------------------
+    def float_to_half(self, f) -> int:
+        """fp16 bits of an fp32 value, round to nearest even."""
+        return int(self.lib.oracle_float_to_half(float(np.float32(f))))
+
+    def quantize_q8_0(self, x32: np.ndarray):
+        """32 fp32 values -> (int8 q[32], fp16 scale bits)."""
+        x = np.ascontiguousarray(x32, dtype=np.float32)
+        assert x.size == 32
+        q = np.zeros(32, dtype=np.int8)
+        d = np.zeros(1, dtype=np.uint16)
+        self.lib.oracle_quantize_q8_0(_ptr(x), _ptr(q), _ptr(d))
+        return q, int(d[0])
+
+    def quantize_row(self, x: np.ndarray):
+        """n fp32 values -> (int8 q[n], fp32 scale)."""
+        xx = np.ascontiguousarray(x, dtype=np.float32)
+        q = np.zeros(xx.size, dtype=np.int8)
+        sc = np.zeros(1, dtype=np.float32)
+        self.lib.oracle_quantize_row(_ptr(xx), xx.size, _ptr(q), _ptr(sc))
+        return q, float(sc[0])
+
+    def cache_write(self, case, k_new: np.ndarray, v_new: np.ndarray):
+        """The case's caches after writing k_new/v_new (fp16 [B][n_new][Hkv][D],
+        n_new = case.n_query) for the last n_new positions of every sequence.
+        Returns (k_cache, v_cache, status)."""
+        keep: list = []
+        p = self._problem(case, keep)
+        kc = np.ascontiguousarray(case.k_cache).copy()
+        vc = np.ascontiguousarray(case.v_cache).copy()
+        kn = np.ascontiguousarray(k_new, dtype=np.float16).view(np.uint16)
+        vn = np.ascontiguousarray(v_new, dtype=np.float16).view(np.uint16)
+        rc = self.lib.oracle_cache_write(ctypes.byref(p), _ptr(kn), _ptr(vn), _ptr(kc), _ptr(vc))
+        return kc, vc, int(rc)
 
     # -- the computation ---------------------------------------------------
     def attend(self, case):

@@ -34,6 +34,14 @@
  *  - query head h reads KV head h / (num_q_heads / num_kv_heads);
  *  - q8_0: value = int8 q times the fp16 scale d of its group of 32
  *    consecutive head_dim elements (exact in fp64);
+ *  - int8 with row scales ("Prefill: teach the fork's fast kernel to read
+ *    the int8 cache": vLLM's int8 cache has per-row scales): value = int8 q
+ *    times the fp32 scale of its (token, head) row (exact in fp64);
+ *  - writing new tokens into the cache (the step before attention; "Bug 2":
+ *    vLLM's cache manager assigns the blocks) quantises in fp32 with IEEE
+ *    rounding, the precision the kernel decides in: q8_0 d = fp16(amax/127)
+ *    per 32 elements, int8 rows s = amax/127 per row, q = round half away
+ *    from zero of x / d (or x / s), clamped to [-127, 127];
  *  - lse is the natural log of sum_j exp(scale * q.k_j).
  *
  * Building with -DORACLE_PLANT=n plants one deliberate mistake (used only by
@@ -113,6 +121,18 @@ static double cache_value(const oracle_problem* p, const void* cache,
     const int64_t row = (block * H + kvh) * bs + slot;
 #endif
     return oracle_half_to_double(c[row * D + d]);
+  } else if (p->kv_dtype == ORACLE_KV_INT8_ROW) {
+    /* int8 with one fp32 scale per (token, head) row: value = q * s */
+    const int64_t tile_bytes = bs * D + bs * 4;
+    const uint8_t* tile = (const uint8_t*)cache + (block * H + kvh) * tile_bytes;
+    const int8_t q = (int8_t)tile[(int64_t)slot * D + d];
+    float s;
+#if ORACLE_PLANT == 9
+    memcpy(&s, tile + bs * D + (int64_t)((slot + 1) % bs) * 4, 4); /* planted: neighbour's scale */
+#else
+    memcpy(&s, tile + bs * D + (int64_t)slot * 4, 4);
+#endif
+    return (double)q * (double)s;
   } else {
     const int64_t groups = D / 32;
     const int64_t tile_bytes = bs * D + bs * groups * 2;
@@ -138,7 +158,8 @@ static int check_problem(const oracle_problem* p) {
       p->num_blocks <= 0 || p->n_query <= 0 || p->window < 0)
     return ORACLE_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads != 0) return ORACLE_ERR_INVALID_ARG;
-  if (p->kv_dtype != ORACLE_KV_FP16 && p->kv_dtype != ORACLE_KV_Q8_0)
+  if (p->kv_dtype != ORACLE_KV_FP16 && p->kv_dtype != ORACLE_KV_Q8_0 &&
+      p->kv_dtype != ORACLE_KV_INT8_ROW)
     return ORACLE_ERR_INVALID_ARG;
   if (p->kv_dtype == ORACLE_KV_Q8_0 && p->head_dim % 32 != 0)
     return ORACLE_ERR_INVALID_ARG;
@@ -353,4 +374,164 @@ int oracle_num_threads(void) {
 #else
   return 1;
 #endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+/* ---------------------------------------------------------------------------
+ * Writing new tokens into the cache (quantise on write).
+ * -------------------------------------------------------------------------*/
+
+/* fp32 -> fp16 bits, round to nearest, ties to even (IEEE 754 binary16),
+ * from the bit patterns.  A finite fp32 value is sig * 2^(E - 23) with sig
+ * its 24-bit significand (implicit bit included) and E its unbiased
+ * exponent.  In fp16 it becomes q units of 2^(E - 10) (normal range,
+ * E >= -14) or of 2^-24 (subnormal), q = sig rounded to the shift that
+ * drops the bits below that unit; the fp16 bits are then (E + 14) * 2^10 + q
+ * (normal: q in [2^10, 2^11], where q = 2^11 carries into the exponent) or
+ * q itself (subnormal: q = 2^10 is the smallest normal), infinity from
+ * 0x7c00 up. */
+uint16_t oracle_float_to_half(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  const int32_t exp = (int32_t)((u >> 23) & 0xffu);
+  const uint32_t mant = u & 0x7fffffu;
+  if (exp == 0xff) return (uint16_t)(sign | 0x7c00u | (mant ? 0x200u : 0u)); /* inf, NaN */
+  const uint32_t sig = exp ? (mant | 0x800000u) : mant;
+  const int32_t E = (exp ? exp : 1) - 127;
+  int32_t shift;
+  uint32_t base;
+  if (E >= -14) {
+    shift = 13;
+    base = (uint32_t)(E + 14) << 10;
+  } else {
+    shift = 13 + (-14 - E);
+    base = 0;
+  }
+  uint32_t q = 0;
+  if (shift < 25) { /* otherwise sig < 2^24 <= half a unit: rounds to 0 */
+    q = sig >> shift;
+    const uint32_t rem = sig & ((1u << shift) - 1u), half = 1u << (shift - 1);
+#if ORACLE_PLANT == 12
+    (void)rem; (void)half; /* planted: truncation instead of rounding */
+#else
+    if (rem > half || (rem == half && (q & 1u))) q += 1u;
+#endif
+  }
+  uint32_t bits = base + q;
+  if (bits >= 0x7c00u) bits = 0x7c00u;
+  return (uint16_t)(sign | bits);
+}
+
+static float half_to_float(uint16_t h) { return (float)oracle_half_to_double(h); }
+
+static int8_t quant_one(float x, float d) {
+  if (!(d > 0.0f)) return 0;
+#if ORACLE_PLANT == 10
+  float r = truncf(x / d); /* planted: rounding toward zero */
+#else
+  float r = roundf(x / d); /* round half away from zero */
+#endif
+  if (r > 127.0f) r = 127.0f;
+  if (r < -127.0f) r = -127.0f;
+  return (int8_t)r;
+}
+
+void oracle_quantize_q8_0(const float* x, int8_t* q, uint16_t* d_bits) {
+  float amax = 0.0f;
+  for (int i = 0; i < 32; ++i) {
+    const float a = fabsf(x[i]);
+    if (a > amax) amax = a;
+  }
+  const uint16_t dh = oracle_float_to_half(amax / 127.0f);
+  const float d = half_to_float(dh);
+  for (int i = 0; i < 32; ++i) q[i] = quant_one(x[i], d);
+  *d_bits = dh;
+}
+
+void oracle_quantize_row(const float* x, int32_t n, int8_t* q, float* s_out) {
+  float amax = 0.0f;
+  for (int32_t i = 0; i < n; ++i) {
+    const float a = fabsf(x[i]);
+    if (a > amax) amax = a;
+  }
+  const float s = amax / 127.0f;
+  for (int32_t i = 0; i < n; ++i) q[i] = quant_one(x[i], s);
+  *s_out = s;
+}
+
+int oracle_cache_write(const oracle_problem* p, const uint16_t* k_new, const uint16_t* v_new,
+                       void* k_cache, void* v_cache) {
+  if (!p || !k_new || !v_new || !k_cache || !v_cache || !p->block_table || !p->context_lens)
+    return ORACLE_ERR_INVALID_ARG;
+  if (p->num_kv_heads <= 0 || p->head_dim <= 0 || p->head_dim % 32 != 0 || p->block_size <= 0 ||
+      p->n_query <= 0)
+    return ORACLE_ERR_INVALID_ARG;
+  const int64_t D = p->head_dim, bs = p->block_size, H = p->num_kv_heads;
+  int first_err = ORACLE_OK;
+  float* x = (float*)malloc(sizeof(float) * D);
+  int8_t* q = (int8_t*)malloc((size_t)D);
+  if (!x || !q) {
+    free(x); free(q);
+    return ORACLE_ERR_NOMEM;
+  }
+  for (int32_t s = 0; s < p->num_seqs; ++s) {
+    const int64_t L = p->context_lens[s];
+    if (L < p->n_query || L > (int64_t)p->max_blocks_per_seq * bs) {
+      if (!first_err) first_err = ORACLE_ERR_BAD_CONTEXT_LEN;
+      continue;
+    }
+    for (int32_t i = 0; i < p->n_query; ++i) {
+#if ORACLE_PLANT == 11
+      const int64_t pos = L - p->n_query + i - (i > 0); /* planted: positions off by one */
+#else
+      const int64_t pos = L - p->n_query + i;
+#endif
+      int64_t b;
+      int32_t slot;
+      if (resolve_key(p, s, pos, &b, &slot)) {
+        if (!first_err) first_err = ORACLE_ERR_BAD_BLOCK_INDEX;
+        continue;
+      }
+      for (int32_t h = 0; h < H; ++h) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint16_t* src = (kv ? v_new : k_new) + (((int64_t)s * p->n_query + i) * H + h) * D;
+          void* cache = kv ? v_cache : k_cache;
+          if (p->kv_dtype == ORACLE_KV_FP16) {
+            uint16_t* c = (uint16_t*)cache + ((b * H + h) * bs + slot) * D;
+            memcpy(c, src, (size_t)D * 2);
+            continue;
+          }
+          for (int64_t e = 0; e < D; ++e) x[e] = half_to_float(src[e]);
+          if (p->kv_dtype == ORACLE_KV_Q8_0) {
+            const int64_t tb = bs * D + bs * (D / 32) * 2;
+            uint8_t* tile = (uint8_t*)cache + (b * H + h) * tb;
+            for (int64_t g = 0; g < D / 32; ++g) {
+              uint16_t dh;
+              oracle_quantize_q8_0(x + 32 * g, q + 32 * g, &dh);
+              memcpy(tile + bs * D + ((int64_t)slot * (D / 32) + g) * 2, &dh, 2);
+            }
+            memcpy(tile + (int64_t)slot * D, q, (size_t)D);
+          } else {
+            const int64_t tb = bs * D + bs * 4;
+            uint8_t* tile = (uint8_t*)cache + (b * H + h) * tb;
+            float sc;
+            oracle_quantize_row(x, (int32_t)D, q, &sc);
+            memcpy(tile + (int64_t)slot * D, q, (size_t)D);
+            memcpy(tile + bs * D + (int64_t)slot * 4, &sc, 4);
+          }
+        }
+      }
+    }
+  }
+  free(x);
+  free(q);
+  return first_err;
 }

@@ -24,7 +24,7 @@
 extern "C" {
 #endif
 
-enum { ORACLE_KV_FP16 = 0, ORACLE_KV_Q8_0 = 1 };
+enum { ORACLE_KV_FP16 = 0, ORACLE_KV_Q8_0 = 1, ORACLE_KV_INT8_ROW = 2 };
 
 enum {
   ORACLE_OK = 0,
@@ -40,6 +40,9 @@ enum {
  *                q8_0:  bytes [num_blocks][num_kv_heads][tile], one tile =
  *                       int8 qs[block_size][head_dim] followed by
  *                       fp16 d[block_size][head_dim/32]
+ *                int8 rows: bytes [num_blocks][num_kv_heads][tile], one tile =
+ *                       int8 qs[block_size][head_dim] followed by
+ *                       fp32 s[block_size]
  *   block_table  int32 [num_seqs][max_blocks_per_seq]
  *   context_lens int32 [num_seqs]; includes the n_query new tokens
  */
@@ -90,8 +93,29 @@ int oracle_trace(const oracle_problem* p, int32_t* trace);
 void oracle_merge(const double* part_out, const double* part_lse, int32_t S,
                   int64_t rows, int32_t D, double* out, double* out_lse);
 
-/* Threads an oracle_paged_attn call will use. */
+/* Threads an oracle_paged_attn call will use; oracle_set_num_threads
+ * changes it (n >= 1). */
 int oracle_num_threads(void);
+void oracle_set_num_threads(int n);
+
+/* Quantise-on-write, fp32 arithmetic with IEEE rounding:
+ *   oracle_float_to_half: fp32 -> fp16 bits, round to nearest even;
+ *   oracle_quantize_q8_0: 32 values -> int8 q[32] and the fp16 scale
+ *     d = fp16(amax / 127), q = clamp(round_half_away(x / d), -127, 127)
+ *     (all zero when d = 0);
+ *   oracle_quantize_row: n values -> int8 q[n] and the fp32 scale
+ *     s = amax / 127, q likewise with s.
+ * oracle_cache_write: for every sequence s, new token i < p->n_query (the
+ * last n_query positions of context_lens[s]) and KV head h, write row
+ * k_new/v_new [s][i][h][:] (fp16 bits, [num_seqs][n_query][Hkv][head_dim])
+ * into its slot of k_cache / v_cache (p->kv_dtype layout), quantised as
+ * above.  Rows with a bad context length or block index are skipped and the
+ * first such error is returned. */
+uint16_t oracle_float_to_half(float f);
+void oracle_quantize_q8_0(const float* x, int8_t* q, uint16_t* d_bits);
+void oracle_quantize_row(const float* x, int32_t n, int8_t* q, float* s);
+int oracle_cache_write(const oracle_problem* p, const uint16_t* k_new, const uint16_t* v_new,
+                       void* k_cache, void* v_cache);
 
 #ifdef __cplusplus
 }

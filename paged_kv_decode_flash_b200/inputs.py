@@ -23,6 +23,8 @@ Layouts (contiguous, row-major):
   q8_0 cache       uint8 [num_blocks][num_kv_heads][tile]; tile =
                    int8 qs[block_size][head_dim] then
                    fp16 d[block_size][head_dim // 32]
+  int8-row cache   uint8 [num_blocks][num_kv_heads][tile]; tile =
+                   int8 qs[block_size][head_dim] then fp32 s[block_size]
   block_table      int32 [num_seqs][max_blocks_per_seq]
   context_lens     int32 [num_seqs]  (includes the n_query new tokens)
 """
@@ -35,6 +37,7 @@ import numpy as np
 
 KV_FP16 = 0
 KV_Q8_0 = 1
+KV_INT8_ROW = 2
 
 
 @dataclasses.dataclass
@@ -70,11 +73,24 @@ class Case:
         """Bytes of K plus V one key of one KV head occupies in the cache."""
         if self.kv_dtype == KV_FP16:
             return 2 * 2 * self.head_dim
-        return 2 * (self.head_dim + 2 * (self.head_dim // 32))
+        if self.kv_dtype == KV_Q8_0:
+            return 2 * (self.head_dim + 2 * (self.head_dim // 32))
+        return 2 * (self.head_dim + 4)
 
 
 def q8_0_tile_bytes(block_size: int, head_dim: int) -> int:
     return block_size * head_dim + block_size * (head_dim // 32) * 2
+
+
+def int8_row_tile_bytes(block_size: int, head_dim: int) -> int:
+    return block_size * head_dim + block_size * 4
+
+
+def cache_tile_bytes(kv_dtype: int, block_size: int, head_dim: int) -> int:
+    """Bytes per (block, KV head) of a quantised cache."""
+    if kv_dtype == KV_Q8_0:
+        return q8_0_tile_bytes(block_size, head_dim)
+    return int8_row_tile_bytes(block_size, head_dim)
 
 
 def quantise_q8_0(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -93,6 +109,29 @@ def quantise_q8_0(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     qv = np.sign(r) * np.floor(np.abs(r) + 0.5)
     qv = np.clip(qv, -127, 127).astype(np.int8).reshape(shp)
     return qv, d16
+
+
+def quantise_rows(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Quantise each row (last axis) with one scale: s = fp32(amax / 127);
+    q = clamp(round_half_away(x / s), -127, 127); an all-zero row gets s = 0,
+    q = 0.  Returns (int8 q, float32 s)."""
+    g = x.astype(np.float64)
+    amax = np.abs(g).max(axis=-1)
+    s32 = (amax / 127.0).astype(np.float32)
+    sc = s32.astype(np.float64)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(sc > 0, g / np.where(sc > 0, sc, 1.0), 0.0)
+    qv = np.clip(np.sign(r) * np.floor(np.abs(r) + 0.5), -127, 127).astype(np.int8)
+    return qv, s32
+
+
+def pack_int8_rows(qs: np.ndarray, sc: np.ndarray) -> np.ndarray:
+    """qs int8 [NB][H][bs][D], sc fp32 [NB][H][bs] -> uint8 tiles."""
+    nb, h, bs, dim = qs.shape
+    out = np.empty((nb, h, int8_row_tile_bytes(bs, dim)), dtype=np.uint8)
+    out[:, :, : bs * dim] = qs.reshape(nb, h, bs * dim).view(np.uint8)
+    out[:, :, bs * dim:] = np.ascontiguousarray(sc, dtype=np.float32).reshape(nb, h, bs).view(np.uint8)
+    return out
 
 
 def pack_q8_0(qs: np.ndarray, d: np.ndarray) -> np.ndarray:
@@ -127,6 +166,7 @@ def make_case(
     spare_blocks: int = 0,
     poison: bool = True,
     nan_below: list[int] | None = None,
+    nan_keys_below: list[int] | None = None,
     spike_frac: float = 0.0,
     spike_gain: float = 8.0,
     q_std: float = 1.0,
@@ -140,7 +180,9 @@ def make_case(
     entry points to are filled with NaN: a kernel that reads any of them
     produces NaN.  ``nan_below[s]`` additionally NaN-fills every block of
     sequence s whose keys all lie below that position (used for sliding
-    windows).  ``spike_frac`` scales round(frac * L) seeded key rows per
+    windows).  ``nan_keys_below[s]`` NaN-fills every key of sequence s below
+    that position, key by key (also inside a block that holds visible keys).
+    ``spike_frac`` scales round(frac * L) seeded key rows per
     (sequence, KV head) by ``spike_gain`` before rounding to fp16.
     """
     rng = np.random.default_rng(seed)
@@ -193,6 +235,10 @@ def make_case(
             full = lo // bs  # logical blocks [0, full) end at or below lo - 1
             if full > 0:
                 bad[table[s, :full], :] = True
+    if nan_keys_below is not None:
+        for s in range(B):
+            for j in range(min(int(nan_keys_below[s]), int(L[s]))):
+                bad[table[s, j // bs], j % bs] = True
 
     if kv_dtype == KV_FP16:
         k = np.ascontiguousarray(k32.astype(np.float16).transpose(0, 2, 1, 3))  # [NB][bs][H][D]
@@ -201,6 +247,15 @@ def make_case(
         v[bad] = np.float16(np.nan)
         k = np.ascontiguousarray(k.transpose(0, 2, 1, 3))  # back to [NB][H][bs][D]
         v = np.ascontiguousarray(v.transpose(0, 2, 1, 3))
+    elif kv_dtype == KV_INT8_ROW:
+        kq, ks = quantise_rows(k32)   # [NB][H][bs][D], [NB][H][bs]
+        vq, vs = quantise_rows(v32)
+        ks = ks.transpose(0, 2, 1).copy()
+        vs = vs.transpose(0, 2, 1).copy()
+        ks[bad] = np.float32(np.nan)  # a NaN scale poisons the whole row
+        vs[bad] = np.float32(np.nan)
+        k = pack_int8_rows(kq, np.ascontiguousarray(ks.transpose(0, 2, 1)))
+        v = pack_int8_rows(vq, np.ascontiguousarray(vs.transpose(0, 2, 1)))
     else:
         kq, kd = quantise_q8_0(k32)
         vq, vd = quantise_q8_0(v32)

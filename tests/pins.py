@@ -16,7 +16,11 @@ What pins what:
   * invariants -- physical block permutation, NaN in never-visible memory,
     batch versus each sequence alone, causal == non-causal at one query token,
     merge of arbitrary key splits == one pass;
-  * exact decoding -- all 65536 fp16 bit patterns against numpy's float16.
+  * exact decoding -- all 65536 fp16 bit patterns against numpy's float16;
+  * quantise on write -- fp32 -> fp16 conversion against numpy on every
+    exponent and on exact ties; hand-worked q8_0 groups and int8 rows, the
+    half-step error bound, the generator's float64 rule away from fp32
+    near-ties; a cache write read back through a one-key window.
 """
 from __future__ import annotations
 
@@ -45,6 +49,13 @@ def dense_kv(case, s: int, which: str) -> np.ndarray:
     cache = case.k_cache if which == "k" else case.v_cache
     if case.kv_dtype == gen.KV_FP16:
         x = cache[phys, :, slot, :].astype(np.float64)  # [L][H][D]
+    elif case.kv_dtype == gen.KV_INT8_ROW:
+        nt = cache[phys]  # [L][H][tile]
+        qs = nt[:, :, : bs * D].view(np.int8).reshape(L, H, bs, D)
+        qs = qs[np.arange(L), :, slot, :].astype(np.float64)  # [L][H][D]
+        sc = np.ascontiguousarray(nt[:, :, bs * D:]).view(np.float32).reshape(L, H, bs)
+        sc = sc[np.arange(L), :, slot].astype(np.float64)  # [L][H]
+        x = qs * sc[:, :, None]
     else:
         nt = cache[phys]  # [L][H][tile]
         qs = nt[:, :, : bs * D].view(np.int8).reshape(L, H, bs, D)
@@ -129,7 +140,7 @@ def check_golden_worked_example(orc):
 
 
 def check_single_key(orc):
-    for dt in (gen.KV_FP16, gen.KV_Q8_0):
+    for dt in (gen.KV_FP16, gen.KV_Q8_0, gen.KV_INT8_ROW):
         # L = 1: the only key is visible; output must equal its value exactly.
         case = gen.make_case(seed=11, context_lens=(1,), n_query=1, num_q_heads=4,
                              num_kv_heads=2, kv_dtype=dt, spare_blocks=3)
@@ -191,7 +202,7 @@ def _random_cases(seed_base=100):
         Hkv = [1, 2][t % 2]
         G = [1, 2, 4][t % 3]
         bs = [16, 32][t % 2]
-        dt = gen.KV_Q8_0 if t % 5 == 4 else gen.KV_FP16
+        dt = gen.KV_Q8_0 if t % 5 == 4 else gen.KV_INT8_ROW if t % 5 == 2 else gen.KV_FP16
         lens = tuple(int(x) for x in rng.integers(nq, 64, size=1 + t % 3))
         yield gen.make_case(seed=seed_base + t, context_lens=lens, n_query=nq,
                             num_q_heads=Hkv * G, num_kv_heads=Hkv, block_size=bs,
@@ -245,25 +256,166 @@ def check_block_permutation(orc):
     assert np.array_equal(out, out2) and np.array_equal(lse, lse2), "block permutation changed result"
 
 
+def zero_nans(case):
+    """The case with every NaN of its caches replaced by 0 (fp16 values; the
+    scales of the int8 caches)."""
+    clean = gen.Case(**case.__dict__)
+    if case.kv_dtype == gen.KV_FP16:
+        clean.k_cache = np.nan_to_num(case.k_cache, nan=0.0)
+        clean.v_cache = np.nan_to_num(case.v_cache, nan=0.0)
+        return clean
+    sdt = np.float16 if case.kv_dtype == gen.KV_Q8_0 else np.float32
+    for name in ("k_cache", "v_cache"):
+        c = getattr(case, name).copy()
+        d = c[:, :, case.block_size * case.head_dim:].view(sdt)
+        d[np.isnan(d)] = 0.0
+        setattr(clean, name, c)
+    return clean
+
+
 def check_nan_invariance(orc):
-    for dt in (gen.KV_FP16, gen.KV_Q8_0):
-        case = gen.make_case(seed=17, context_lens=(100, 57), n_query=3, num_q_heads=4,
-                             num_kv_heads=2, causal=0, window=40, kv_dtype=dt,
-                             spare_blocks=3, nan_below=[100 - 40, 57 - 40])
-        out, lse = orc.attend(case)
-        assert np.all(np.isfinite(out)), "NaN leaked from never-visible memory"
-        clean = gen.Case(**case.__dict__)
-        if dt == gen.KV_FP16:
-            clean.k_cache = np.nan_to_num(case.k_cache, nan=0.0)
-            clean.v_cache = np.nan_to_num(case.v_cache, nan=0.0)
+    for dt in (gen.KV_FP16, gen.KV_Q8_0, gen.KV_INT8_ROW):
+        # whole out-of-window blocks (non-causal window) and, key by key, every
+        # key below the window edge of the earliest query (causal window)
+        for causal, kw in ((0, dict(nan_below=[100 - 40, 57 - 40])),
+                           (1, dict(nan_keys_below=[100 - 3 - 40 + 1, 57 - 3 - 40 + 1]))):
+            case = gen.make_case(seed=17, context_lens=(100, 57), n_query=3, num_q_heads=4,
+                                 num_kv_heads=2, causal=causal, window=40, kv_dtype=dt,
+                                 spare_blocks=3, **kw)
+            out, lse = orc.attend(case)
+            assert np.all(np.isfinite(out)), "NaN leaked from never-visible memory"
+            out2, lse2 = orc.attend(zero_nans(case))
+            assert np.array_equal(out, out2) and np.array_equal(lse, lse2), "NaN-poisoned != zeroed"
+
+
+# ---------------------------------------------------------------------------
+# quantise on write
+# ---------------------------------------------------------------------------
+def _half_midpoint(v32: np.float32) -> bool:
+    """Is the fp32 value exactly halfway between two adjacent fp16 values?"""
+    h = np.float16(v32)
+    if not np.isfinite(h):
+        return False
+    a = np.float64(h)
+    nb = np.nextafter(h, np.float16(np.inf) if np.float64(v32) > a else np.float16(-np.inf))
+    return np.float64(v32) * 2 == a + np.float64(nb)
+
+
+def check_float_to_half(orc):
+    """fp32 -> fp16 round to nearest even, against numpy's conversion: every
+    exponent (normal, subnormal, overflow), random mantissas, exact ties."""
+    rng = np.random.default_rng(40)
+    bits = rng.integers(0, 2 ** 32, size=20000, dtype=np.uint64).astype(np.uint32)
+    exps = rng.integers(100, 145, size=20000).astype(np.uint32)  # around fp16's range
+    bits2 = (bits & np.uint32(0x807FFFFF)) | (exps << np.uint32(23))
+    ties = []
+    for e in range(-26, 17):  # fp16 value k * 2^(e-10) plus half an ulp
+        for k in (1024, 1025, 1500, 2047):
+            ties.append(np.float32((k + 0.5) * 2.0 ** (e - 10)))
+    vals = np.concatenate([bits.view(np.float32), bits2.view(np.float32), np.array(ties, np.float32),
+                           np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, 2 ** -24, 2 ** -25,
+                                     3 * 2 ** -26, np.inf, -np.inf], dtype=np.float32)])
+    for v in vals:
+        with np.errstate(over="ignore"):
+            ref = np.array([v], dtype=np.float32).astype(np.float16).view(np.uint16)[0]
+        got = orc.float_to_half(v)
+        if np.isnan(v):
+            assert (got & 0x7c00) == 0x7c00 and (got & 0x3ff) != 0, "NaN"
         else:
-            for name in ("k_cache", "v_cache"):
-                c = getattr(case, name).copy()
-                d = c[:, :, 16 * case.head_dim:].view(np.float16)
-                d[np.isnan(d)] = 0.0
-                setattr(clean, name, c)
-        out2, lse2 = orc.attend(clean)
-        assert np.array_equal(out, out2) and np.array_equal(lse, lse2), "NaN-poisoned != zeroed"
+            assert got == ref, f"float_to_half({v!r}) = {got:#06x}, numpy {ref:#06x}"
+
+
+def check_quantize_q8_0(orc):
+    """q8_0 on write: hand-worked groups, the error bound, and agreement with
+    the float64 rule of the data generator except where fp32 and fp64 may
+    legitimately differ (an fp32 quotient on an fp16 tie, or x / d within
+    fp32 rounding of a half-integer)."""
+    x = np.zeros(32, np.float32)
+    x[:5] = [127.0, 2.5, -2.5, 0.49, -0.5]  # amax 127 -> d = 1; ties go away from zero
+    q, d = orc.quantize_q8_0(x)
+    assert d == 0x3C00 and q[:5].tolist() == [127, 3, -3, 0, -1], (q[:5], hex(d))
+    x[:] = 0
+    x[:3] = [-254.0, 3.0, 1.0]  # d = 2: 3/2 = 1.5 -> 2, 1/2 -> 1
+    q, d = orc.quantize_q8_0(x)
+    assert d == 0x4000 and q[:3].tolist() == [-127, 2, 1]
+    q, d = orc.quantize_q8_0(np.zeros(32, np.float32))
+    assert d == 0 and not q.any()
+    rng = np.random.default_rng(41)
+    xs = (rng.standard_normal((400, 32)) * rng.choice([1e-3, 1.0, 50.0], size=(400, 1))
+          ).astype(np.float16).astype(np.float32)
+    gq, gd = gen.quantise_q8_0(xs)
+    for r in range(xs.shape[0]):
+        q, d = orc.quantize_q8_0(xs[r])
+        dv = np.float64(np.array([d], np.uint16).view(np.float16)[0])
+        rec = q.astype(np.float64) * dv
+        assert np.all(np.abs(rec - xs[r]) <= 0.5 * dv * (1 + 1e-5) + (np.abs(xs[r]) - 127 * dv).clip(0)), "error bound"
+        if d != gd[r, 0].view(np.uint16):
+            assert _half_midpoint(np.float32(np.abs(xs[r]).max()) / np.float32(127)), f"scale {r}"
+            continue
+        ratio = xs[r].astype(np.float64) / dv
+        near = np.abs(np.abs(ratio) - np.floor(np.abs(ratio)) - 0.5) < 1e-5
+        assert np.array_equal(q[~near], gq[r][~near]), f"codes of group {r}"
+
+
+def check_quantize_row(orc):
+    """int8 rows on write: hand-worked row, the error bound, the generator's
+    float64 rule away from fp32 near-ties."""
+    x = np.zeros(128, np.float32)
+    x[:5] = [127.0, -63.5, 0.5, -0.5, 2.4999]  # s = 1
+    q, sc = orc.quantize_row(x)
+    assert sc == 1.0 and q[:5].tolist() == [127, -64, 1, -1, 2]
+    q, sc = orc.quantize_row(np.zeros(128, np.float32))
+    assert sc == 0.0 and not q.any()
+    rng = np.random.default_rng(42)
+    xs = (rng.standard_normal((200, 128)) * 3).astype(np.float16).astype(np.float32)
+    gq, gs = gen.quantise_rows(xs)
+    for r in range(xs.shape[0]):
+        q, sc = orc.quantize_row(xs[r])
+        assert np.float32(sc) == gs[r] or abs(sc - gs[r]) <= 1.2e-7 * sc, f"scale of row {r}"
+        rec = q.astype(np.float64) * sc
+        assert np.all(np.abs(rec - xs[r]) <= 0.5 * sc * (1 + 1e-5) +
+                      (np.abs(xs[r]) - 127 * np.float64(sc)).clip(0)), "error bound"
+        ratio = xs[r].astype(np.float64) / np.float64(sc)
+        near = np.abs(np.abs(ratio) - np.floor(np.abs(ratio)) - 0.5) < 1e-5
+        assert np.array_equal(q[~near], gq[r][~near]), f"codes of row {r}"
+
+
+def check_cache_write(orc):
+    """Writing the newest tokens: exactly their slots change, and attention
+    with a window of one key returns, for each new token, the value just
+    written (fp16: bit for bit; int8: its quantisation, within half a step)."""
+    for dt in (gen.KV_FP16, gen.KV_Q8_0, gen.KV_INT8_ROW):
+        case = gen.make_case(seed=43, context_lens=(70, 33), n_query=3, num_q_heads=4,
+                             num_kv_heads=2, kv_dtype=dt, spare_blocks=2, causal=1, window=1)
+        rng = np.random.default_rng(44)
+        kn = rng.standard_normal((2, 3, 2, 128)).astype(np.float16)
+        vn = rng.standard_normal((2, 3, 2, 128)).astype(np.float16)
+        kc, vc, rc = orc.cache_write(case, kn, vn)
+        assert rc == 0
+        changed = np.zeros(case.num_blocks, dtype=bool)
+        for s, L in enumerate(case.context_lens.tolist()):
+            for i in range(3):
+                changed[case.block_table[s, (L - 3 + i) // case.block_size]] = True
+        for new_c, old_c in ((kc, case.k_cache), (vc, case.v_cache)):  # bytes: NaN-safe
+            assert np.array_equal(new_c[~changed].view(np.uint8), old_c[~changed].view(np.uint8)), \
+                "other blocks written"
+        w = gen.Case(**{**case.__dict__, "k_cache": kc, "v_cache": vc})
+        out, _ = orc.attend(w)  # window 1: each query returns its own position's value
+        for s in range(2):
+            V = dense_kv(w, s, "v")
+            for i in range(3):
+                for h in range(4):
+                    new = vn[s, i, h // 2].astype(np.float64)
+                    got = out[s, i, h]
+                    assert np.array_equal(got, V[h // 2, int(w.context_lens[s]) - 3 + i])
+                    if dt == gen.KV_FP16:
+                        assert np.array_equal(got, new), "fp16 write not exact"
+                    else:
+                        step = np.abs(new).max() / 127 * (1 + 2 ** -10)
+                        assert np.all(np.abs(got - new) <= 0.5 * step), "int8 write error"
+        bad = gen.Case(**{**case.__dict__, "block_table": case.block_table.copy()})
+        bad.block_table[0, (70 - 1) // case.block_size] = case.num_blocks + 3
+        assert orc.cache_write(bad, kn, vn)[2] != 0, "bad block not reported"
 
 
 def check_batch_equals_alone(orc):
@@ -335,5 +487,6 @@ ALL_CHECKS = [
     check_mean_forms, check_two_keys_logistic, check_dense_bruteforce,
     check_trace_bruteforce, check_block_permutation, check_nan_invariance,
     check_batch_equals_alone, check_causal_single_query, check_merge_of_splits,
-    check_error_codes,
+    check_error_codes, check_float_to_half, check_quantize_q8_0, check_quantize_row,
+    check_cache_write,
 ]

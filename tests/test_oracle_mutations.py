@@ -3,7 +3,8 @@ oracle.c) and check that at least one pin fails for each.  This shows the
 pins would catch a plausible bug in the oracle: a window or causal edge off by
 one, a strided GQA head mapping, swapped cache axes, a dropped scale, a sign
 error in the exponent, the wrong q8_0 group scale, or a dropped term in the
-log-sum-exp."""
+log-sum-exp, the wrong int8 row scale, a quantiser or fp16 conversion that
+truncates, or new tokens written one slot off."""
 import os
 import tempfile
 
@@ -21,6 +22,10 @@ PLANTS = {
     6: "exponent sign flipped",
     7: "q8_0 scale of the wrong group",
     8: "max term dropped from lse",
+    9: "int8 row scale of the neighbouring slot",
+    10: "quantiser rounds toward zero",
+    11: "cache write positions off by one",
+    12: "fp32 -> fp16 truncates",
 }
 
 # The quick checks (skip the 65536-pattern fp16 decode, which no plant touches).
