@@ -1,19 +1,22 @@
 #!/usr/bin/env python3
 """Benchmark of paged-KV decode attention (libpagedattn, B200).
 
-One step = one paged_attn_decode call (split-KV decode + merge) over the
-workload's whole visible KV cache.  Default workload: speculative verify,
+One step = one paged_attn_decode call (split-KV decode with its merge) over
+the workload's whole visible KV cache.  Default workload: speculative verify,
 batch 1, 8 causal query tokens after 61440 cached tokens (L = 61448), 32/8
 heads, head_dim 128, block_size 16, fp16 cache.  The 200k-context decode
 (1 query token, 32/4 heads, L = 196608) is measured the same way and reported
-alongside.
+alongside under "also"; the other configurations under "configs".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--split replicas|context]
 
-N > 1 (launched with torch.distributed.run): every rank runs an independent
-replica of the workload on its own GPU (weak scaling, no data-path
-collective); the time is the max over ranks and the value the sum of all
-ranks' KV bytes over that time.
+N > 1 (launched with torch.distributed.run): --split replicas (default) runs
+an independent replica of the workload on every rank (weak scaling, no
+data-path collective); --split context cuts one long sequence's KV blocks
+across the ranks, each rank computes fp32 partials (O, lse) of its share,
+one all-gather exchanges them and every rank merges (paged_attn_merge).  The
+time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -23,6 +26,7 @@ import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -39,24 +43,48 @@ METRIC = "µs/call and KV-read HBM GB/s (% of B200 peak) at 61k and 200k context
 NOMINAL_HBM_GBS = 8000.0
 PRIMARY = "spec_verify_61k"
 SECONDARY = "decode_200k"
+DRIFT_LIMIT_PCT = 1.5
 WORKLOAD_TEXT = {
     "spec_verify_61k": "speculative verify: B=1, 8 causal query tokens after 61440 cached "
                        "(L=61448), Hq/Hkv=32/8, head_dim 128, block_size 16, fp16 N(0,1), "
                        "seeded random block permutation",
     "decode_200k": "200k-context decode: B=1, 1 query token, Hq/Hkv=32/4, head_dim 128, "
                    "L=196608, block_size 16, fp16 N(0,1) with 1% of keys x8",
-}
-
-
-OTHER_CONFIGS = ("tiny", "sliding_window", "mixed_q8_0")
-CONFIG_TEXT = {
     "tiny": "tiny decode: B=1, 1 query token, Hq/Hkv=8/2, L=1024, block_size 16, fp16, "
             "64 of 128 pool blocks (latency-bound: the whole KV is 1 MB)",
     "sliding_window": "sliding-window drafter: B=1, 8 non-causal query tokens, window 2048 "
                       "of L=24576, Hq/Hkv=32/8, fp16; blocks outside the window hold NaN",
     "mixed_q8_0": "mixed batch: B=8, 4 causal query tokens, L_s ~ U[4096, 65536], "
                   "Hq/Hkv=32/8, q8_0 cache (int8 + fp16 scale per 32)",
+    "mtp_q8_0_61k": "MTP verify over an int8 cache (the pages' decode shape): B=1, 4 causal "
+                    "query tokens x 6 query heads per KV head (24 rows), Hq/Hkv=24/4, "
+                    "L=61448, q8_0 cache",
+    "mtp_int8_row_61k": "the same shape over an int8 cache with fp32 row scales",
+    "verify_64rows_61k": "8-token verify at GQA 8 (64 rows per KV head): B=1, Hq/Hkv=64/8, "
+                         "L=61448, fp16",
 }
+OTHER_CONFIGS = ("tiny", "sliding_window", "mixed_q8_0", "mtp_q8_0_61k", "mtp_int8_row_61k",
+                 "verify_64rows_61k")
+
+
+def make_workload(name, seed=0):
+    if name in gen.CONFIGS:
+        return gen.CONFIGS[name](seed)
+    if name in ("mtp_q8_0_61k", "mtp_int8_row_61k"):
+        dt = gen.KV_Q8_0 if name == "mtp_q8_0_61k" else gen.KV_INT8_ROW
+        return gen.make_case(name=name, seed=seed, context_lens=(61448,), n_query=4,
+                             num_q_heads=24, num_kv_heads=4, causal=1, kv_dtype=dt)
+    if name == "verify_64rows_61k":
+        return gen.make_case(name=name, seed=seed, context_lens=(61448,), n_query=8,
+                             num_q_heads=64, num_kv_heads=8, causal=1)
+    raise KeyError(name)
+
+
+def config_dict(name, world, split="replicas"):
+    """The workload description, the same for both arms."""
+    case = make_workload(name)
+    return {"workload": WORKLOAD_TEXT[name], "kv_bytes_per_step": gen.visible_kv_bytes(case),
+            "parallelism": (f"{split} x{world}" if world > 1 else "single GPU")}
 
 
 def env_int(name, default):
@@ -112,6 +140,24 @@ def job_gbs(kv_bytes_per_rank, world, seconds_per_step):
     """Whole-job KV-read rate: every rank reads its own replica's bytes each
     step (weak scaling), over the slowest rank's time per step."""
     return world * kv_bytes_per_rank / seconds_per_step / 1e9
+
+
+def spread(values):
+    """median, min, max and (max - min) / median in percent of a list."""
+    med = statistics.median(values)
+    return {"median": med, "min": min(values), "max": max(values),
+            "spread_pct": 100.0 * (max(values) - min(values)) / med if med > 0 else 0.0}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 class ClockSampler:
@@ -170,6 +216,39 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
+def read_peak(device, torch, B):
+    """Read-only HBM ceiling of the decode kernel's access pattern: the
+    library's streaming probe (4 KB bulk copies into 32 KB shared-memory
+    slots, one CTA per SM) over 4 GiB, best of 5 (CUDA events)."""
+    import ctypes
+    L = B.lib()
+    f = L.paged_attn_stream_read
+    f.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    nbytes = 4 << 30
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    buf.fill_(1)
+    sink = torch.empty(sms, dtype=torch.int32, device=device)
+    st = torch.cuda.current_stream(device)
+    best = 0.0
+    for it in range(6):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        rc = f(buf.data_ptr(), nbytes, sink.data_ptr(), sms, st.cuda_stream)
+        b.record(st)
+        torch.cuda.synchronize()
+        if rc != 0 or bool((sink == -559038737).any()):  # 0xdeadbeef: a wait timed out
+            return None
+        if it > 0:
+            best = max(best, (nbytes // 32768 * 32768) / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del buf
+    torch.cuda.empty_cache()
+    return {"value": round(best, 1), "unit": "GB/s", "what": "read-only streaming probe "
+            "(paged_attn_stream_read: 4 KB bulk copies into 6 x 32 KB smem slots per SM, "
+            f"{sms} CTAs, 4 GiB, best of 5)"}
+
+
 def bench_ours(args, rank, world, dist):
     import torch
     from paged_kv_decode_flash_b200 import binding as B
@@ -179,11 +258,14 @@ def bench_ours(args, rank, world, dist):
     device = torch.device("cuda", dev_index)
     l2_bytes = torch.cuda.get_device_properties(device).L2_cache_size
 
-    def measure(name, steps, warmup, with_e2e):
-        case = gen.CONFIGS[name](seed=rank)
+    def measure(name, steps, warmup, reps, with_e2e):
+        case = make_workload(name, seed=rank)
         kv_bytes = gen.visible_kv_bytes(case)
         pool_bytes = case.k_cache.nbytes + case.v_cache.nbytes
-        copies = max(2, math.ceil(3 * l2_bytes / pool_bytes))
+        # Inputs larger than L2: enough copies of the pool that the VISIBLE
+        # bytes the rotated calls read add up to 3x L2 (at most 48 GB of copies).
+        copies = max(2, math.ceil(3 * l2_bytes / kv_bytes))
+        copies = max(2, min(copies, int(48e9 // pool_bytes)))
         base = B.case_to_device(case, device)
         pools = [(base["k_cache"], base["v_cache"])]
         for _ in range(copies - 1):
@@ -221,23 +303,26 @@ def bench_ours(args, rank, world, dist):
             graph.replay()
         torch.cuda.synchronize()
 
-        # Timed region: exactly `steps` calls back to back between two events
-        # on the launching stream (barrier + synchronize on both sides).
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
+        # Timed regions: exactly `steps` calls back to back between two events
+        # on the launching stream (barrier + synchronize on both sides); the
+        # first is the reported one, all `reps` give the spread.
+        times = []
         with ClockSampler(dev_index) as clk:
-            if dist:
-                dist.barrier()
-            torch.cuda.synchronize()
-            with torch.cuda.stream(gstream):  # replay() launches on the current stream
-                t0.record(gstream)
-                for _ in range(steps // G):
-                    graph.replay()
-                t1.record(gstream)
-            torch.cuda.synchronize()
-            if dist:
-                dist.barrier()
-        total_ms = t0.elapsed_time(t1)
+            for _ in range(reps):
+                t0 = torch.cuda.Event(enable_timing=True)
+                t1 = torch.cuda.Event(enable_timing=True)
+                if dist:
+                    dist.barrier()
+                torch.cuda.synchronize()
+                with torch.cuda.stream(gstream):  # replay() launches on the current stream
+                    t0.record(gstream)
+                    for _ in range(steps // G):
+                        graph.replay()
+                    t1.record(gstream)
+                torch.cuda.synchronize()
+                if dist:
+                    dist.barrier()
+                times.append(max_over_ranks(t0.elapsed_time(t1), dist, device))
         if dec.get_error(gstream) != 0:
             raise RuntimeError("device reported a data error in the timed region")
         # The same calls launched one by one from Python (reported beside).
@@ -251,7 +336,6 @@ def bench_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         eager_us = ea.elapsed_time(eb) * 1e3 / n_eager
         del graph
-        total_ms = max_over_ranks(total_ms, dist, device)
         # Per-call spread (outside the timed region): events around each call.
         n_ev = min(steps, 300)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -262,38 +346,51 @@ def bench_ours(args, rank, world, dist):
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         per_call = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)  # us
+        rep_us = [t * 1e3 / steps for t in times]
         res = {
             "case": case, "kv_bytes": kv_bytes, "copies": copies, "pool_bytes": pool_bytes,
-            "ms_per_step": total_ms / steps, "eager_us": eager_us, "graph_calls": G,
-            "us_median": per_call[len(per_call) // 2], "us_min": per_call[0],
+            "ms_per_step": times[0] / steps, "rep_us": rep_us, "eager_us": eager_us,
+            "graph_calls": G, "us_median": per_call[len(per_call) // 2], "us_min": per_call[0],
             "us_p90": per_call[min(len(per_call) - 1, int(0.9 * len(per_call)))],
             "clocks": clk.summary(), "splits": dec.num_splits(case.kv_dtype),
             "launches": dec.launches_per_call(case.kv_dtype),
         }
         if with_e2e:
-            res["e2e"] = e2e(case, dec, base, pools[0], steps=min(steps, 500))
+            res["e2e"] = e2e(case, dec, pools[0], steps=min(steps, 500))
         del pools, base
         torch.cuda.empty_cache()
         return res
 
-    def e2e(case, dec, base, pool, steps):
-        """Per step: pinned host -> device copy of the step's inputs (q,
-        block_table, context_lens), the C-ABI decode, device -> pinned host
-        copy of the output, synchronise.  The KV cache is the persistent
-        cache state and stays resident."""
-        hq = torch.from_numpy(case.q).pin_memory()
-        hbt = torch.from_numpy(case.block_table).pin_memory()
-        hcl = torch.from_numpy(case.context_lens).pin_memory()
-        hout = torch.empty(hq.shape, dtype=torch.float16).pin_memory()
-        dq, dbt, dcl = (torch.empty_like(x, device=device) for x in (hq, hbt, hcl))
+    def e2e(case, dec, pool, steps):
+        """Per step, through the library's public call: ONE pinned host ->
+        device copy of the step's inputs (q, block_table and context_lens
+        packed in one buffer), the C-ABI decode, a device -> pinned host copy
+        of the output, synchronise.  The KV cache is the persistent cache
+        state and stays resident."""
+        parts = [("q", case.q), ("block_table", case.block_table),
+                 ("context_lens", case.context_lens)]
+        offs, off = {}, 0
+        for n, a in parts:
+            offs[n] = off
+            off = (off + a.nbytes + 255) // 256 * 256
+        host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        for n, a in parts:
+            host[offs[n]: offs[n] + a.nbytes].copy_(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)))
+        dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+
+        def view(n, a, dt):
+            return dbuf[offs[n]: offs[n] + a.nbytes].view(dt).view(a.shape)
+
+        dq = view("q", case.q, torch.float16)
+        dbt = view("block_table", case.block_table, torch.int32)
+        dcl = view("context_lens", case.context_lens, torch.int32)
+        hout = torch.empty(case.q.shape, dtype=torch.float16).pin_memory()
         dout = torch.empty_like(dq)
         kw = dict(causal=case.causal, window=case.window, scale=case.scale,
                   kv_dtype=case.kv_dtype)
 
         def one():
-            dq.copy_(hq, non_blocking=True)
-            dbt.copy_(hbt, non_blocking=True)
-            dcl.copy_(hcl, non_blocking=True)
+            dbuf.copy_(host, non_blocking=True)
             dec(dq, pool[0], pool[1], dbt, dcl, out=dout, **kw)
             hout.copy_(dout, non_blocking=True)
             torch.cuda.current_stream().synchronize()
@@ -307,28 +404,29 @@ def bench_ours(args, rank, world, dist):
             one()
         dt = (time.perf_counter() - t) / steps
         dt = max_over_ranks(dt, dist, device)
-        h2d = hq.nbytes + hbt.nbytes + hcl.nbytes
-        return {"s_per_step": dt, "h2d": h2d, "d2h": hout.nbytes}
+        return {"s_per_step": dt, "h2d": host.numel(), "d2h": hout.nbytes}
 
     primary = args.workload
-    if primary not in WORKLOAD_TEXT and not args.primary_only:
+    if primary not in (PRIMARY, SECONDARY) and not args.primary_only:
         raise SystemExit("--workload " + primary + " is timed alone: add --primary-only")
     secondary = SECONDARY if primary == PRIMARY else PRIMARY
-    prim = measure(primary, args.steps, args.warmup, with_e2e=True)
-    sec = measure(secondary, max(1, args.steps // 2), args.warmup, with_e2e=False) \
+    reps = max(3, args.reps)
+    prim = measure(primary, args.steps, args.warmup, reps, with_e2e=True)
+    sec = measure(secondary, args.steps, args.warmup, reps, with_e2e=False) \
         if not args.primary_only else None
-    # The parity-test configurations, timed the same way (reported, not the
-    # headline): tiny decode, sliding window, mixed batch over a q8_0 cache.
+    # The other configurations, timed the same way with the full step count
+    # (reported, not the headline).
     others = {}
     if not args.primary_only:
         for name in OTHER_CONFIGS:
-            r = measure(name, max(3, min(args.steps // 10, 200)), args.warmup, with_e2e=False)
-            others[name] = r
+            others[name] = measure(name, args.steps, args.warmup, reps, with_e2e=False)
+    probe = read_peak(device, torch, B) if not args.no_probe else None
 
     peak, peak_kind = measured_peaks()
     kv = prim["kv_bytes"]
     value = job_gbs(kv, world, prim["ms_per_step"] * 1e-3)
-    achieved = kv / (prim["ms_per_step"] * 1e-3) / 1e9  # per launch pair, timed region
+    achieved = kv / (prim["ms_per_step"] * 1e-3) / 1e9
+    rs = spread(prim["rep_us"])
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -338,34 +436,39 @@ def bench_ours(args, rank, world, dist):
         "warmup": args.warmup,
         "ms_per_step": round(prim["ms_per_step"], 5),
         "us_per_call": round(prim["ms_per_step"] * 1e3, 2),
-        "pct_of_8TBps": round(100 * kv / (prim["ms_per_step"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 1),
+        "pct_of_8TBps": round(100 * achieved / NOMINAL_HBM_GBS, 1),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded N(0,1) fp16 KV, random block permutation)",
         "impl": "ours",
-        "config": {
-            "workload": WORKLOAD_TEXT.get(primary) or CONFIG_TEXT[primary],
-            "kv_bytes_per_step": kv,
-            "num_splits": prim["splits"],
-            "l2": f"inputs larger than L2: {prim['copies']} KV pools of "
-                  f"{prim['pool_bytes'] / 1e6:.0f} MB rotated per step (L2 {l2_bytes / 1e6:.0f} MB)",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-        },
+        "config": config_dict(primary, world),
+        "setup": {"num_splits": prim["splits"],
+                  "l2": f"inputs larger than L2: {prim['copies']} KV pools of "
+                        f"{prim['pool_bytes'] / 1e6:.0f} MB rotated per step "
+                        f"({prim['copies'] * kv / 1e6:.0f} MB of visible KV; L2 {l2_bytes / 1e6:.0f} MB)"},
+        "repeats": {"n": reps, "us_per_call": [round(x, 2) for x in prim["rep_us"]],
+                    "median_us": round(rs["median"], 2), "min_us": round(rs["min"], 2),
+                    "spread_pct": round(rs["spread_pct"], 2),
+                    "drift_flag": rs["spread_pct"] > DRIFT_LIMIT_PCT,
+                    "what": f"{reps} timed regions of `steps` calls each; the first is the "
+                            f"reported value; drift_flag when (max - min) / median > {DRIFT_LIMIT_PCT}%"},
         "per_call_us": {"median": round(prim["us_median"], 2), "min": round(prim["us_min"], 2),
                         "p90": round(prim["us_p90"], 2),
                         "what": "events around single eager calls (includes launch gaps)"},
         "eager_us_per_call": round(prim["eager_us"], 2),
         "timing": f"CUDA graph of {prim['graph_calls']} calls replayed {args.steps // prim['graph_calls']}x "
-                  "inside the timed region; eager_us_per_call = the same calls launched one by one",
+                  "inside each timed region; eager_us_per_call = the same calls launched one by one",
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": recorded_traffic(primary),
+            "read_peak": probe,
+            "frac_of_read_peak": round(achieved / probe["value"], 4) if probe else None,
             "kernel": "one paged_attn_decode call: one launch of the split-KV decode kernel "
-                      "(cooperative when its grid fits on the device at once), whose CTAs "
-                      "also merge the split partials; time = timed region / steps",
+                      "(cooperative), whose CTAs also merge the split partials; "
+                      "time = timed region / steps",
         },
         "clocks": prim["clocks"],
         "gpu_launches": prim["launches"] * args.steps,
@@ -373,9 +476,12 @@ def bench_ours(args, rank, world, dist):
     e = prim["e2e"]
     line["e2e"] = {"value": round(job_gbs(kv, world, e["s_per_step"]), 1), "unit": "GB/s",
                    "us_per_call": round(e["s_per_step"] * 1e6, 2),
-                   "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+                   "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                   "what": "one pinned H2D copy of the packed q / block_table / context_lens, "
+                           "the C-ABI call, a pinned D2H copy of the output, synchronise"}
     if sec is not None:
         kv2 = sec["kv_bytes"]
+        rs2 = spread(sec["rep_us"])
         line["also"] = {
             "workload": WORKLOAD_TEXT[secondary],
             "us_per_call": round(sec["ms_per_step"] * 1e3, 2),
@@ -383,6 +489,9 @@ def bench_ours(args, rank, world, dist):
             "value": round(job_gbs(kv2, world, sec["ms_per_step"] * 1e-3), 1), "unit": "GB/s",
             "pct_of_8TBps": round(100 * kv2 / (sec["ms_per_step"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 1),
             "roofline_frac": round(kv2 / (sec["ms_per_step"] * 1e-3) / 1e9 / peak, 4),
+            "repeats_us": [round(x, 2) for x in sec["rep_us"]],
+            "spread_pct": round(rs2["spread_pct"], 2),
+            "drift_flag": rs2["spread_pct"] > DRIFT_LIMIT_PCT,
             "per_call_us": {"median": round(sec["us_median"], 2), "min": round(sec["us_min"], 2),
                             "p90": round(sec["us_p90"], 2)},
             "kv_bytes_per_step": kv2, "num_splits": sec["splits"],
@@ -393,14 +502,20 @@ def bench_ours(args, rank, world, dist):
         for name, r in others.items():
             kvb = r["kv_bytes"]
             gbs = kvb / (r["ms_per_step"] * 1e-3) / 1e9
+            rsn = spread(r["rep_us"])
             line["configs"][name] = {
-                "workload": CONFIG_TEXT[name], "kv_bytes_per_step": kvb,
+                "workload": WORKLOAD_TEXT[name], "kv_bytes_per_step": kvb,
                 "us_per_call": round(r["ms_per_step"] * 1e3, 2), "GB/s": round(gbs, 1),
+                "repeats_us": [round(x, 2) for x in r["rep_us"]],
+                "spread_pct": round(rsn["spread_pct"], 2),
+                "drift_flag": rsn["spread_pct"] > DRIFT_LIMIT_PCT,
                 "eager_us_per_call": round(r["eager_us"], 2),
                 "roofline_frac": round(gbs / peak, 4), "num_splits": r["splits"],
                 "launches_per_call": r["launches"],
                 "per_call_us": {"median": round(r["us_median"], 2), "min": round(r["us_min"], 2)},
-                "l2": f"{r['copies']} KV pool copies rotated",
+                "l2": f"{r['copies']} KV pool copies rotated "
+                      f"({r['copies'] * kvb / 1e6:.0f} MB of visible KV)",
+                "traffic": recorded_traffic(name),
             }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(prim["case"], budget_s=args.cpu_seconds)
@@ -410,50 +525,77 @@ def bench_ours(args, rank, world, dist):
 # ---------------------------------------------------------------------------
 # the fp64 oracle on the host cores (baseline, never the product path)
 # ---------------------------------------------------------------------------
-def cpu_baseline(case, budget_s=15.0):
+def oracle_sample(orc, case, rows, threads):
+    """Wall time of the oracle on the given query rows with `threads` threads."""
+    orc.set_num_threads(threads)
+    t = time.perf_counter()
+    orc.attend_rows(case, rows)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(case, budget_s=10.0):
     import oracle
     orc = oracle.load()
-    threads = orc.num_threads()
+    cores = os.cpu_count() or 1
     rows = np.random.default_rng(0).permutation(case.rows)
     done, t_total = 0, 0.0
-    batch = max(1, threads)
     while done < rows.size and t_total < budget_s:
-        ids = rows[done: done + batch]
-        t = time.perf_counter()
-        orc.attend_rows(case, ids)
-        t_total += time.perf_counter() - t
+        ids = rows[done: done + cores]
+        t_total += oracle_sample(orc, case, ids, cores)
         done += ids.size
     per_call = t_total / done * case.rows
+    # one thread, a smaller sample
+    n1 = max(1, min(4, case.rows))
+    t1 = oracle_sample(orc, case, rows[:n1], 1) / n1 * case.rows
+    orc.set_num_threads(cores)
     kv = gen.visible_kv_bytes(case)
     return {"value": round(kv / per_call / 1e9, 4), "unit": "GB/s",
-            "us_per_call": round(per_call * 1e6, 1), "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {case.rows} query rows of one call, "
-                      f"{t_total:.1f} s of fp64 C with OpenMP, extrapolated to the full call"}
+            "us_per_call": round(per_call * 1e6, 1), "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": f"{done} of {case.rows} query rows of one call, {t_total:.1f} s of fp64 C "
+                      f"with OpenMP on {cores} threads, scaled to the full call",
+            "single_thread": {"us_per_call": round(t1 * 1e6, 1),
+                              "value": round(kv / t1 / 1e9, 5), "unit": "GB/s",
+                              "sample": f"{n1} query rows on 1 thread, scaled to the full call"}}
 
 
 def bench_reference(args, rank, world):
-    """The oracle, as it stands, on this host's cores: each step is a bounded
-    sample of the workload's rows, timed and extrapolated to a full call."""
+    """The oracle, as it stands, on this host's cores.  Each step is one
+    bounded sample of the workload's query rows (the same sample every step),
+    timed in full: ms_per_step is that sample's time, and value the sample's
+    share of the algorithmic KV bytes over it."""
     if rank != 0:
         return None
-    case = gen.CONFIGS[PRIMARY](seed=0)
-    budget = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    import oracle
+    orc = oracle.load()
+    case = make_workload(PRIMARY, seed=0)
+    cores = os.cpu_count() or 1
+    orc.set_num_threads(cores)
+    n_rows = min(case.rows, max(cores, 32))
+    rows = np.random.default_rng(0).permutation(case.rows)[:n_rows]
     for _ in range(args.warmup):
-        cpu_baseline(case, budget_s=budget)
-    samples = [cpu_baseline(case, budget_s=budget) for _ in range(args.steps)]
-    us = statistics.median(s["us_per_call"] for s in samples)
-    kv = gen.visible_kv_bytes(case)
-    value = kv / (us * 1e-6) / 1e9
-    cb = dict(samples[-1])
-    cb["value"] = round(value, 4)
+        orc.attend_rows(case, rows)
+    ts = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        orc.attend_rows(case, rows)
+        ts.append(time.perf_counter() - t)
+    sec = statistics.mean(ts)
+    kv = gen.visible_kv_bytes(case) * n_rows / case.rows
+    value = kv / sec / 1e9
     return {
         "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
-        "us_per_call": round(us, 1), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD_TEXT[PRIMARY], "kv_bytes_per_step": kv,
-                   "parallelism": "host cores (OpenMP)"},
-        "cpu_baseline": cb,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+        "us_per_call": round(sec * 1e6 * case.rows / n_rows, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": config_dict(PRIMARY, world),
+        "setup": {"step": f"{n_rows} of {case.rows} query rows of one call per step "
+                          f"(the fp64 oracle, OpenMP on {cores} threads); us_per_call scales "
+                          "that to the full call"},
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "cpu_model": cpu_model(),
+                         "value": round(value, 4), "unit": "GB/s",
+                         "sample": f"{n_rows} query rows per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -462,11 +604,14 @@ def bench_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--split", choices=["replicas", "context"], default="replicas")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-probe", action="store_true")
     ap.add_argument("--primary-only", action="store_true")
     ap.add_argument("--workload", choices=[PRIMARY, SECONDARY, *OTHER_CONFIGS], default=PRIMARY,
                     help="workload of the headline line (the other of the two headline "
@@ -494,11 +639,15 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     try:
-        line = bench_ours(args, rank, world, dist)
+        if args.split == "context" and world > 1:
+            from paged_kv_decode_flash_b200 import context_parallel
+            line = context_parallel.bench(args, rank, world, dist)
+        else:
+            line = bench_ours(args, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
-    if rank == 0:
+    if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
 
 

@@ -17,7 +17,8 @@
  *     drafter uses a non-causal path;
  *   - sections "200k context for coding agents" and "Prefill: teach the
  *     fork's fast kernel to read the int8 cache": an int8 KV cache with
- *     scales is what makes a 200k-token context fit.
+ *     scales (vLLM's has one scale per row) is what makes a 200k-token
+ *     context fit; scale products and accumulators are fp32.
  *
  * For every sequence s, query token i < n_query and query head h the call
  * computes softmax(scale * q K^T) V over the keys j of sequence s that are
@@ -36,18 +37,24 @@
  * Layouts (all contiguous, row-major, device memory unless stated):
  *   q, out        fp16 [num_seqs][n_query][num_q_heads][head_dim]
  *   k/v cache     PA_KV_FP16: fp16 [num_blocks][num_kv_heads][block_size][head_dim]
- *                 PA_KV_Q8_0: bytes [num_blocks][num_kv_heads][tile] with one
- *                   tile = int8 qs[block_size][head_dim] followed by
+ *                 PA_KV_Q8_0: bytes [num_blocks][num_kv_heads][tile], one tile =
+ *                   int8 qs[block_size][head_dim] followed by
  *                   fp16 d[block_size][head_dim/32]; element value = qs * d of
  *                   its group of 32 consecutive head_dim elements; scales of
- *                   keys that a query can see must be finite with |d| < 1024
- *                   (true of any cache quantised from fp16 data, where
- *                   d = amax / 127 <= 516): larger ones give non-finite rows
+ *                   keys a query can see must be finite with |d| <= 512
+ *                   (true of any cache quantised from fp16 data whose
+ *                   magnitudes stay below 65024, d = amax / 127)
+ *                 PA_KV_INT8_ROW: bytes [num_blocks][num_kv_heads][tile], one
+ *                   tile = int8 qs[block_size][head_dim] followed by
+ *                   fp32 s[block_size]; element value = qs * s of its row;
+ *                   scales of visible keys must be finite with |s| <= 512
+ *                   (each value reaches the tensor core as two fp16 parts:
+ *                   relative error below 2^-21, absolute below 2^-25)
  *   block_table   int32 [num_seqs][max_blocks_per_seq]
  *   context_lens  int32 [num_seqs]
  * Supported: head_dim 128; block_size a multiple of 16 (the kernels work in
- * 16-key chunks; sizes 16 to 112 are exercised by the tests); n_query 1..8;
- * num_q_heads a multiple of num_kv_heads with
+ * 16-key chunks; sizes 16 to 112 are exercised by the tests); n_query
+ * 1..16; num_q_heads a multiple of num_kv_heads with
  * n_query * num_q_heads / num_kv_heads <= 64.
  *
  * Ownership and synchronisation: the caller owns every buffer, including the
@@ -61,11 +68,9 @@
  * that only the device can see (a block index outside [0, num_blocks), a
  * context length outside [n_query, max_blocks_per_seq * block_size]) do not
  * trap and never dereference the bad index: the rows of a sequence with a
- * bad length are written as 0; rows whose visible keys reach an out-of-range
- * block get finite values that are otherwise unspecified (the tensor-core
- * kernel writes the rows of that (sequence, KV head) as 0, the CUDA-core
- * kernel leaves the block's keys out); either way a flag is raised in the
- * workspace that paged_attn_get_error reports.
+ * bad length are written as 0, and so are the rows of a (sequence, KV head)
+ * whose visible keys reach an out-of-range block; either way a flag is
+ * raised in the workspace that paged_attn_get_error reports.
  */
 #ifndef PAGEDATTN_H
 #define PAGEDATTN_H
@@ -77,7 +82,7 @@
 extern "C" {
 #endif
 
-typedef enum { PA_KV_FP16 = 0, PA_KV_Q8_0 = 1 } pa_kv_dtype;
+typedef enum { PA_KV_FP16 = 0, PA_KV_Q8_0 = 1, PA_KV_INT8_ROW = 2 } pa_kv_dtype;
 
 typedef enum {
   PA_OK = 0,
@@ -103,30 +108,58 @@ typedef struct {
   size_t workspace_bytes;     /* >= paged_attn_workspace_size(dims, n_query) */
 } pa_dims;
 
-/* Bytes of workspace paged_attn_decode needs for these shapes: a 256-byte
- * status header, two int32 arrival counters per (sequence, KV head) and the
- * split partials.  Host only, no device access.  Returns 0 for invalid
- * shapes. */
+/* Bytes of workspace paged_attn_decode needs for these shapes, any cache
+ * type, any device: a 256-byte status header, arrival and queue counters
+ * and the split partials.  Host only, no device access.  Returns 0 for
+ * invalid shapes. */
 size_t paged_attn_workspace_size(const pa_dims* dims, int32_t n_query);
 
-/* Zero the workspace status header and arrival counters (enqueued on
- * `stream`).  Call once after allocating a workspace, before its first
+/* Zero the workspace status header and counters (enqueued on `stream`).
+ * Call once after allocating a workspace, before its first
  * paged_attn_decode; every decode call leaves the counters ready for the
- * next (their low 31 bits at zero). */
+ * next, a timed-out one included. */
 int paged_attn_workspace_init(const pa_dims* dims, void* stream);
 
 /* Decode attention (see the header comment for the exact definition).
  * q, k_cache, v_cache, block_table, context_lens, out: device pointers,
- * 16-byte aligned.  n_query in 1..8; causal 0 or 1; window >= 0 (0 = no
+ * 16-byte aligned.  n_query in 1..16; causal 0 or 1; window >= 0 (0 = no
  * window); scale multiplies q.k (usually 1/sqrt(head_dim)); kv_dtype a
- * pa_kv_dtype.  Enqueues the split-KV kernel and the merge of its partials
- * on `stream` (see paged_attn_launches_per_call).  Calls that share a
- * workspace must not overlap on the GPU (order them on one stream). */
+ * pa_kv_dtype.  Enqueues the split-KV kernel, whose CTAs also merge the
+ * split partials, on `stream` (see paged_attn_launches_per_call).  Calls
+ * that share a workspace must not overlap on the GPU (order them on one
+ * stream).  A sequence's result depends only on its own inputs, and
+ * repeated calls give bit-identical results. */
 int paged_attn_decode(const pa_dims* dims, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* block_table,
                       const int32_t* context_lens, int32_t n_query,
                       int32_t causal, int32_t window, float scale,
                       int32_t kv_dtype, void* out, void* stream);
+
+/* Partial decode of a share of each sequence's keys, for context-parallel
+ * decode across GPUs ("Dual MI50, part 2", section "Decode: a new kernel
+ * for the shape MTP actually runs": the work is split along the context
+ * and the partial results are merged at the end).  The same computation as
+ * paged_attn_decode, restricted for sequence s to the keys j in
+ * [key_begin[s], key_begin[s] + key_count[s]) (device int32 [num_seqs]);
+ * context_lens are the full lengths, so query positions and masks are the
+ * global ones.  key_begin[s] must be a multiple of block_size, the range
+ * must lie inside [0, L_s), and block_table row s maps the LOCAL block b
+ * (keys key_begin[s] + b * block_size ...) to a physical block of this
+ * call's cache pool.  Instead of fp16 rows it writes, per row,
+ *   out      fp32 [num_seqs][n_query][num_q_heads][head_dim]: the softmax-
+ *            weighted mean of V over the row's visible keys in the range
+ *   out_lse  fp32 [num_seqs][n_query][num_q_heads]: the natural log of
+ *            sum exp(scale q.k) over them
+ * (0 and -inf for a row that sees none of them).  paged_attn_merge over the
+ * ranks' (out, out_lse) gives the full-context result.  A range that is not
+ * whole blocks inside the context and the table is a data error
+ * (PA_ERR_BAD_CONTEXT_LEN from paged_attn_get_error). */
+int paged_attn_decode_partial(const pa_dims* dims, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* block_table,
+                              const int32_t* context_lens, const int32_t* key_begin,
+                              const int32_t* key_count, int32_t n_query, int32_t causal,
+                              int32_t window, float scale, int32_t kv_dtype, float* out,
+                              float* out_lse, void* stream);
 
 /* Log-sum-exp merge of split partials ("Dual MI50, part 2", section
  * "Decode: a new kernel for the shape MTP actually runs": partial results
@@ -148,25 +181,54 @@ int paged_attn_merge(const float* partial_out, const float* partial_lse,
  * flag of the workspace: PA_OK, PA_ERR_TIMEOUT, PA_ERR_BAD_BLOCK_INDEX or
  * PA_ERR_BAD_CONTEXT_LEN (the first of these that was raised, in that order),
  * or PA_ERR_CUDA if the stream reports an error.  PA_ERR_TIMEOUT means a
- * pipeline wait inside a kernel passed its time limit (about a second): the
- * kernel released its resources and returned, and its output is not valid. */
+ * pipeline wait inside a kernel passed its time limit: the kernel released
+ * its resources and returned and its output is not valid; the workspace
+ * stays usable (this call also clears its counters, as a safety net). */
 int paged_attn_get_error(const pa_dims* dims, void* stream);
 
-/* Debug: the key-resolution record of every row, computed on the device
- * with the same range, mask and block-table code the decode kernels use.
- * trace: device int32 [num_seqs][n_query][num_q_heads][5] =
- *   {visible key count, min j, max j, xor of physical slot ids,
- *    sum of physical slot ids mod 2^32}, physical slot id =
- *   block * block_size + slot; empty rows {0, -1, -1, 0, 0}.
- * Cost grows with the context (one thread walks each row): tests only. */
-int paged_attn_trace(const pa_dims* dims, const int32_t* block_table,
-                     const int32_t* context_lens, int32_t n_query,
-                     int32_t causal, int32_t window, int32_t* trace,
-                     void* stream);
+/* Sets the time after which a device-side pipeline wait gives up (raising
+ * PA_ERR_TIMEOUT) for calls enqueued afterwards by this process, and
+ * returns the previous value.  0 restores the default of one second.  A
+ * test aid: a limit the pipeline cannot meet makes the kernels exercise
+ * their give-up path without faulting or hanging the GPU. */
+uint64_t paged_attn_set_wait_limit(uint64_t nanoseconds);
 
-/* Number of key splits paged_attn_decode uses for these shapes and cache
- * type on the current device (host only; negative pa_status on error). */
-int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
+/* Debug: paged_attn_decode (same arguments and output) that also records,
+ * for every output row, which keys the decode kernel scored and where it
+ * read them: trace is device int32 [num_seqs][n_query][num_q_heads][5] =
+ *   {visible key count, min j, max j, xor of physical slot ids,
+ *    sum of physical slot ids mod 2^32},
+ * physical slot id = block * block_size + slot of the K row the kernel
+ * copied; rows without keys get {0, -1, -1, 0, 0}.  Slower (atomics per
+ * scored pair): tests only. */
+int paged_attn_trace(const pa_dims* dims, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_table,
+                     const int32_t* context_lens, int32_t n_query, int32_t causal,
+                     int32_t window, float scale, int32_t kv_dtype, void* out,
+                     int32_t* trace, void* stream);
+
+/* Writes the keys and values of the n_new newest tokens of every sequence
+ * into the paged cache: token i < n_new of sequence s sits at position
+ * L_s - n_new + i (L_s = context_lens[s], which includes them), in slot
+ * position % block_size of block block_table[s][position / block_size].
+ *   k_new, v_new  fp16 [num_seqs][n_new][num_kv_heads][head_dim] (device)
+ *   k/v cache     the layouts above (device, written)
+ * The int8 caches are quantised on the way, in fp32 with IEEE rounding:
+ *   PA_KV_Q8_0, per 32 elements: d = fp16(amax / 127),
+ *     q = d > 0 ? clamp(round_half_away(x / d), -127, 127) : 0;
+ *   PA_KV_INT8_ROW, per row: s = amax / 127, q as above with s.
+ * Uses the status word of dims->workspace (>= 256 bytes) for data errors (a
+ * block index or context length out of range: that row is not written),
+ * which paged_attn_get_error reports.  n_new in 1..16. */
+int paged_attn_cache_write(const pa_dims* dims, const void* k_new, const void* v_new,
+                           const int32_t* block_table, const int32_t* context_lens,
+                           int32_t n_new, int32_t kv_dtype, void* k_cache, void* v_cache,
+                           void* stream);
+
+/* The most split partials one (sequence, KV head, row part) of a call with
+ * these shapes and cache type is merged from on the current device (host
+ * only; negative pa_status on error). */
+int paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
 
 /* Allocation-free variant of paged_attn_decode.  The paper has no
  * counterpart: it exists for callers that cannot give the library device
@@ -174,16 +236,19 @@ int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_d
  * (a serving engine with one fixed pool planned at start-up, a plug-in host
  * without an allocator) or hot paths that must not call cudaMalloc, which can
  * implicitly synchronise the device.  Same arguments, layouts and results as
- * paged_attn_decode; the workspace fields of *dims are ignored.  The split
- * partials live in one array of PA_NOALLOC_SCRATCH_BYTES inside the
- * library's device image, held by every GPU that loads the library until
- * exit; shapes that need more return PA_ERR_WORKSPACE before anything is
- * enqueued.  All calls on a device share that array: calls whose work
- * overlaps on the GPU race and corrupt each other, so order them (one
+ * paged_attn_decode (bit-identical); the workspace fields of *dims are
+ * ignored.  The split partials live in one array of PA_NOALLOC_SCRATCH_BYTES
+ * inside the library's device image, held by every GPU that loads the
+ * library until exit; shapes that need more return PA_ERR_WORKSPACE before
+ * anything is enqueued.  All calls on a device share that array: calls whose
+ * work overlaps on the GPU race and corrupt each other, so order them (one
  * stream, or events).  The first call on a device looks up the array's
- * device address and caches it; make it before any stream capture begins.
- * Device-side data errors are handled as in paged_attn_decode (masked keys,
- * zeroed rows) but are not reported: the status word is cleared per call. */
+ * device address and caches it (safe from several host threads); make it
+ * before any stream capture begins.  The array's counters and status word
+ * are cleared at the start of every call, so device-side data errors are
+ * handled as in paged_attn_decode (masked keys, zeroed rows) but are not
+ * reported, and neither is a timeout of a device-side wait: such a call
+ * leaves its output undefined and cannot be detected. */
 #define PA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_cache,
                               const void* v_cache, const int32_t* block_table,
@@ -191,12 +256,20 @@ int paged_attn_decode_noalloc(const pa_dims* dims, const void* q, const void* k_
                               int32_t causal, int32_t window, float scale,
                               int32_t kv_dtype, void* out, void* stream);
 
+/* Measurement aid, not part of the attention: streams `bytes` (rounded
+ * down to 32 KB) of device memory at `src` (16-byte aligned) into shared
+ * memory the way the decode kernel moves KV tiles (4 KB bulk copies into a
+ * ring of 32 KB slots, completion on mbarriers, six slots in flight) on
+ * `ctas` CTAs, and writes one word per CTA to sink (device uint32
+ * [ctas]; 0xdeadbeef from a CTA whose wait timed out).  Timing it gives the
+ * read-only HBM ceiling of that access pattern. */
+int paged_attn_stream_read(const void* src, size_t bytes, uint32_t* sink, int32_t ctas,
+                           void* stream);
+
 /* Kernel launches one paged_attn_decode call makes for these shapes and
- * cache type on the current device: 1 where the tensor-core kernel runs (its
- * CTAs also merge the split partials of each (sequence, KV head)), 2 for
- * the CUDA-core kernel followed by the merge kernel (launched as a
- * programmatic dependent so that it starts as soon as the split-KV kernel
- * ends).  Host only; negative pa_status on error. */
+ * cache type on the current device: 1, or, for a batch large enough to use
+ * the work queue, one per 256 sequences.  Host only; negative pa_status on
+ * error. */
 int32_t paged_attn_launches_per_call(const pa_dims* dims, int32_t n_query, int32_t kv_dtype);
 
 /* Static string for a pa_status. */

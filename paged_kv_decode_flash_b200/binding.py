@@ -28,6 +28,7 @@ PA_ERR_TIMEOUT = -7
 
 KV_FP16 = _inputs.KV_FP16
 KV_Q8_0 = _inputs.KV_Q8_0
+KV_INT8_ROW = _inputs.KV_INT8_ROW
 
 
 class PagedAttnError(RuntimeError):
@@ -72,8 +73,15 @@ def lib() -> ctypes.CDLL:
             L.paged_attn_merge.restype = ctypes.c_int
             L.paged_attn_get_error.argtypes = [P, vp]
             L.paged_attn_get_error.restype = ctypes.c_int
-            L.paged_attn_trace.argtypes = [P, vp, vp, i32, i32, i32, vp, vp]
+            L.paged_attn_trace.argtypes = [P, vp, vp, vp, vp, vp, i32, i32, i32, f32, i32, vp, vp, vp]
             L.paged_attn_trace.restype = ctypes.c_int
+            L.paged_attn_decode_partial.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                                    f32, i32, vp, vp, vp]
+            L.paged_attn_decode_partial.restype = ctypes.c_int
+            L.paged_attn_set_wait_limit.argtypes = [ctypes.c_uint64]
+            L.paged_attn_set_wait_limit.restype = ctypes.c_uint64
+            L.paged_attn_cache_write.argtypes = [P, vp, vp, vp, vp, i32, i32, vp, vp, vp]
+            L.paged_attn_cache_write.restype = ctypes.c_int
             L.paged_attn_num_splits.argtypes = [P, i32, i32]
             L.paged_attn_num_splits.restype = ctypes.c_int32
             L.paged_attn_launches_per_call.argtypes = [P, i32, i32]
@@ -123,11 +131,23 @@ def _expect(t: torch.Tensor, name: str, dtype, shape) -> None:
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def cache_block_size(k_cache: torch.Tensor, kv_dtype: int, head_dim: int) -> int:
-    if kv_dtype == KV_FP16:
-        return int(k_cache.shape[2])
-    per_slot = head_dim + 2 * (head_dim // 32)
-    return int(k_cache.shape[2]) // per_slot
+def set_wait_limit(nanoseconds: int) -> int:
+    """Time after which device-side pipeline waits give up (PA_ERR_TIMEOUT)
+    for later calls of this process; 0 restores the default (1 s).  Returns
+    the previous value."""
+    return int(lib().paged_attn_set_wait_limit(int(nanoseconds)))
+
+
+def cache_shape(kv_dtype: int, num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int):
+    """(torch dtype, shape) of one cache tensor (include/pagedattn.h layouts)."""
+    if int(kv_dtype) == KV_FP16:
+        return torch.float16, (num_blocks, num_kv_heads, block_size, head_dim)
+    if int(kv_dtype) == KV_Q8_0:
+        return torch.uint8, (num_blocks, num_kv_heads, block_size * (head_dim + 2 * (head_dim // 32)))
+    if int(kv_dtype) == KV_INT8_ROW:
+        return torch.uint8, (num_blocks, num_kv_heads, block_size * (head_dim + 4))
+    raise ValueError(f"kv_dtype {kv_dtype}: expected {KV_FP16} (fp16), {KV_Q8_0} (q8_0) "
+                     f"or {KV_INT8_ROW} (int8 rows)")
 
 
 class PagedDecode:
@@ -187,12 +207,7 @@ class PagedDecode:
             _expect(out, "out", torch.float16, (B, nq, Hq, D))
         _expect(block_table, "block_table", torch.int32, (B, d.max_blocks_per_seq))
         _expect(context_lens, "context_lens", torch.int32, (B,))
-        if int(kv_dtype) == KV_FP16:
-            cache = (torch.float16, (d.num_blocks, Hkv, d.block_size, D))
-        elif int(kv_dtype) == KV_Q8_0:
-            cache = (torch.uint8, (d.num_blocks, Hkv, d.block_size * (D + 2 * (D // 32))))
-        else:
-            raise ValueError(f"kv_dtype {kv_dtype}: expected {KV_FP16} (fp16) or {KV_Q8_0} (q8_0)")
+        cache = cache_shape(kv_dtype, d.num_blocks, Hkv, d.block_size, D)
         _expect(k_cache, "k_cache", *cache)
         _expect(v_cache, "v_cache", *cache)
         dev = self.workspace.device
@@ -214,20 +229,71 @@ class PagedDecode:
         _check(rc, "paged_attn_decode")
         return out
 
+    def partial(self, q, k_cache, v_cache, block_table, context_lens, key_begin, key_count, *,
+                causal: int, window: int, scale: float, kv_dtype: int, out=None, out_lse=None,
+                stream=None):
+        """paged_attn_decode_partial: this call's share of each sequence's
+        keys, [key_begin, key_begin + key_count), with block_table mapping
+        local blocks.  Returns (out fp32 [B][nq][Hq][D], out_lse fp32
+        [B][nq][Hq])."""
+        self.check_args(q, k_cache, v_cache, block_table, context_lens, kv_dtype, None)
+        B = self.dims.num_seqs
+        _expect(key_begin, "key_begin", torch.int32, (B,))
+        _expect(key_count, "key_count", torch.int32, (B,))
+        shp = tuple(q.shape)
+        if out is None:
+            out = torch.empty(shp, dtype=torch.float32, device=q.device)
+        if out_lse is None:
+            out_lse = torch.empty(shp[:-1], dtype=torch.float32, device=q.device)
+        _expect(out, "out", torch.float32, shp)
+        _expect(out_lse, "out_lse", torch.float32, shp[:-1])
+        rc = lib().paged_attn_decode_partial(
+            ctypes.byref(self.dims), _dptr(q), _dptr(k_cache), _dptr(v_cache),
+            _dptr(block_table), _dptr(context_lens), _dptr(key_begin), _dptr(key_count),
+            self.n_query, int(causal), int(window), float(scale), int(kv_dtype), _dptr(out),
+            _dptr(out_lse), _stream_ptr(stream))
+        _check(rc, "paged_attn_decode_partial")
+        return out, out_lse
+
     def get_error(self, stream=None) -> int:
         """Synchronises and returns (and clears) the device data-error status."""
         return lib().paged_attn_get_error(ctypes.byref(self.dims), _stream_ptr(stream))
 
-    def trace(self, block_table, context_lens, *, causal: int, window: int, stream=None):
+    def trace(self, q, k_cache, v_cache, block_table, context_lens, *, causal: int,
+              window: int, scale: float, kv_dtype: int, out=None, stream=None):
+        """paged_attn_trace: the decode plus the key-resolution record of the
+        kernel that read the cache.  Returns (out, trace int32 [B][nq][Hq][5])."""
+        self.check_args(q, k_cache, v_cache, block_table, context_lens, kv_dtype, out)
+        if out is None:
+            out = torch.empty_like(q)
         B, nq, Hq = self.dims.num_seqs, self.n_query, self.dims.num_q_heads
-        _expect(block_table, "block_table", torch.int32, (B, self.dims.max_blocks_per_seq))
-        _expect(context_lens, "context_lens", torch.int32, (B,))
-        t = torch.empty((B, nq, Hq, 5), dtype=torch.int32, device=block_table.device)
-        rc = lib().paged_attn_trace(ctypes.byref(self.dims), _dptr(block_table),
-                                    _dptr(context_lens), nq, int(causal), int(window),
-                                    _dptr(t), _stream_ptr(stream))
+        t = torch.empty((B, nq, Hq, 5), dtype=torch.int32, device=q.device)
+        rc = lib().paged_attn_trace(
+            ctypes.byref(self.dims), _dptr(q), _dptr(k_cache), _dptr(v_cache),
+            _dptr(block_table), _dptr(context_lens), nq, int(causal), int(window),
+            float(scale), int(kv_dtype), _dptr(out), _dptr(t), _stream_ptr(stream))
         _check(rc, "paged_attn_trace")
-        return t
+        return out, t
+
+    def cache_write(self, k_new, v_new, block_table, context_lens, *, kv_dtype: int, k_cache,
+                    v_cache, stream=None):
+        """paged_attn_cache_write: the n_query newest tokens' K/V (fp16
+        [B][n_query][Hkv][D]) into the paged cache, quantised for the int8
+        caches.  Data errors go to this decoder's workspace (get_error)."""
+        d = self.dims
+        shp = (d.num_seqs, self.n_query, d.num_kv_heads, d.head_dim)
+        _expect(k_new, "k_new", torch.float16, shp)
+        _expect(v_new, "v_new", torch.float16, shp)
+        _expect(block_table, "block_table", torch.int32, (d.num_seqs, d.max_blocks_per_seq))
+        _expect(context_lens, "context_lens", torch.int32, (d.num_seqs,))
+        cache = cache_shape(kv_dtype, d.num_blocks, d.num_kv_heads, d.block_size, d.head_dim)
+        _expect(k_cache, "k_cache", *cache)
+        _expect(v_cache, "v_cache", *cache)
+        rc = lib().paged_attn_cache_write(
+            ctypes.byref(d), _dptr(k_new), _dptr(v_new), _dptr(block_table),
+            _dptr(context_lens), self.n_query, int(kv_dtype), _dptr(k_cache), _dptr(v_cache),
+            _stream_ptr(stream))
+        _check(rc, "paged_attn_cache_write")
 
 
 def merge(partial_out: torch.Tensor, partial_lse: torch.Tensor, out=None, out_lse=None,

@@ -1,5 +1,5 @@
 // decode_tc.cu -- split-KV paged decode attention on the sm_100a tensor
-// cores (tcgen05 + TMEM), with TMA staging of the paged KV tiles.
+// cores (tcgen05 + TMEM), with TMA / bulk-copy staging of the paged KV tiles.
 //
 // What it computes is the decode step of "Dual MI50, part 2: from 10 to 74
 // tokens/s, a 200k-token context, and two attention kernels" (sbm-labs
@@ -7,73 +7,59 @@
 // query rows that share one KV head (n_query tokens x the query heads of the
 // group) are scored against the same keys, the context is split so that
 // every SM is busy at batch 1, and one fp32 partial (O, lse) per split is
-// left for the log-sum-exp merge.  Masks and block-table resolution follow
-// section "Bug 2: the drafter read freed memory".
+// merged by log-sum-exp weights.  Masks and block-table resolution follow
+// section "Bug 2: the drafter read freed memory"; the int8 caches follow
+// sections "200k context for coding agents" and "Prefill: teach the fork's
+// fast kernel to read the int8 cache" (per-row scales, fp32 scale products).
 //
-// Hardware mapping (one CTA per SM, 11 warps; 19 for the q8_0 cache):
-//   warps 0, 10 TMA producers for K and for V: resolve the block table and
-//               load whole 16-key chunks into separate rings of 128-key tiles
-//               (fp16: 4-D boxes of two 64-column halves with the 128-byte
-//               swizzle, 2-3 slots; q8_0: untiled bulk copies of the raw
-//               chunk into the upper half of a slot, 2 K and 3 V slots).  K
-//               slots are released as soon as QK^T has read them, so K runs
-//               ahead.  With each K copy the same chunk of V is prefetched
-//               into L2, so that V's own copy a tile later is short.
-//   warp 1      MMA issuer (one thread), fixed order QK(0), QK(1), then
-//               PV(t), QK(t+2): S^T = K Q^T with M = 128 keys and N = the
-//               query rows (double-buffered in TMEM), O^T += V^T
-//               [P_hi | P_lo]^T with M = 128 head_dim lanes (one TMEM
-//               accumulator over all tiles); P is double-buffered in shared
-//               memory (fp16) so that the softmax of tile t+1 overlaps PV(t).
-//   warps 2-9   two softmax warpgroups, each owning half of the query rows:
-//               thread = key for S (row max by a warp transpose-reduction
-//               plus one named barrier per group); when a row's reference
-//               maximum rises, its O column is rescaled in TMEM in place
-//               (thread = head_dim lane) before the tile's P is published.
-//   warps 11-18 (q8_0 cache only) converters, four for K and four for V:
-//               each raw int8 tile is expanded in place into its exact fp16
-//               operand tile (see below).
-// Putting keys and head_dim on the MMA's M side keeps the tensor core free of
-// padding even at 4-32 query rows.
+// Work: a CTA streams *segments* -- runs of 16-key chunks of one group (a
+// sequence, a KV head and a part of its query rows) -- through one
+// pipeline, 128-key tiles at a time, and writes one partial per segment
+// (DecodeParams in common.cuh describes the two ways the work is cut).
 //
-// Exactness: Q, K and V are fed to the tensor core as the exact fp16 inputs.
-// The softmax weights are scaled by 2^14 (2^13 for q8_0, so that weights
-// down to ~4e-12 of the row maximum stay representable) and split into an fp16 high part and
-// an fp16 residual; both are multiplied with V and accumulated in fp32, which
-// keeps the weights to about 2^-22 relative.  Keys no query row can see are
-// never multiplied: their chunks are not loaded when wholly outside the
-// visible range, their scores are selected to -inf, and their V rows are
-// zero-filled in shared memory before the PV product (the NaN-poisoned
-// out-of-window blocks of the pages' regression test must not leak).
+// Roles (one CTA per SM; 11 warps for fp16, 19 for the int8 caches):
+//   warp 0      K producer: takes the CTA's segments (a static range, or
+//               items from a queue), resolves the block table one tile
+//               ahead, bounds-checks every block, publishes each tile's
+//               description and copies its 16-key chunks into the K ring
+//               (fp16: 4-D TMA boxes in the 128-byte-swizzled operand
+//               layout; int8: untiled bulk copies of the raw chunk into the
+//               upper half of a slot); it also stages each segment's Q rows.
+//   warp 1      MMA issuer (one thread): QK(0), QK(1), then PV(t), QK(t+2):
+//               S^T = K Q^T (M = 128 keys, N = query rows) double-buffered
+//               in TMEM, O^T += V^T [P_hi | P_lo]^T (M = 128 head_dim lanes)
+//               into one of two O accumulators (a segment's O stays put
+//               while the next segment's accumulates).
+//   warps 2..   softmax warpgroups (rows split between two): thread = key
+//               for S; lazy per-row reference maximum in the log2 domain;
+//               O rescaled in TMEM when it rises; P split into an fp16 high
+//               part and residual; at a segment's last tile the partial
+//               (O / l, lse) is written.
+//   next warp   V producer: follows the published tiles.
+//   last 8      (int8 caches) converters, four for K and four for V.
 //
-// q8_0 cache (int8 qs with one fp16 scale d per 32 head_dim elements): the
-// scale stays out of the operands, so that they remain exact without a
-// high/residual split.  K's operand is qs; S^T gets one TMEM accumulator per
-// scale group, and the softmax forms each score as the sum over the groups of
-// K's scale times the group's partial product, in fp32.  V's operand is
-// qs * 2^e, with d = m * 2^e split into its power of two and its mantissa m;
-// P gets one copy per scale group with the weights multiplied by that
-// group's m (then split into fp16 parts as above), and each group has its
-// own O^T accumulator, of which a head_dim lane reads only its own group's.
-// The softmax reads the scales of its keys from the cache (L2) a tile ahead.
-// Batches with many (sequence, KV head) groups cut every group's tiles into
-// fixed-size items, one CTA each, over several waves; the size depends on
-// the shapes only, so a sequence's output does not depend on the others.
+// Exactness: Q, K and V reach the tensor core as exact fp16 values.  Softmax
+// weights are scaled by 2^14 and split into two fp16 parts (error ~2^-22).
+// Both int8 caches: K's operand is qs itself (q8_0: S^T gets one accumulator
+// per 32-element scale group and the softmax adds the groups times K's fp16
+// scales in fp32; int8 rows: the score is multiplied by K's fp32 row scale).
+// V's operand is the pair V_hi = fp16(qs * d), V_lo = fp16(qs * d - V_hi),
+// multiplied as V_hi [P_hi | P_lo] + V_lo P_hi: exact for q8_0 (qs * d has
+// at most 19 significant bits), within 2^-22 for an fp32 row scale.  Keys
+// that no row of a part can see are never multiplied: wholly invisible
+// chunks are not loaded, their scores are selected to -inf and their V rows
+// are written as zeros before PV (NaN-poisoned memory cannot leak).
 //
-// Merge: every CTA writes its fp32 partial (O, lse).  With a cooperative
-// launch (every CTA resident) the CTAs of one (sequence, KV head) meet at a
-// bounded counter barrier and each merges a slice of the group's rows;
-// otherwise the last CTA of the group to arrive merges all of it.  Splits
-// are added in a fixed order (log-sum-exp weights), so results are
-// bit-reproducible.  A call is one launch.
-//
-// Every wait is bounded (sm100::mbar_wait and the group barrier): on a
-// timeout the kernel raises kFlagTimeout, drains its own copies and MMAs,
-// frees TMEM and still takes part in the merge (its rows count as empty).
+// Every wait is bounded (DecodeParams::wait_limit_ns): on a timeout the
+// kernel raises kFlagTimeout, stops issuing work, drains its own copies and
+// MMAs with a fixed one-second bound, frees TMEM, and keeps the workspace
+// counters consistent for the next call (every segment it owns is counted
+// in, with an invalid partial).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstring>
 
@@ -86,134 +72,148 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTileKeys = 128;                 // keys per pipeline tile (M of S^T)
-constexpr int kChunksPerTile = kTileKeys / kChunk;
-constexpr int kMaxStages = 3;                  // slots per K ring and per V ring (at most)
+constexpr int kMaxStages = 3;
 // A K or V tile of 128 keys in shared memory: [key group of 8][half][8 keys]
-// [64 fp16] with the 128-byte swizzle, i.e. 1 KB swizzle atoms; the atoms of
-// one 64-column half sit 2 KB apart, the two halves of a key group 1 KB apart.
-// One 16-key chunk (a contiguous 4 KB (block, head) tile in the cache for
-// block_size 16) is a single TMA box.
-constexpr uint32_t kAtomBytes = 1024;              // 8 keys x 128 bytes
-constexpr uint32_t kGroupBytes = 2 * kAtomBytes;   // both halves of 8 keys
-constexpr uint32_t kKVBytes = kTileKeys / 8 * kGroupBytes;  // one K (or V) tile
-constexpr uint32_t kChunkBytes = kChunk * 256;     // one 16-key chunk (TMA box)
-// q8_0: a raw 128-key tile in shared memory is qs [128 keys][128 int8] then
-// d [128 keys][4 fp16]; a 16-key chunk arrives as two bulk copies (2048 B of
-// qs, 128 B of scales).
-constexpr uint32_t kRawOff = kKVBytes / 2;          // q8_0: raw qs in the slot's upper half
-constexpr uint32_t kQ8QsChunk = kChunk * kHeadDim;    // 2048 B of qs per 16-key chunk
-constexpr uint32_t kQ8DChunk = kChunk * 8;            // 128 B of scales per 16-key chunk
-constexpr int kSoftmaxThreads = 128;           // per softmax warpgroup
-constexpr uint32_t kBarSetup = 1;              // named barrier: set-up done
-constexpr uint32_t kBarGroup0 = 2;             // named barriers 2, 3: softmax groups
-constexpr uint32_t kBarConv0 = 4;              // named barriers 4, 5: q8_0 K / V converters
-// A row's reference max is only raised when a score passes it by more than
-// kLazy (log2 units); weights scaled by 2^kPShift (see Cfg) then stay below
-// 2^(kPShift + kLazy), inside fp16 range.
+// [64 fp16] with the 128-byte swizzle (1 KB atoms; the two 64-column halves
+// of a key group 1 KB apart, key groups 2 KB apart).  One 16-key chunk is a
+// single TMA box of 4 KB.
+constexpr uint32_t kAtomBytes = 1024;
+constexpr uint32_t kGroupBytes = 2 * kAtomBytes;
+constexpr uint32_t kKVBytes = kTileKeys / 8 * kGroupBytes;  // 32 KB
+constexpr uint32_t kChunkBytes = kChunk * 256;
+constexpr uint32_t kRawOff = kKVBytes / 2;       // in-place K slots: raw int8 in the upper half
+constexpr uint32_t kQsChunk = kChunk * kHeadDim; // 2 KB of int8 per 16-key chunk
+constexpr uint32_t kRawScales = kQsChunk * kChunksPerTile;  // raw V slot: scales after the qs
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kBarSetup = 1;   // named barrier: set-up done
+constexpr uint32_t kBarGroup0 = 2;  // named barriers 2, 3: softmax warpgroups
+constexpr uint32_t kBarConv0 = 4;   // named barriers 4, 5: K / V converters
+// A row's reference maximum is raised only when a score passes it by more
+// than kLazy (log2 units); weights scaled by 2^kPShift then stay below
+// 2^(kPShift + kLazy), inside the fp16 range.
 constexpr float kLazy = 1.5f;
+constexpr int kPShift = 14;
+constexpr int kInfoSlots = 8;
+constexpr int kSegSlots = 8;
+constexpr int kMergeListLen = 64;
+constexpr unsigned kInvalidLse = 0x7fc00000u;  // NaN: a partial that must not be used
 
 enum : int {
-  BAR_KFULL = 0,    // [3] K tile landed
-  BAR_KEMPTY = 3,   // [3] K tile read by QK^T
-  BAR_VFULL = 6,    // [3] V tile landed
-  BAR_VEMPTY = 9,   // [3] V tile read by PV
-  BAR_SFULL = 12,   // [2] S^T in TMEM
-  BAR_SEMPTY = 14,  // [2] S^T read by the softmax warps
-  BAR_PFULL = 16,   // [2] P of one tile written to shared memory
-  BAR_OFULL = 18,   // PV of one more tile accumulated into O^T
-  BAR_DONE = 22,    // every MMA finished
-  BAR_INFO = 23,    // [8] a tile's number, chunk mask and cache rows published
-  BAR_CKFULL = 31,  // [3] q8_0: K slot converted to fp16
-  BAR_CVFULL = 34,  // [3] q8_0: V slot converted to fp16
-  BAR_COUNT = 37
+  BAR_KFULL = 0,     // [3] K chunks landed (int8: raw)
+  BAR_KEMPTY = 3,    // [3] K slot read by QK^T
+  BAR_VFULL = 6,     // [3] V chunks landed (int8: in a raw slot)
+  BAR_VEMPTY = 9,    // [3] V slot free again
+  BAR_CKFULL = 12,   // [3] int8: K slot converted
+  BAR_CVFULL = 15,   // int8: converted V (hi | lo) ready
+  BAR_CVEMPTY = 16,  // int8: converted V read by PV
+  BAR_SFULL = 17,    // [2] S^T in TMEM
+  BAR_SEMPTY = 19,   // [2] S^T read by the softmax
+  BAR_PFULL = 21,    // [2] P of a tile in shared memory
+  BAR_OFULL = 23,    // PV of one more tile accumulated
+  BAR_OEMPTY = 24,   // [2] a segment's O accumulator read out
+  BAR_QFULL = 26,    // [2] a segment's Q staged
+  BAR_QEMPTY = 28,   // [2] Q buffer free
+  BAR_DONE = 30,     // every MMA finished
+  BAR_INFO = 31,     // [8] a tile's description published
+  BAR_COUNT = 39
 };
 constexpr int kBarSlots = 40;
-constexpr int kInfoSlots = 8;  // depth of the tile-information ring
 
-// NG softmax warpgroups of RW query rows each; NR = the MMA's N for S
-// (>= 16).  Warps: 0 K producer, 1 MMA issuer, 2 .. 4*NG+1 softmax, then the
-// V producer (and, q8_0 only, four converter warps).
-// KS / VS slots in the K / V rings, PB buffers for P.  fp16: two P buffers,
-// so that the softmax of tile t+1 never waits for PV(t); at 32 rows they take
-// 32 KB and the V ring keeps two slots (measured: three V slots with one P
-// buffer is slower).  q8_0: a slot is the fp16 operand tile; the raw int8
-// tile lands in its upper half and the converters expand it in place (a V
-// slot also keeps the raw scales after the tile); two K slots, three V
-// slots, one P buffer that holds a P per scale group (the softmax of tile t
-// waits for PV(t-1) before it stores P(t)).
-template <int RW, int NG, bool Q8>
-struct Cfg {
-  static constexpr int kGroups = NG;
-  static constexpr int kVWarp = 2 + NG * 4;      // the V producer's warp
-  static constexpr int kConvWarp = kVWarp + 1;   // q8_0: first converter warp
-  static constexpr int kConvWarps = 4;           // q8_0: converter warps per stream (K, V)
-  static constexpr int kThreads = 32 * (kVWarp + 1 + (Q8 ? 2 * kConvWarps : 0));
-  static constexpr int NR = (kGroups * RW < 16) ? 16 : kGroups * RW;
-  // q8_0: one S^T accumulator, one P and one O^T accumulator per group of 32
-  // head_dim elements that shares a scale; fp16: one of each.
-  static constexpr int kSG = Q8 ? kHeadDim / 32 : 1;
-  static constexpr int KS = Q8 ? 2 : 3;
-  static constexpr int VS = Q8 ? 3 : (NR > 16 ? 2 : 3);
-  static constexpr int PB = Q8 ? 1 : 2;  // q8_0 measured: two V slots and two P buffers are slower
-  // Weights are scaled by 2^kPShift before they are split into fp16 parts.
-  // q8_0 multiplies them by a scale mantissa in [1, 2) as well, so it keeps
-  // one bit of headroom more.
-  static constexpr int kPShift = Q8 ? 13 : 14;
-  static constexpr uint32_t kKSlot = kKVBytes;                           // K slot
-  static constexpr uint32_t kVSlot = kKVBytes + (Q8 ? kTileKeys * 8 : 0);  // V slot (+ scales)
-  static constexpr uint32_t kK = 0;                                      // K ring
-  static constexpr uint32_t kV = KS * kKSlot;                            // V ring
-  static constexpr uint32_t kQ = kV + VS * kVSlot;
-  static constexpr uint32_t kQHalf = NR * 128;
-  // P^T of one tile: per scale group 2*NR "rows" (the fp16 high parts of the
-  // NR query rows, then their residuals), the groups side by side, so that
-  // one MMA with N = kSG * 2 * NR multiplies all of them with each V step
-  // (V is read once).  Tile t uses buffer t % PB.
-  static constexpr int kPN = kSG * 2 * NR;  // N of the PV product
-  static constexpr uint32_t kP = kQ + 2 * kQHalf;
-  static constexpr uint32_t kPBytes = kTileKeys * kPN * 2;
-  static constexpr uint32_t kRed = kP + PB * kPBytes;               // float [2 grp][2][4][32]
-  static constexpr uint32_t kAlpha = kRed + kGroups * 2 * 4 * 32 * 4;  // float [4 tiles][32 rows]
-  static constexpr uint32_t kLsum = kAlpha + 4 * 32 * 4;            // float [2 grp][4][32]
-  static constexpr uint32_t kBcast = kLsum + kGroups * 4 * 32 * 4;  // float [4*NG warps][2][32]
-  static constexpr uint32_t kBars = kBcast + kGroups * 4 * 2 * 32 * 4;  // uint64 [kBarSlots]
-  static constexpr uint32_t kInfo = kBars + kBarSlots * 8;          // TileInfo [8]
-  static constexpr uint32_t kMisc = kInfo + kInfoSlots * 48;        // small ints
-  static constexpr uint32_t kTotal = kMisc + 64;
-  // TMEM columns: S^T[2] (kSG accumulators of NR columns each), then O^T
-  // from column kTmemS (kSG accumulators of 2*NR: high | residual).
-  static constexpr uint32_t kTmemS = 2 * kSG * NR;
-  static constexpr uint32_t kTmemUsed = kTmemS + kSG * 2 * NR;
-  static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
-                                        : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
-  static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
-  static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
-  static_assert(kV % 1024 == 0 && kVSlot % 1024 == 0, "tiles sit on 1 KB swizzle atoms");
-  static_assert(kTmemUsed <= 512, "TMEM columns");
+// A tile as the K producer publishes it.
+struct TileInfo {
+  int seg;       // segment number within this CTA (-1: end of the stream)
+  int flags;     // 1: first tile of its segment, 2: last tile
+  int key0;      // key of the tile's first chunk
+  int vis_lo;    // keys of the segment that some row of its part can see
+  int vis_hi;
+  uint32_t mask; // 16-key chunks copied
+  int row8[kChunksPerTile];  // fp16: TMA row coordinate / 8; int8: (block, head) tile
+  int pad[2];
 };
+static_assert(sizeof(TileInfo) == 64, "TileInfo layout");
+
+struct SegInfo {
+  int s, kvh, h, slot;  // sequence (of this launch), KV head, row part, partial slot
+  int L;                // the sequence's context length
+  int rows;             // valid rows of the part
+  int group;            // (s * Hkv + kvh) * halves + h
+  int first;            // this segment makes the group's designated first arrival
+  int expect;           // arrivals the group expects (segments x softmax warpgroups)
+  int bad;              // a block index out of range was replaced by block 0
+  int pad[6];
+};
+static_assert(sizeof(SegInfo) == 64, "SegInfo layout");
 
 struct Misc {
   uint32_t tmem_base;
   int abort;
-  int k_consumed, v_consumed;
-  int last;  // this CTA arrived last in its (sequence, KV head): it merges
-  int bad;   // a block index of this CTA's keys was out of range
+  int nqk, npv;                // QK and PV products issued (drains)
+  int k_conv, v_conv;          // int8: tiles converted (drains)
+  int n_merge;                 // mode 1: groups this CTA merges at the end
+  int own_group;               // mode 0: the KV head whose merge this CTA shares (-1: none)
+  int own_phase;               // ... its barrier phase before this call's arrivals
+  int own_first, own_count;    // ... its partials: CTAs [first, first + count) of the set
+  int own_slice, own_slices;   // ... this CTA's share of the merge
+  int own_s, own_h, own_rows;
+  int segs_published;          // segments whose description was published
+  int segs_done[2];            // segments each softmax warpgroup counted in
+  int last;
+  int pad[11];
+};
+static_assert(sizeof(Misc) <= 128, "Misc layout");
+
+template <int RW, int NG, int KV>
+struct Cfg {
+  static constexpr bool kQuant = KV != kKvFp16;
+  static constexpr bool kQ8 = KV == kKvQ8_0;
+  static constexpr int kVWarp = 2 + NG * 4;      // the V producer's warp
+  static constexpr int kConvWarp = kVWarp + 1;   // int8: first converter warp
+  static constexpr int kConvWarps = 4;           // converter warps per stream (K, V)
+  static constexpr int kThreads = 32 * (kVWarp + 1 + (kQuant ? 2 * kConvWarps : 0));
+  static constexpr int NR = (NG * RW < 16) ? 16 : NG * RW;  // MMA N of QK^T
+  static constexpr int kSG = kQ8 ? kHeadDim / 32 : 1;      // S^T accumulators per tile
+  static constexpr int KS = kQuant ? 2 : 3;
+  static constexpr int VS = kQuant ? 3 : (NR > 16 ? 2 : 3);
+  static constexpr uint32_t kKSlot = kKVBytes;
+  // int8: raw V slots (16 KB of qs, then the tile's scales); the converted V
+  // (hi tile | lo tile) has one slot of its own.
+  static constexpr uint32_t kVSlot = kQuant ? kRawScales + 1024 : kKVBytes;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = KS * kKSlot;
+  static constexpr uint32_t kVC = kV + VS * kVSlot;
+  static constexpr uint32_t kVCBytes = kQuant ? 2 * kKVBytes : 0;
+  static constexpr uint32_t kQ = kVC + kVCBytes;
+  static constexpr uint32_t kQHalf = NR * 128;       // one 64-column half of Q
+  static constexpr uint32_t kQBuf = 2 * kQHalf;      // Q of one segment
+  static constexpr int kPN = 2 * NR;                 // N of the PV product
+  static constexpr int PB = 2;
+  static constexpr uint32_t kP = kQ + 2 * kQBuf;
+  static constexpr uint32_t kPBytes = kTileKeys * kPN * 2;
+  static constexpr uint32_t kRed = kP + PB * kPBytes;                 // float [NG][2][4][32]
+  static constexpr uint32_t kLsum = kRed + NG * 2 * 4 * 32 * 4;       // float [NG][4][32]
+  static constexpr uint32_t kBars = kLsum + NG * 4 * 32 * 4;          // uint64 [kBarSlots]
+  static constexpr uint32_t kInfo = kBars + kBarSlots * 8;
+  static constexpr uint32_t kSeg = kInfo + kInfoSlots * sizeof(TileInfo);
+  static constexpr uint32_t kMisc = kSeg + kSegSlots * sizeof(SegInfo);
+  static constexpr uint32_t kQueueArr = kMisc + 128;   // mode 1: int [3][kMaxQueueSeqs + 1]
+  static constexpr uint32_t kMergeList = kQueueArr + 3 * (kMaxQueueSeqs + 1) * 4;
+  static constexpr uint32_t kTotal = kMergeList + kMergeListLen * 4;
+  // TMEM: S^T[2] (kSG accumulators of NR columns), then O^T[2] (2 NR: the
+  // high parts' products, then the residuals').
+  static constexpr uint32_t kTmemS = 2 * kSG * NR;
+  static constexpr uint32_t kTmemO = 2 * NR;
+  static constexpr uint32_t kTmemUsed = kTmemS + 2 * kTmemO;
+  static constexpr uint32_t kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64
+                                        : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
+  static_assert(KS <= kMaxStages && VS <= kMaxStages, "ring depth");
+  static_assert(kTotal + 1024 <= 232448, "shared memory per CTA");
+  static_assert(kV % 1024 == 0 && kVSlot % 1024 == 0 && kVC % 1024 == 0 && kQ % 1024 == 0,
+                "tiles sit on 1 KB swizzle atoms");
+  static_assert(kTmemUsed <= 512, "TMEM columns");
+  static_assert(NG == 2 && NG * RW <= 32 && RW % 4 == 0, "rows per part");
 };
 
-// What the K producer publishes for each local tile of a CTA: the tile's
-// number in the head's key space (-1: no more tiles), which of its 16-key
-// chunks were loaded, and each loaded chunk's TMA row coordinate (row / 8).
-struct TileInfo {
-  int tile;
-  uint32_t mask;
-  int row8[kChunksPerTile];
-  int pad[2];
-};
-static_assert(sizeof(TileInfo) == 48, "TileInfo layout");
-
-// 32-bit load through the non-coherent path, issued in program order with
-// the other volatile loads (so that two independent loads are in flight).
+// ---------------------------------------------------------------- helpers
 __device__ __forceinline__ int ld_nc_s32(const int* p) {
   int r;
   asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(r) : "l"(p));
@@ -231,13 +231,16 @@ __device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
   asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
   return r;
 }
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
+  uint32_t r;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
 __device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
 }
-// Shared-memory loads by 32-bit shared address (issued in program order with
-// the other volatile shared-memory accesses).
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 r;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -250,103 +253,25 @@ __device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
   return r;
 }
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+  return r;
+}
 __device__ __forceinline__ void sts_v2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
 
-// Visible 128-key tiles of a sequence of context length L (0 for a length
-// outside [n_query, max_blocks_per_seq * block_size]); also its first key
-// rounded down to a 16-key chunk and its visible range.
-struct SeqTiles {
-  int lo, hi, base, tiles;
-};
-__device__ __forceinline__ SeqTiles seq_tiles(const DecodeParams& p, int L) {
-  SeqTiles t{0, -1, 0, 0};
-  if (context_len_ok(L, p.n_query, p.max_blocks_per_seq, p.block_size)) {
-    union_range(L, p.n_query, p.causal, p.window, t.lo, t.hi);
-    t.base = (t.lo / kChunk) * kChunk;
-    if (t.hi >= t.lo) t.tiles = (t.hi + 1 - t.base + kTileKeys - 1) / kTileKeys;
-  }
-  return t;
-}
-
-// Which (sequence, KV head) group CTA c of the C CTAs works for.  Each of the
-// G = num_seqs * num_kv_heads groups gets C / G CTAs, as even as whole CTAs
-// allow: group g owns CTAs [cum(g), cum(g+1)) with cum(g) = g + floor((C -
-// G) g / G), in blockIdx order.  The grid and this mapping depend on the
-// shapes alone, never on the context lengths, so a sequence's splits, and
-// with them every bit of its output, do not depend on the other sequences
-// of the batch.
-struct GroupOf {
-  int s, kvh, split, splits, first;  // first: the group's first CTA
-};
-__device__ __forceinline__ GroupOf group_of(const DecodeParams& p, int c, int C) {
-  GroupOf r;
-  if (p.tiles_per_item > 0) {  // items: num_splits consecutive CTAs per group
-    const int g = c / p.num_splits;
-    r.s = g / p.num_kv_heads;
-    r.kvh = g % p.num_kv_heads;
-    r.splits = p.num_splits;
-    r.first = g * p.num_splits;
-    r.split = c - r.first;
-    return r;
-  }
-  const int G = p.num_seqs * p.num_kv_heads;
-  const long long E = (long long)C - G;
-  auto cum = [&](int g) { return g + (int)(E * g / G); };
-  int g = (int)((long long)c * G / C);
-  while (g > 0 && cum(g) > c) --g;
-  while (g + 1 < G && cum(g + 1) <= c) ++g;
-  r.s = g / p.num_kv_heads;
-  r.kvh = g % p.num_kv_heads;
-  r.first = cum(g);
-  r.splits = cum(g + 1) - r.first;
-  r.split = c - r.first;
-  return r;
-}
-
-// q8_0 cache: byte offset of the qs rows of the 16-key chunk that starts at
-// key key0 of (block, head) tile `tile` (tiles are block_size * (128 + 8)
-// bytes: qs [block_size][128] then fp16 d [block_size][4]).
-__device__ __forceinline__ long long q8_chunk_offset(const DecodeParams& p, int tile, int key0) {
-  return (long long)tile * p.block_size * (kHeadDim + 8) + (long long)(key0 % p.block_size) * kHeadDim;
-}
-// ... and from there to the chunk's scales.
-__device__ __forceinline__ long long q8_scale_offset(const DecodeParams& p, int key0) {
-  const int slot = key0 % p.block_size;
-  return (long long)(p.block_size - slot) * kHeadDim + slot * 8;
-}
-
-// ... and of the four scales of one key (slot `slot` of its block) of q8_0
-// (block, head) tile `tile`.
-__device__ __forceinline__ long long q8_key_scales_offset(const DecodeParams& p, int tile, int slot) {
-  return (long long)tile * p.block_size * (kHeadDim + 8) + (long long)p.block_size * kHeadDim +
-         (long long)slot * 8;
-}
-
-// A q8_0 scale d (fp16 bits) as d = m * 2^e with 2^e the power of two of its
-// exponent field (2^-14 for zero and subnormal scales): 2^e as fp16 bits, and
-// the factor 2^-e that turns d into m (|m| in [1, 2), below 1 for subnormal
-// scales).  Both are exact.
-__device__ __forceinline__ uint16_t q8_scale_pow2_bits(uint16_t d) {
-  const uint16_t e = d & 0x7C00u;
-  return e != 0 ? e : (uint16_t)0x0400u;
-}
-__device__ __forceinline__ float q8_scale_mantissa(uint16_t d) {
-  const int E = max((int)((d >> 10) & 31u), 1);
-  return __half2float(__ushort_as_half(d)) * __int_as_float((127 + 15 - E) << 23);
-}
-
-// Eight signed bytes -> eight exact fp16 values, two per half2: byte b
+// Four signed bytes -> four exact fp16 values, two per half2: byte b
 // becomes the low mantissa byte of the fp16 1024 + (b + 128) (bits 0x6400 |
 // (b ^ 0x80)), minus 1152; every integer below 2048 is exact in fp16.
-__device__ __forceinline__ void q8_to_half8(uint2 q, __half2 (&x)[4]) {
-  const uint32_t w0 = q.x ^ 0x80808080u, w1 = q.y ^ 0x80808080u;
-  const uint32_t u[4] = {__byte_perm(w0, 0x64646464u, 0x5140), __byte_perm(w0, 0x64646464u, 0x7362),
-                         __byte_perm(w1, 0x64646464u, 0x5140), __byte_perm(w1, 0x64646464u, 0x7362)};
+__device__ __forceinline__ void q8_to_half4(uint32_t q, __half2& lo, __half2& hi) {
+  const uint32_t w = q ^ 0x80808080u;
+  const uint32_t a = __byte_perm(w, 0x64646464u, 0x5140), b = __byte_perm(w, 0x64646464u, 0x7362);
   const __half2 off = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));  // 1152
-#pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = __hsub2(*reinterpret_cast<const __half2*>(&u[e]), off);
+  lo = __hsub2(*reinterpret_cast<const __half2*>(&a), off);
+  hi = __hsub2(*reinterpret_cast<const __half2*>(&b), off);
 }
 
 // Warp transpose-reduction over the 32 lanes (= 32 keys): lane l ends with
@@ -372,227 +297,256 @@ __device__ __forceinline__ float warp_row_reduce(float (&v)[RW], int lane) {
   return v[0];
 }
 
-// The last CTA of a (sequence, KV head) merges the group's split partials
-// into the output rows: M = max_k lse_k, w_k = exp(lse_k - M) (0 for an
-// empty split), out = sum_k w_k O_k / sum_k w_k, splits added in index
-// order.  The group's partial rows are staged in shared memory with 16-byte
-// asynchronous copies, as many splits per round as fit, all of a round in
-// flight at once, so that the merge costs a few memory latencies rather than
-// one per split.
-template <int RW, int NG, bool Q8>
-__device__ __forceinline__ void merge_group(const DecodeParams& p, int s, int kvh, int S, int first,
-                                            uint8_t* smem, uint32_t sbase) {
-  using C = Cfg<RW, NG, Q8>;
-  constexpr int kThreads = C::kThreads;
-  constexpr int kRowF4 = kHeadDim / 4;  // float4 per partial row
+// ----------------------------------------------------- the work decomposition
+// Visible keys of a sequence (all its tokens; in partial mode only those in
+// its key range) cut into 16-key chunks from `base` (the first visible key
+// rounded down to a chunk).  bad: a context length outside [n_query,
+// max_blocks_per_seq * block_size], or a key range that is not whole blocks
+// inside the context and the table; nch = 0 then, and also for a valid key
+// range that no query sees.
+struct SeqVis {
+  int lo, hi, base, nch, kb;
+  bool bad;
+};
+__device__ __forceinline__ SeqVis seq_vis(const DecodeParams& p, int s, int L) {
+  SeqVis v{0, -1, 0, 0, 0, false};
+  int kb = 0, kc = 0;
+  bool ok;
+  if (p.key_begin != nullptr) {
+    kb = ld_nc_s32(p.key_begin + s);
+    kc = ld_nc_s32(p.key_count + s);
+    ok = L >= p.n_query && kb >= 0 && kb % p.block_size == 0 && kc >= 0 &&
+         (long long)kb + kc <= L && (long long)kc <= (long long)p.max_blocks_per_seq * p.block_size;
+  } else {
+    ok = context_len_ok(L, p.n_query, p.max_blocks_per_seq, p.block_size);
+  }
+  if (!ok) {
+    v.bad = true;
+    return v;
+  }
+  union_range(L, p.n_query, p.causal, p.window, v.lo, v.hi);
+  if (p.key_begin != nullptr) {
+    v.lo = max(v.lo, kb);
+    v.hi = min(v.hi, kb + kc - 1);
+  }
+  v.kb = kb;
+  v.base = (v.lo / kChunk) * kChunk;
+  if (v.hi >= v.lo) v.nch = (v.hi + 1 - v.base + kChunk - 1) / kChunk;
+  return v;
+}
+__device__ __forceinline__ int part_rows(const DecodeParams& p, int h) {
+  return min(p.rows, (h + 1) * p.rows_half) - h * p.rows_half;
+}
+// Keys that some row of part h can see: the union over the part's tokens
+// (consecutive tokens' ranges overlap, so the union is one range).
+__device__ __forceinline__ void part_range(const DecodeParams& p, int L, int h, int& lo, int& hi) {
+  const int r0 = h * p.rows_half;
+  const int r1 = r0 + part_rows(p, h) - 1;
+  int lo0, hi0, lo1, hi1;
+  key_range(L, p.n_query, r0 / p.group, p.causal, p.window, lo0, hi0);
+  key_range(L, p.n_query, r1 / p.group, p.causal, p.window, lo1, hi1);
+  lo = min(lo0, lo1);
+  hi = max(hi0, hi1);
+}
+// Mode 0: the CTA of Ce whose chunk range [k W / Ce, (k+1) W / Ce) holds
+// chunk x, and the first CTA whose range ends at or after chunk y.
+__device__ __forceinline__ int cta_holding(long long x, int Ce, long long W) {
+  return (int)(((x + 1) * Ce - 1) / W);
+}
+__device__ __forceinline__ int cta_ending_from(long long y, int Ce, long long W) {
+  return (int)(((y + 1) * Ce + W - 1) / W) - 1;
+}
+// Mode 1: a group's chunks are items of 8T chunks, the last of which is cut
+// into up to four sub-items (processed after every big item).
+__device__ __forceinline__ void seq_items(int nch, int T, int& n_big, int& n_sub) {
+  if (nch <= 0) {  // a sequence with a bad length: one item that writes its rows as 0
+    n_big = 0;
+    n_sub = 1;
+    return;
+  }
+  n_big = (nch + 8 * T - 1) / (8 * T) - 1;
+  const int last = nch - n_big * 8 * T;
+  n_sub = min(4, (last + kChunksPerTile - 1) / kChunksPerTile);
+}
+
+// What the K producer knows of the segment it streams (kb: the sequence's
+// first key in this call's block table, 0 outside partial mode).
+struct SegDesc {
+  int s, kvh, h, c0, c1, slot, L, base, kb, lo, hi, vis_lo, vis_hi, expect, first;
+};
+
+// Output row of local row r of part h of (sequence s, KV head kvh).
+__device__ __forceinline__ long long out_row(const DecodeParams& p, int s, int kvh, int h, int r) {
+  const int gr = h * p.rows_half + r;
+  return ((long long)s * p.n_query + gr / p.group) * p.num_q_heads + kvh * p.group + gr % p.group;
+}
+
+// A group's arrival counter pair: [0] mode 0 barrier, [1] mode 1 count.
+__device__ __forceinline__ int* group_counter(const DecodeParams& p, int group) {
+  return p.arrivals + (long long)group * 2;
+}
+
+// Count `n` arrivals of a segment into its group (the designated first
+// arrival adds 2^31 minus the others, so that the top bit flips once every
+// arrival is in and the low bits return to zero).  Mode 1: the arrival that
+// completes the group resets the counter and returns true.
+__device__ __forceinline__ bool arrive(const DecodeParams& p, int group, int expect, bool first,
+                                       int n) {
+  int* cnt = group_counter(p, group);
+  if (p.mode == 0) {
+    red_release_add_gpu(cnt, first ? 0x80000000u - (unsigned)(expect - n) : (unsigned)n);
+    return false;
+  }
+  const int old = atomicAdd(cnt + 1, n);
+  if (old + n == expect) {
+    atomicExch(cnt + 1, 0);
+    return true;
+  }
+  return false;
+}
+
+// ------------------------------------------------------------------ merges
+// Merge of S consecutive partial slots [slot0, slot0 + S) of one group into
+// its output rows, the (row, float4 column) pairs [pa, pb) of it: M = max_k
+// lse_k, w_k = exp(lse_k - M) (0 for an empty split), out = sum_k w_k O_k /
+// sum_k w_k, splits added in slot order with a fixed lane split, so results
+// are reproducible.  A NaN log-sum-exp marks a partial that read a
+// stand-in for an out-of-range block: the group's rows are written as 0.
+// The partial columns are staged with 16-byte asynchronous copies, all of a
+// round in flight at once.
+template <int kThreads>
+__device__ __forceinline__ void merge_pairs(const DecodeParams& p, long long slot0, int S, int rows,
+                                            int s, int kvh, int h, int pa, int pb, uint8_t* smem,
+                                            uint32_t sbase, uint32_t smem_cap) {
+  constexpr int kRowF4 = kHeadDim / 4;
   constexpr int kWarps = kThreads / 32;
-  constexpr int kPairsMax = (NG * RW * kRowF4 + kThreads - 1) / kThreads;  // rows <= NG * RW
-  const int R = p.rows, G = p.group, Hq = p.num_q_heads;
-  const long long rps = (long long)p.n_query * Hq;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  float* w = reinterpret_cast<float*>(smem);  // [S][R]
-  float* inv = w + S * R;                     // [R]
-  const uint32_t stage_off = ((uint32_t)(S * R + R) * 4u + 1023u) & ~1023u;
-  const uint32_t stage = sbase + stage_off;
-  const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);
-  const int per_round = max(1, (int)((C::kRed - stage_off) / (uint32_t)(R * kHeadDim * 4)));
-  auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
-  const long long split0 = (long long)first * R;  // partial row of (split 0, row 0) of the group
-
-  // Raw log-sum-exps, all loads in flight together.
-  for (int i0 = 0; i0 < S * R; i0 += 8 * kThreads) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads + threadIdx.x;
-      v[u] = i < S * R ? __ldcg(p.part_lse + split0 + i) : 0.f;  // [split][row]
+  const long long RHs = p.rows_half;  // partial rows per slot
+  while (pa < pb) {
+    const int r_lo = pa / kRowF4;
+    int np = pb - pa;  // as many pairs per round as the staging area holds
+    for (;;) {
+      const int nr = (pa + np - 1) / kRowF4 - r_lo + 1;
+      const uint32_t stage_off = ((uint32_t)(nr * S + nr) * 4u + 1023u) & ~1023u;
+      if (stage_off + (uint32_t)(S * np) * 16u <= smem_cap || np == 1) break;
+      np = max(1, np / 2);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads + threadIdx.x;
-      if (i < S * R) w[i] = v[u];
+    const int nr = (pa + np - 1) / kRowF4 - r_lo + 1;
+    float* w = reinterpret_cast<float*>(smem);  // [nr][S]
+    float* inv = w + nr * S;                    // [nr]
+    const uint32_t stage_off = ((uint32_t)(nr * S + nr) * 4u + 1023u) & ~1023u;
+    const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);  // [S][np]
+    for (int e = threadIdx.x; e < S * np; e += kThreads) {
+      const int k = e / np, pr = pa + e % np;
+      const float* src =
+          p.part_out + ((slot0 + k) * RHs + pr / kRowF4) * kHeadDim + (pr % kRowF4) * 4;
+      cp_async_16(sbase + stage_off + (uint32_t)e * 16u, src);
     }
-  }
-  __syncthreads();
-  for (int r = warp; r < R; r += kWarps) {
-    float M = -INFINITY;
-    bool bad = false;  // a split read a stand-in for an out-of-range block
-    for (int k = lane; k < S; k += 32) {
-      M = fmaxf(M, w[k * R + r]);
-      bad |= isnan(w[k * R + r]);
-    }
-    bad = __any_sync(0xffffffffu, bad);
+    for (int e = threadIdx.x; e < nr * S; e += kThreads)
+      w[e] = __ldcg(p.part_lse + (slot0 + e % S) * RHs + r_lo + e / S);
+    __syncthreads();
+    for (int j = warp; j < nr; j += kWarps) {
+      float M = -INFINITY;
+      bool bad = false;
+      for (int k = lane; k < S; k += 32) {
+        M = fmaxf(M, w[j * S + k]);
+        bad |= isnan(w[j * S + k]);
+      }
+      bad = __any_sync(0xffffffffu, bad);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float sum = 0.f;
-    for (int k = lane; k < S; k += 32) {
-      const float l = w[k * R + r];
-      const float wk = (bad || l == -INFINITY) ? 0.f : expf(l - M);
-      w[k * R + r] = wk;
-      sum += wk;
-    }
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float sum = 0.f;
+      for (int k = lane; k < S; k += 32) {
+        const float l = w[j * S + k];
+        const float wk = (bad || l == -INFINITY) ? 0.f : expf(l - M);
+        w[j * S + k] = wk;
+        sum += wk;
+      }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) inv[r] = sum > 0.f ? 1.f / sum : 0.f;
-  }
-
-  // Thread = (row, 4 consecutive head_dim elements), up to kPairsMax pairs;
-  // empty splits carry weight 0 and a zero partial.
-  float4 acc[kPairsMax];
-#pragma unroll
-  for (int q = 0; q < kPairsMax; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k0 = 0; k0 < S; k0 += per_round) {
-    const int k1 = min(S, k0 + per_round);
-    __syncthreads();  // weights ready / the previous round's reads done
-    // Staged row q = (k - k0) * R + r; lane = its float4 column (kThreads is
-    // a multiple of 32, so every copy of this thread has column `lane`).
-    const int nrows = (k1 - k0) * R;
-    for (int q = warp; q < nrows; q += kWarps) {
-      const int k = k0 + q / R, r = q % R;
-      const float* src = p.part_out + (split0 + (long long)k * R + r) * kHeadDim + lane * 4;
-      cp_async_16(stage + (uint32_t)(q * kRowF4 + lane) * 16u, src);
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) {
+        inv[j] = sum > 0.f ? 1.f / sum : 0.f;
+        // partial mode: the row's log-sum-exp, written by the share that
+        // holds the row's first column
+        const int r = r_lo + j;
+        if (p.out_lse != nullptr && r < rows && r * kRowF4 >= pa && r * kRowF4 < pb)
+          p.out_lse[out_row(p, s, kvh, h, r)] = sum > 0.f ? M + logf(sum) : -INFINITY;
+      }
     }
     cp_async_wait_all();
     __syncthreads();
-#pragma unroll
-    for (int q = 0; q < kPairsMax; ++q) {
-      const int pr = threadIdx.x + q * kThreads;
-      if (pr < R * kRowF4) {
-        const int r = pr / kRowF4, c4 = pr % kRowF4;
-        for (int k = k0; k < k1; ++k) {
-          const float wk = w[k * R + r];
-          const float4 v = stage4[((k - k0) * R + r) * kRowF4 + c4];
-          acc[q].x = fmaf(wk, v.x, acc[q].x);
-          acc[q].y = fmaf(wk, v.y, acc[q].y);
-          acc[q].z = fmaf(wk, v.z, acc[q].z);
-          acc[q].w = fmaf(wk, v.w, acc[q].w);
+    // tp lanes of one warp per pair, each adding every tp-th split, then a
+    // fixed butterfly; loop bounds are uniform per warp.
+    int tp = 1;
+    while (tp < 32 && 2 * tp * np <= kThreads) tp *= 2;
+    const int per_warp = 32 / tp, sub = lane % tp;
+    for (int q0 = warp * per_warp; q0 < np; q0 += kWarps * per_warp) {
+      const int q = q0 + lane / tp;
+      const bool valid = q < np;
+      const int pr = pa + (valid ? q : 0), r = pr / kRowF4, c4 = pr % kRowF4, j = r - r_lo;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (valid) {
+        for (int k = sub; k < S; k += tp) {
+          const float wk = w[j * S + k];
+          const float4 v = stage4[k * np + q];
+          acc.x = fmaf(wk, v.x, acc.x);
+          acc.y = fmaf(wk, v.y, acc.y);
+          acc.z = fmaf(wk, v.z, acc.z);
+          acc.w = fmaf(wk, v.w, acc.w);
+        }
+      }
+      for (int o = tp / 2; o > 0; o >>= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+      }
+      if (valid && sub == 0 && r < rows) {
+        const float iv = inv[j];
+        if (p.out_f32 != nullptr) {
+          *reinterpret_cast<float4*>(p.out_f32 + out_row(p, s, kvh, h, r) * kHeadDim + c4 * 4) =
+              make_float4(acc.x * iv, acc.y * iv, acc.z * iv, acc.w * iv);
+        } else {
+          uint2 u;
+          u.x = h2_bits(__floats2half2_rn(acc.x * iv, acc.y * iv));
+          u.y = h2_bits(__floats2half2_rn(acc.z * iv, acc.w * iv));
+          *reinterpret_cast<uint2*>(p.out + out_row(p, s, kvh, h, r) * kHeadDim + c4 * 4) = u;
         }
       }
     }
+    __syncthreads();  // the staging area is reused by the next round
+    pa += np;
   }
-#pragma unroll
-  for (int q = 0; q < kPairsMax; ++q) {
-    const int pr = threadIdx.x + q * kThreads;
-    if (pr < R * kRowF4) {
-      const int r = pr / kRowF4, c4 = pr % kRowF4;
-      const float iv = inv[r];
-      const __half2 h0 = __floats2half2_rn(acc[q].x * iv, acc[q].y * iv);
-      const __half2 h1 = __floats2half2_rn(acc[q].z * iv, acc[q].w * iv);
-      uint2 u;
-      u.x = *reinterpret_cast<const uint32_t*>(&h0);
-      u.y = *reinterpret_cast<const uint32_t*>(&h1);
-      *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
+}
+
+// Output rows of part h of (s, kvh) that see no key (a bad length, or in
+// partial mode a key range no query sees): 0 (partial mode: O = 0,
+// lse = -inf).
+__device__ __forceinline__ void zero_rows(const DecodeParams& p, int s, int kvh, int h, int lane) {
+  const int rows = part_rows(p, h);
+  for (int e = lane; e < rows * (kHeadDim / 8); e += 32) {
+    const int r = e / (kHeadDim / 8), c = e % (kHeadDim / 8);
+    const long long row = out_row(p, s, kvh, h, r);
+    if (p.out_f32 != nullptr) {
+      float4* o = reinterpret_cast<float4*>(p.out_f32 + row * kHeadDim + c * 8);
+      o[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      o[1] = o[0];
+      if (c == 0) p.out_lse[row] = -INFINITY;
+    } else {
+      *reinterpret_cast<uint4*>(p.out + row * kHeadDim + c * 8) = make_uint4(0, 0, 0, 0);
     }
   }
 }
 
-// Cooperative merge (every CTA of the grid resident): once its whole group
-// has written its partials, split k of a (sequence, KV head) merges pairs
-// [k*P/S, (k+1)*P/S) of the group's P = R*32 (row, float4 column) pairs.
-// The log-sum-exp weights of merge_group, spread over all S CTAs of the
-// group so that each stages only a few kilobytes of partials with one round
-// of 16-byte asynchronous copies; the weighted partials of a pair are added
-// in a fixed order (lane i of a pair's lanes takes splits i, i + tp, ...,
-// then a butterfly), so results stay reproducible.
-template <int RW, int NG, bool Q8>
-__device__ __forceinline__ void merge_slice(const DecodeParams& p, int s, int kvh, int split, int S,
-                                            int first, uint8_t* smem, uint32_t sbase) {
-  constexpr int kThreads = Cfg<RW, NG, Q8>::kThreads;
-  constexpr int kRowF4 = kHeadDim / 4;
-  constexpr int kWarps = kThreads / 32;
-  const int R = p.rows, G = p.group, Hq = p.num_q_heads;
-  const long long rps = (long long)p.n_query * Hq;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int P = R * kRowF4;
-  const int pa = (int)((long long)split * P / S), pb = (int)((long long)(split + 1) * P / S);
-  if (pa >= pb) return;  // uniform across the CTA
-  const int r_lo = pa / kRowF4, nr = (pb - 1) / kRowF4 - r_lo + 1, np = pb - pa;
-  auto row_index = [&](int r) { return (long long)(r / G) * Hq + kvh * G + (r % G); };
-  const long long split0 = (long long)first * R;  // partial row of (split 0, row 0) of the group
-  float* w = reinterpret_cast<float*>(smem);  // [nr][S]
-  float* inv = w + nr * S;                    // [nr]
-  const uint32_t stage_off = ((uint32_t)(nr * S + nr) * 4u + 1023u) & ~1023u;
-  const float4* stage4 = reinterpret_cast<const float4*>(smem + stage_off);  // [S][np]
-
-  // The partial columns first (the longest wait), then the log-sum-exps.
-  for (int e = threadIdx.x; e < S * np; e += kThreads) {
-    const int k = e / np, pr = pa + e % np;
-    const float* src =
-        p.part_out + (split0 + (long long)k * R + pr / kRowF4) * kHeadDim + (pr % kRowF4) * 4;
-    cp_async_16(sbase + stage_off + (uint32_t)e * 16u, src);
-  }
-  for (int e = threadIdx.x; e < nr * S; e += kThreads)
-    w[e] = __ldcg(p.part_lse + split0 + (long long)(e % S) * R + r_lo + e / S);
-  __syncthreads();
-  for (int j = warp; j < nr; j += kWarps) {
-    float M = -INFINITY;
-    bool bad = false;  // a split read a stand-in for an out-of-range block
-    for (int k = lane; k < S; k += 32) {
-      M = fmaxf(M, w[j * S + k]);
-      bad |= isnan(w[j * S + k]);
-    }
-    bad = __any_sync(0xffffffffu, bad);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float sum = 0.f;
-    for (int k = lane; k < S; k += 32) {
-      const float l = w[j * S + k];
-      const float wk = (bad || l == -INFINITY) ? 0.f : expf(l - M);
-      w[j * S + k] = wk;
-      sum += wk;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) inv[j] = sum > 0.f ? 1.f / sum : 0.f;
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  // tp threads (lanes of one warp) per pair, each adding every tp-th split;
-  // then a fixed butterfly over the tp lanes.  Loop bounds are uniform per
-  // warp, so every lane takes part in the shuffles.
-  int tp = 1;
-  while (tp < 32 && 2 * tp * np <= kThreads) tp *= 2;
-  const int per_warp = 32 / tp, sub = lane % tp;
-  for (int q0 = warp * per_warp; q0 < np; q0 += kWarps * per_warp) {
-    const int q = q0 + lane / tp;
-    const bool valid = q < np;
-    const int pr = pa + (valid ? q : 0), r = pr / kRowF4, c4 = pr % kRowF4, j = r - r_lo;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (valid) {
-      for (int k = sub; k < S; k += tp) {
-        const float wk = w[j * S + k];
-        const float4 v = stage4[k * np + q];
-        acc.x = fmaf(wk, v.x, acc.x);
-        acc.y = fmaf(wk, v.y, acc.y);
-        acc.z = fmaf(wk, v.z, acc.z);
-        acc.w = fmaf(wk, v.w, acc.w);
-      }
-    }
-    for (int o = tp / 2; o > 0; o >>= 1) {
-      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
-      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
-      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
-      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
-    }
-    if (valid && sub == 0) {
-      const float iv = inv[j];
-      const __half2 h0 = __floats2half2_rn(acc.x * iv, acc.y * iv);
-      const __half2 h1 = __floats2half2_rn(acc.z * iv, acc.w * iv);
-      uint2 u;
-      u.x = *reinterpret_cast<const uint32_t*>(&h0);
-      u.y = *reinterpret_cast<const uint32_t*>(&h1);
-      *reinterpret_cast<uint2*>(p.out + ((long long)s * rps + row_index(r)) * kHeadDim + c4 * 4) = u;
-    }
-  }
-}
-
-template <int RW, int NG, bool Q8>
-__global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
+template <int RW, int NG, int KV, bool TR>
+__global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using C = Cfg<RW, NG, Q8>;
-  constexpr int kThreads = C::kThreads, kGroups = NG, kVWarp = C::kVWarp;
+  using C = Cfg<RW, NG, KV>;
+  constexpr bool kQuant = C::kQuant, kQ8 = C::kQ8;
+  constexpr int kThreads = C::kThreads, kVWarp = C::kVWarp;
   constexpr int NR = C::NR, KS = C::KS, VS = C::VS, PB = C::PB;
+  constexpr int kScaleBytes = KV == kKvQ8_0 ? 8 : 4;  // scales of one key (int8 caches)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the __shared__ array by pointer
   // arithmetic so that accesses through it stay shared-space loads/stores.
@@ -600,203 +554,409 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   Misc* misc = reinterpret_cast<Misc*>(smem + C::kMisc);
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + C::kInfo);
+  SegInfo* seginfo = reinterpret_cast<SegInfo*>(smem + C::kSeg);
+  int* merge_list = reinterpret_cast<int*>(smem + C::kMergeList);
   volatile int* abort = &misc->abort;
+  const unsigned long long wl = p.wait_limit_ns;
   auto bar = [&](int i) { return sbase + C::kBars + 8u * i; };
+  auto wait = [&](int b, int parity) { return mbar_wait(bar(b), (uint32_t)parity, abort, wl); };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nq = p.n_query, G = p.group, Hq = p.num_q_heads, R = p.rows;
-  const int C_all = gridDim.x, cta = blockIdx.x;
-
-  // Launched as a programmatic dependent of whatever precedes it on the
-  // stream: set-up above touched only registers; nothing global is read
-  // before that grid has completed and flushed.  Dependents of this grid
-  // may launch at once (they wait the same way).
-  griddep_wait();
-  griddep_launch_dependents();
-  // Which (sequence, KV head) this CTA works for: every thread computes it
-  // (arithmetic only), so that no barrier stands between the grid
-  // dependency and the first memory reads.  The context length is read at
-  // once; with one sequence, the K producer lanes read the block-table
-  // entries of this CTA's first tile at the same time, on the guess that the
-  // whole table is visible (no window, full length), used below only if the
-  // guess held.  Both latencies overlap.
-  const GroupOf go = group_of(p, cta, C_all);
-  const int s = go.s, kvh = go.kvh, split = go.split, S = go.splits, first = go.first;
-  const int L = ld_nc_s32(p.context_lens + s);
-  int spec_key0 = -1, spec_phys = 0;
-  if (warp == 0 && p.num_seqs == 1 && p.tiles_per_item == 0 && lane < kChunksPerTile) {
-    const int ntg =
-        (int)(((long long)p.max_blocks_per_seq * p.block_size + kTileKeys - 1) / kTileKeys);
-    const int tfg = go.split * (ntg / go.splits) + min(go.split, ntg % go.splits);
-    const int key0 = tfg * kTileKeys + lane * kChunk;
-    if (ntg / go.splits + (go.split < ntg % go.splits ? 1 : 0) > 0 &&
-        key0 / p.block_size < p.max_blocks_per_seq) {
-      spec_key0 = key0;
-      spec_phys = ld_nc_s32(p.block_table + key0 / p.block_size);
-    }
-  }
-  // Group barrier of the cooperative merge (below): its phase bit, read
-  // before this CTA arrives (it cannot flip before then).
-  int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
-  unsigned int bar_phase = 0;
-  if (p.coop && threadIdx.x == 0) bar_phase = (unsigned int)ld_acquire_gpu(cnt) & 0x80000000u;
-  // Partials: CTA c owns rows [c*R, c*R + R) of the partial outputs and
-  // log-sum-exps; the CTAs of one group are consecutive.
-  const long long part_base = (long long)cta * R;
-  auto row_index = [&](int r) { return (r / G) * Hq + kvh * G + (r % G); };
-
-  // ---- the head's visible keys and its tiles (uniform across the CTA) ------
-  // The keys of (sequence s, KV head kvh) that any query token sees form
-  // [lo_u, hi_u]; they are cut into 128-key tiles from `base`, and the S
-  // splits take contiguous runs of them (as even as whole tiles allow, or
-  // items of tiles_per_item tiles).  The partition depends only on the
-  // sequence's own context length and the shapes, so every call on the same
-  // inputs adds the same tiles in the same order: results are
-  // bit-reproducible.
-  const int* table = p.block_table + (long long)s * p.max_blocks_per_seq;
-  const SeqTiles st_ = seq_tiles(p, L);
-  const int lo_u = st_.lo, hi_u = st_.hi, base = st_.base, ntiles_h = st_.tiles;
-  if (!context_len_ok(L, nq, p.max_blocks_per_seq, p.block_size) && split == 0 && kvh == 0 &&
-      threadIdx.x == 0)
-    atomicOr(p.flags, kFlagBadLen);
-  int t_first, t_count;
-  if (p.tiles_per_item > 0) {  // item `split` of T tiles
-    t_first = split * p.tiles_per_item;
-    t_count = max(0, min(p.tiles_per_item, ntiles_h - t_first));
-  } else {  // the S CTAs of the group take contiguous runs, as even as whole tiles allow
-    const int t_per = ntiles_h / S, t_rem = ntiles_h % S;
-    t_first = split * t_per + min(split, t_rem);
-    t_count = t_per + (split < t_rem ? 1 : 0);
-  }
-
-  const uint32_t sKr = sbase + C::kK, sVr = sbase + C::kV;
+  const int Hkv = p.num_kv_heads, H = p.halves;
+  const uint32_t sK = sbase + C::kK, sV = sbase + C::kV, sVC = sbase + C::kVC;
   const uint32_t sQ = sbase + C::kQ, sP = sbase + C::kP;
 
-  if (t_count == 0) {
-    // Every tile is another CTA's: an empty partial (weight 0 in the merge).
-    for (int t = threadIdx.x; t < R * kHeadDim; t += kThreads) {
-      const int r = t / kHeadDim;
-      p.part_out[(part_base + r) * kHeadDim + t % kHeadDim] = 0.f;
-      if (t % kHeadDim == 0) p.part_lse[part_base + r] = -INFINITY;
-    }
-  } else if (warp == 0) {
-    // ======================= K producer (also sets up the barriers) ========
+  // Launched as a programmatic dependent of whatever precedes it on the
+  // stream: nothing global is read before that grid has completed.
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // =========================== K producer ===================================
     if (lane == 0) {
       for (int i = 0; i < kMaxStages; ++i) {
         mbar_init(bar(BAR_KFULL + i), 1);
         mbar_init(bar(BAR_KEMPTY + i), 1);
         mbar_init(bar(BAR_VFULL + i), 1);
-        mbar_init(bar(BAR_VEMPTY + i), 1);
-        if (Q8) {  // q8_0: a slot's fp16 tile is ready once every converter warp arrived
-          mbar_init(bar(BAR_CKFULL + i), C::kConvWarps);
-          mbar_init(bar(BAR_CVFULL + i), C::kConvWarps);
-        }
+        // int8 raw V slots are freed by the converter warps, fp16 ones by a commit
+        mbar_init(bar(BAR_VEMPTY + i), kQuant ? C::kConvWarps : 1);
+        mbar_init(bar(BAR_CKFULL + i), C::kConvWarps);
       }
+      mbar_init(bar(BAR_CVFULL), C::kConvWarps);
+      mbar_init(bar(BAR_CVEMPTY), 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(bar(BAR_SFULL + i), 1);
-        mbar_init(bar(BAR_SEMPTY + i), 4 * kGroups);
-        mbar_init(bar(BAR_PFULL + i), 4 * kGroups);
+        mbar_init(bar(BAR_SEMPTY + i), 4 * NG);
+        mbar_init(bar(BAR_PFULL + i), 4 * NG);
+        mbar_init(bar(BAR_OEMPTY + i), 4 * NG);
+        mbar_init(bar(BAR_QFULL + i), 1);
+        mbar_init(bar(BAR_QEMPTY + i), 1);
       }
       mbar_init(bar(BAR_OFULL), 1);
       mbar_init(bar(BAR_DONE), 1);
       for (int i = 0; i < kInfoSlots; ++i) mbar_init(bar(BAR_INFO + i), 1);
       misc->abort = 0;
-      misc->bad = 0;
-      misc->k_consumed = misc->v_consumed = 0;
+      misc->nqk = misc->npv = misc->k_conv = misc->v_conv = 0;
+      misc->n_merge = 0;
+      misc->own_group = -1;
+      misc->segs_published = 0;
+      misc->segs_done[0] = misc->segs_done[1] = 0;
       fence_mbar_init();
     }
     __syncwarp();
-    // The other roles wait for these barriers; this warp starts loading now.
     named_bar_arrive(kBarSetup, kThreads);
 
-    // Lane c < 8 owns chunk c of every tile.  Its block-table entry for tile
-    // t + 1 is read right after tile t's copy is issued and used one slot
-    // wait later, so the load's latency hides behind that wait.
-    const int c = lane;
-    constexpr long long kNone = -(1LL << 40);
-    auto tile_of = [&](int t) { return t < t_count ? t_first + t : -1; };
-    // Physical block of chunk c of local tile t (kNone: not loaded).
-    auto lookup_raw = [&](int t) -> long long {
-      const int g = tile_of(t);
-      if (g < 0 || c >= kChunksPerTile) return kNone;
-      const int key0 = base + g * kTileKeys + c * kChunk;
-      if (key0 > hi_u || key0 + kChunk - 1 < lo_u) return kNone;
-      return table[key0 / p.block_size];
+    const int c = lane;  // lane c < 8 owns chunk c of every tile
+    const int cta = blockIdx.x, Cgrid = gridDim.x;
+    int* qarr = reinterpret_cast<int*>(smem + C::kQueueArr);  // mode 1: Ls, P1, P2
+    int* Ls = qarr;
+    int* P1 = Ls + (kMaxQueueSeqs + 1);
+    int* P2 = P1 + (kMaxQueueSeqs + 1);
+    const int nseq = p.num_seqs;
+    int total_items = 0, p1_total = 0;
+    int next_q = 0;  // mode 1: the next item index, taken one segment ahead
+
+    // -- mode 0: this CTA's chunk range of its (sequence, part) set ---------
+    int m0_s = 0, m0_h = 0, m0_k = 0, m0_L = 0, m0_Ce = 0, m0_nseg = 0, m0_next = 0;
+    SeqVis m0_v{0, -1, 0, 0};
+    long long m0_a = 0, m0_b = 0, m0_W = 0;
+    if (p.mode == 0) {
+      const int sigma = cta / p.ctas_per_set;
+      m0_k = cta % p.ctas_per_set;
+      m0_s = sigma / H;
+      m0_h = sigma % H;
+      m0_L = ld_nc_s32(p.context_lens + m0_s);
+      m0_v = seq_vis(p, m0_s, m0_L);
+      m0_W = (long long)Hkv * m0_v.nch;
+      m0_Ce = (int)(m0_W < (long long)p.ctas_per_set ? m0_W : (long long)p.ctas_per_set);
+      if (m0_W == 0) {
+        // No key (a bad length, or a key range no query sees): the set's
+        // first CTA writes the part's rows.
+        if (m0_k == 0) {
+          for (int g = 0; g < Hkv; ++g) zero_rows(p, m0_s, g, m0_h, lane);
+          if (lane == 0 && m0_h == 0 && m0_v.bad) atomicOr(p.flags, kFlagBadLen);
+        }
+      } else if (m0_k < m0_Ce) {
+        m0_a = (long long)m0_k * m0_W / m0_Ce;
+        m0_b = (long long)(m0_k + 1) * m0_W / m0_Ce;
+        const int kvh0 = (int)(m0_a / m0_v.nch);
+        m0_nseg = (m0_b > (long long)(kvh0 + 1) * m0_v.nch) ? 2 : 1;
+        // Merge duty: the KV head of this CTA's last chunk, shared with the
+        // other CTAs whose range ends in it.
+        const int g = (int)((m0_b - 1) / m0_v.nch);
+        const long long g0 = (long long)g * m0_v.nch;
+        const int ko_lo = cta_ending_from(g0, m0_Ce, m0_W);
+        const int ko_hi =
+            g + 1 < Hkv ? cta_ending_from(g0 + m0_v.nch, m0_Ce, m0_W) - 1 : m0_Ce - 1;
+        const int kf = cta_holding(g0, m0_Ce, m0_W);
+        const int kl = cta_holding(g0 + m0_v.nch - 1, m0_Ce, m0_W);
+        if (lane == 0) {
+          const int grp = (m0_s * Hkv + g) * H + m0_h;
+          misc->own_phase = (int)((unsigned)ld_acquire_gpu(group_counter(p, grp)) & 0x80000000u);
+          misc->own_group = g;
+          misc->own_first = kf;
+          misc->own_count = kl - kf + 1;
+          misc->own_slice = m0_k - ko_lo;
+          misc->own_slices = ko_hi - ko_lo + 1;
+          misc->own_s = m0_s;
+          misc->own_h = m0_h;
+          misc->own_rows = part_rows(p, m0_h);
+        }
+      }
+    } else {
+      // -- mode 1: per-sequence item counts and their prefix sums ----------
+      const int GH = Hkv * H;
+      int run1 = 0, run2 = 0;
+      if (lane == 0) {
+        P1[0] = 0;
+        P2[0] = 0;
+      }
+      for (int s0 = 0; s0 < nseq; s0 += 32) {
+        const int s = s0 + lane;
+        int nb = 0, ns = 0;
+        if (s < nseq) {
+          const int L = ld_nc_s32(p.context_lens + s);
+          seq_items(seq_vis(p, s, L).nch, p.item_tiles, nb, ns);
+          Ls[s] = L;
+        }
+        int a = nb * GH, b = ns * GH;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {  // inclusive scans
+          const int ya = __shfl_up_sync(0xffffffffu, a, o), yb = __shfl_up_sync(0xffffffffu, b, o);
+          if (lane >= o) {
+            a += ya;
+            b += yb;
+          }
+        }
+        if (s < nseq) {
+          P1[s + 1] = run1 + a;
+          P2[s + 1] = run2 + b;
+        }
+        run1 += __shfl_sync(0xffffffffu, a, 31);
+        run2 += __shfl_sync(0xffffffffu, b, 31);
+      }
+      p1_total = run1;
+      total_items = run1 + run2;
+      __syncwarp();
+      if (lane == 0) next_q = atomicAdd(p.queue, 1);
+      next_q = __shfl_sync(0xffffffffu, next_q, 0);
+    }
+
+    // The next segment of this CTA (false: none left).  Mode 1 takes items
+    // off the queue until one with keys comes up; every CTA makes exactly one
+    // take past the end, and the last of all takes resets the counter.
+    auto next_segment = [&](SegDesc& d) -> bool {
+      if (p.mode == 0) {
+        if (m0_next >= m0_nseg) return false;
+        d.kvh = (int)(m0_a / m0_v.nch) + m0_next;
+        const long long g0 = (long long)d.kvh * m0_v.nch;
+        d.c0 = (int)max(0LL, m0_a - g0);
+        d.c1 = (int)min((long long)m0_v.nch, m0_b - g0);
+        d.s = m0_s;
+        d.h = m0_h;
+        d.L = m0_L;
+        d.base = m0_v.base;
+        d.kb = m0_v.kb;
+        d.lo = m0_v.lo;
+        d.hi = m0_v.hi;
+        d.slot = (m0_s * H + m0_h) * (p.ctas_per_set + Hkv) + m0_k + d.kvh;
+        const int kf = cta_holding(g0, m0_Ce, m0_W);
+        const int kl = cta_holding(g0 + m0_v.nch - 1, m0_Ce, m0_W);
+        d.expect = (kl - kf + 1) * NG;
+        d.first = d.c0 == 0;
+        ++m0_next;
+      } else {
+        for (;;) {
+          int q = next_q;
+          if (q >= total_items) {
+            if (q == total_items + Cgrid - 1 && lane == 0) atomicExch(p.queue, 0);
+            return false;
+          }
+          if (lane == 0) next_q = atomicAdd(p.queue, 1);  // the one after, in flight
+          next_q = __shfl_sync(0xffffffffu, next_q, 0);
+          const bool phase1 = q < p1_total;
+          const int* P = phase1 ? P1 : P2;
+          if (!phase1) q -= p1_total;
+          int lo = 0, hi = nseq - 1;  // the last s with P[s] <= q
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (P[mid] <= q) lo = mid; else hi = mid - 1;
+          }
+          const int s = lo;
+          int rem = q - P[s];
+          d.h = rem % H;
+          rem /= H;
+          d.kvh = rem % Hkv;
+          const int i = rem / Hkv;
+          d.s = s;
+          d.L = Ls[s];
+          const SeqVis v = seq_vis(p, s, d.L);
+          int nb, ns;
+          seq_items(v.nch, p.item_tiles, nb, ns);
+          if (v.nch == 0) {  // no key: write the part's rows
+            zero_rows(p, s, d.kvh, d.h, lane);
+            if (lane == 0 && d.kvh == 0 && d.h == 0 && v.bad) atomicOr(p.flags, kFlagBadLen);
+            continue;
+          }
+          const int g = (s * Hkv + d.kvh) * H + d.h;
+          d.base = v.base;
+          d.kb = v.kb;
+          d.lo = v.lo;
+          d.hi = v.hi;
+          if (phase1) {
+            d.c0 = i * 8 * p.item_tiles;
+            d.c1 = d.c0 + 8 * p.item_tiles;
+            d.slot = g * p.slots_per_group + i;
+          } else {
+            const int start = nb * 8 * p.item_tiles, last = v.nch - start;
+            d.c0 = start + (int)((long long)i * last / ns);
+            d.c1 = start + (int)((long long)(i + 1) * last / ns);
+            d.slot = g * p.slots_per_group + nb + i;
+          }
+          d.expect = (nb + ns) * NG;
+          d.first = 0;
+          break;
+        }
+      }
+      int plo, phi;
+      part_range(p, d.L, d.h, plo, phi);
+      d.vis_lo = max(max(plo, d.lo), d.base + d.c0 * kChunk);
+      d.vis_hi = min(min(phi, d.hi), d.base + d.c1 * kChunk - 1);
+      return true;
     };
-    // TMA row coordinate (row / 8) of that chunk, -1 if it is not loaded.
-    // An out-of-range block is never dereferenced: row 0 of the cache stands
-    // in for it (so that every visible key has finite-or-not data the
-    // softmax need not know about), the error flag is raised, and the CTA's
-    // partial is marked invalid so that the merge writes the group's rows
-    // as 0.
-    auto to_row8 = [&](long long phys, int t) -> int {
+
+    // Q rows of a segment -> registers (lane-strided 16-byte pieces), later
+    // -> shared memory, K-major with the 128-byte swizzle: row n, piece cc of
+    // half cc / 8 at half * kQHalf + n * 128 + ((cc % 8) ^ (n % 8)) * 16.
+    // Rows past the part's valid rows are zero.  A negative scale is moved
+    // into Q (an exact sign flip), so scores are only multiplied by cs >= 0.
+    constexpr int kQPer = NR * 16 / 32;  // 16-byte pieces per lane
+    uint4 qreg[kQPer];
+    const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+    auto load_q = [&](const SegDesc& d) {
+      const int rows = part_rows(p, d.h);
+#pragma unroll
+      for (int k = 0; k < kQPer; ++k) {
+        const int e = k * 32 + lane, n = e / 16, cc = e % 16;
+        qreg[k] = make_uint4(0, 0, 0, 0);
+        if (n < rows) qreg[k] = ldg_nc_v4(p.q + out_row(p, d.s, d.kvh, d.h, n) * kHeadDim + cc * 8);
+      }
+    };
+    auto store_q = [&](int qb) {
+      const uint32_t dst = sQ + qb * C::kQBuf;
+#pragma unroll
+      for (int k = 0; k < kQPer; ++k) {
+        const int e = k * 32 + lane, n = e / 16, cc = e % 16;
+        uint4 v = qreg[k];
+        v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
+        sts_v4(dst + (cc / 8) * C::kQHalf + n * 128 + (((cc % 8) ^ (n & 7)) * 16), v);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_QFULL + qb));
+    };
+
+    // Block-table entry of chunk c of the tile that starts at chunk tc0
+    // (kNone: not copied).
+    constexpr long long kNone = -(1LL << 40);
+    auto lookup = [&](const SegDesc& d, int tc0) -> long long {
+      const int ci = tc0 + c;
+      if (c >= kChunksPerTile || ci >= d.c1) return kNone;
+      const int key0 = d.base + ci * kChunk;
+      if (key0 > d.vis_hi || key0 + kChunk - 1 < d.vis_lo) return kNone;
+      return ld_nc_s32(p.block_table + (long long)d.s * p.max_blocks_per_seq +
+                       (key0 - d.kb) / p.block_size);
+    };
+    // TMA row coordinate / 8 (fp16) or (block, head) tile (int8) of that
+    // chunk; -1 if not copied.  An out-of-range block is never dereferenced:
+    // block 0 stands in for it, the error flag is raised and the segment is
+    // marked, so that the merge writes the group's rows as 0.
+    auto to_row8 = [&](long long phys, const SegDesc& d, int tc0, int segslot) -> int {
       if (phys == kNone) return -1;
       if (phys < 0 || phys >= p.num_blocks) {
         atomicOr(p.flags, kFlagBadBlock);
-        misc->bad = 1;
-        return 0;
+        seginfo[segslot].bad = 1;
+        phys = 0;
       }
-      if (Q8) return (int)(phys * p.num_kv_heads + kvh);  // q8_0: the (block, head) tile
-      const int key0 = base + tile_of(t) * kTileKeys + c * kChunk;
-      return (int)(((phys * p.num_kv_heads + kvh) * p.block_size + key0 % p.block_size) / 8);
+      if (kQuant) return (int)(phys * Hkv + d.kvh);
+      const int key0 = d.base + (tc0 + c) * kChunk;
+      return (int)(((phys * Hkv + d.kvh) * p.block_size + key0 % p.block_size) / 8);
     };
-    long long raw0 = kNone;
-    if (c < kChunksPerTile && t_count > 0) {
-      const int key0 = base + t_first * kTileKeys + c * kChunk;
-      if (key0 <= hi_u && key0 + kChunk - 1 >= lo_u)
-        raw0 = key0 == spec_key0 ? (long long)spec_phys : (long long)table[key0 / p.block_size];
-    }
-    int row_cur = to_row8(raw0, 0);
-    long long raw_nxt = lookup_raw(1);
-    int issued = 0;
-    for (int t = 0;; ++t) {
-      const int g_cur = tile_of(t);
-      const bool w_cur = row_cur >= 0;
-      // Publish tile t for the V producer, the MMA issuer and the softmax.
-      const uint32_t mask = __ballot_sync(0xffffffffu, w_cur);
-      TileInfo& ti = info[t % kInfoSlots];
-      if (lane < kChunksPerTile) ti.row8[lane] = row_cur;
+    // A segment this CTA owns but will not compute (abort path): an invalid
+    // partial, counted in for every softmax warpgroup.
+    auto give_up = [&](const SegDesc& d) {
+      const int rows = part_rows(p, d.h);
+      for (int r = lane; r < rows; r += 32)
+        p.part_lse[(long long)d.slot * p.rows_half + r] = __uint_as_float(kInvalidLse);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) arrive(p, (d.s * Hkv + d.kvh) * H + d.h, d.expect, d.first, NG);
+    };
+
+    int t = 0, seg_n = 0, seg_written = 0;
+    SegDesc cur{};
+    bool have = next_segment(cur);
+    if (have) load_q(cur);
+    long long raw_cur = have ? lookup(cur, cur.c0) : kNone;
+    bool ok = true;
+    while (have && ok) {
+      const int segslot = seg_n % kSegSlots, qb = seg_n % 2;
       if (lane == 0) {
-        ti.tile = g_cur;
-        ti.mask = mask;
+        SegInfo& si = seginfo[segslot];
+        si.s = cur.s; si.kvh = cur.kvh; si.h = cur.h; si.slot = cur.slot;
+        si.L = cur.L; si.rows = part_rows(p, cur.h);
+        si.group = (cur.s * Hkv + cur.kvh) * H + cur.h;
+        si.first = cur.first; si.expect = cur.expect; si.bad = 0;
       }
+      seg_written = seg_n + 1;
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_INFO + t % kInfoSlots));
-      if (g_cur < 0) break;
-      // Wait for the slot, then every lane issues its chunk's copy.
-      const int st = t % KS;
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar(BAR_KEMPTY + st), ((t / KS) & 1) ^ 1, abort);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // The Q buffer of this segment is free once QK of segment seg_n - 2 ended.
+      int w = 1;
+      if (lane == 0) w = wait(BAR_QEMPTY + qb, ((seg_n / 2) & 1) ^ 1);
+      ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       if (!ok) break;
-      const uint32_t fb = bar(BAR_KFULL + st);
-      if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8QsChunk : kChunkBytes));
-      __syncwarp();
-      if (w_cur) {
-        if constexpr (Q8) {
-          // K's scales are read by the softmax (from L2), not staged here.
-          const long long off = q8_chunk_offset(p, row_cur, base + g_cur * kTileKeys + c * kChunk);
-          const uint8_t* src = static_cast<const uint8_t*>(p.k);
-          bulk_load(sKr + st * C::kKSlot + kRawOff + c * kQ8QsChunk, src + off, kQ8QsChunk, fb);
-          bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off, kChunk * kHeadDim);
-          bulk_prefetch_l2(static_cast<const uint8_t*>(p.v) + off +
-                               q8_scale_offset(p, base + g_cur * kTileKeys + c * kChunk),
-                           kChunk * 8);
-        } else {
-          tma_load_4d(sKr + st * kKVBytes + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
-          tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+      const int ntile = (cur.c1 - cur.c0 + kChunksPerTile - 1) / kChunksPerTile;
+      SegDesc nxt{};
+      for (int tau = 0; tau < ntile; ++tau) {
+        const int tc0 = cur.c0 + tau * kChunksPerTile;
+        const int row_cur = to_row8(raw_cur, cur, tc0, segslot);
+        // The next tile's block-table entries, in flight during this one.
+        const bool more = tau + 1 < ntile;
+        long long raw_nxt = more ? lookup(cur, tc0 + kChunksPerTile) : kNone;
+        const uint32_t mask = __ballot_sync(0xffffffffu, row_cur >= 0);
+        TileInfo& ti = info[t % kInfoSlots];
+        if (lane < kChunksPerTile) ti.row8[lane] = row_cur;
+        if (lane == 0) {
+          ti.seg = seg_n;
+          ti.flags = (tau == 0 ? 1 : 0) | (tau == ntile - 1 ? 2 : 0);
+          ti.key0 = cur.base + tc0 * kChunk;
+          ti.vis_lo = cur.vis_lo;
+          ti.vis_hi = cur.vis_hi;
+          ti.mask = mask;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_INFO + t % kInfoSlots));
+        const int st = t % KS;
+        if (lane == 0) w = wait(BAR_KEMPTY + st, ((t / KS) & 1) ^ 1);
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
+        if (!ok) break;
+        const uint32_t fb = bar(BAR_KFULL + st);
+        if (lane == 0) mbar_arrive_expect_tx(fb, __popc(mask) * (kQuant ? kQsChunk : kChunkBytes));
+        __syncwarp();
+        if (row_cur >= 0) {
+          if constexpr (kQuant) {
+            const long long tb = quant_tile_bytes(KV, p.block_size);
+            const int slot0 = (cur.base + (tc0 + c) * kChunk) % p.block_size;
+            const long long off = (long long)row_cur * tb + (long long)slot0 * kHeadDim;
+            const long long soff = (long long)row_cur * tb + (long long)p.block_size * kHeadDim +
+                                   (long long)slot0 * kScaleBytes;
+            const uint8_t* kc = static_cast<const uint8_t*>(p.k);
+            const uint8_t* vc = static_cast<const uint8_t*>(p.v);
+            bulk_load(sK + st * C::kKSlot + kRawOff + c * kQsChunk, kc + off, kQsChunk, fb);
+            bulk_prefetch_l2(kc + soff, kChunk * kScaleBytes);  // K scales: the softmax reads them
+            bulk_prefetch_l2(vc + off, kQsChunk);
+            bulk_prefetch_l2(vc + soff, kChunk * kScaleBytes);
+          } else {
+            tma_load_4d(sK + st * C::kKSlot + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
+            tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+          }
+        }
+        __syncwarp();
+        if (tau == 0) store_q(qb);
+        ++t;
+        if (!more) {
+          // Next segment: its descriptor, Q rows and first block-table entries.
+          ++seg_n;
+          have = next_segment(nxt);
+          if (have) {
+            load_q(nxt);
+            raw_nxt = lookup(nxt, nxt.c0);
+          }
+        }
+        raw_cur = raw_nxt;
       }
-      __syncwarp();
-      issued = t + 1;
-      row_cur = to_row8(raw_nxt, t + 1);
-      raw_nxt = lookup_raw(t + 2);
+      cur = nxt;
     }
+    if (ok) {  // end of the stream
+      if (lane == 0) {
+        TileInfo& ti = info[t % kInfoSlots];
+        ti.seg = -1;
+        ti.flags = 0;
+        mbar_arrive(bar(BAR_INFO + t % kInfoSlots));
+      }
+    } else {
+      // Abort: count in every segment this CTA owns but did not publish, and
+      // (mode 1) take the remaining items off the queue the same way.
+      SegDesc d{};
+      while (next_segment(d)) give_up(d);
+    }
+    if (lane == 0) misc->segs_published = seg_written;
+    __syncwarp();
     __syncthreads();  // (A) every role finished its loop
-    if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
+    if (lane == 0) {  // drain copies that no consumer waited for (abort path only)
       volatile int no_abort = 0;
-      for (int t = misc->k_consumed; t < issued; ++t)
-        mbar_wait(bar(BAR_KFULL + t % KS), (t / KS) & 1, &no_abort);
+      for (int u = kQuant ? misc->k_conv : misc->nqk; u < t; ++u)
+        mbar_wait(bar(BAR_KFULL + u % KS), (u / KS) & 1, &no_abort);
     }
   } else {
     // ---- set-up of the other roles ----------------------------------------
@@ -804,453 +964,476 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
       tmem_alloc(sbase + C::kMisc + offsetof(Misc, tmem_base), C::kTmemCols);
       tmem_relinquish();
     }
-    if (warp >= 2 && warp < kVWarp) {
-      // Q rows of this KV head -> shared memory, K-major with 128-byte
-      // swizzle: row n, 16-byte chunk c of half h at h*NR*128 + n*128 +
-      // ((c ^ n%8) * 16).  Rows >= R are zero; so are P's padding rows (never
-      // written later).  A negative scale is moved into Q (an exact sign
-      // flip) so that the kernel only multiplies scores by a factor >= 0.
-      const int t = threadIdx.x - 64;
-      const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-      for (int c = t; c < NR * 16; c += kGroups * kSoftmaxThreads) {
-        const int n = c / 16, cc = c % 16, h = cc / 8, k8 = cc % 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < R) {
-          const long long qrow = ((long long)s * nq + n / G) * Hq + kvh * G + (n % G);
-          v = ldg_nc_v4(p.q + qrow * kHeadDim + cc * 8);
-          v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
-        }
-        sts_v4(sQ + h * C::kQHalf + n * 128 + ((k8 ^ (n & 7)) * 16), v);
-      }
-      for (uint32_t off = t * 16; off < PB * C::kPBytes; off += kGroups * kSoftmaxThreads * 16)
+    if (warp == kVWarp) {
+      // P buffers start at zero: the columns of padding rows are never written.
+      for (uint32_t off = lane * 16; off < PB * C::kPBytes; off += 32 * 16)
         sts_v4(sP + off, make_uint4(0, 0, 0, 0));
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    named_bar_sync(kBarSetup, kThreads);  // barriers initialised, TMEM allocated, Q staged
+    named_bar_sync(kBarSetup, kThreads);  // barriers initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
 
     if (warp == kVWarp) {
       // ===================== V producer ======================================
-      // Follows the K producer's published tiles; lane c < 8 issues chunk c.
       const int c = lane;
       int issued = 0;
       for (int t = 0;; ++t) {
-        int ok = 1;
-        if (lane == 0)
-          ok = mbar_wait(bar(BAR_INFO + t % kInfoSlots), (t / kInfoSlots) & 1, abort);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        __syncwarp();  // lane 0's acquire orders the other lanes' reads below
-        if (!ok) break;
+        int w = 1;
+        if (lane == 0) w = wait(BAR_INFO + t % kInfoSlots, (t / kInfoSlots) & 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        __syncwarp();
+        if (!w) break;
         const TileInfo& ti = info[t % kInfoSlots];
-        if (ti.tile < 0) break;
+        if (ti.seg < 0) break;
         const uint32_t mask = ti.mask;
-        const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;  // q8_0: the tile index
+        const int row8 = c < kChunksPerTile ? ti.row8[c] : 0;
+        const int key0 = ti.key0 + c * kChunk;
         const int st = t % VS;
-        if (lane == 0) ok = mbar_wait(bar(BAR_VEMPTY + st), ((t / VS) & 1) ^ 1, abort);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        if (lane == 0) w = wait(BAR_VEMPTY + st, ((t / VS) & 1) ^ 1);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) break;
         const uint32_t fb = bar(BAR_VFULL + st);
         if (lane == 0)
-          mbar_arrive_expect_tx(fb, __popc(mask) * (Q8 ? kQ8QsChunk + kQ8DChunk : kChunkBytes));
+          mbar_arrive_expect_tx(fb, __popc(mask) * (kQuant ? kQsChunk + kChunk * kScaleBytes
+                                                           : kChunkBytes));
         __syncwarp();
         if (c < kChunksPerTile && ((mask >> c) & 1u)) {
-          if constexpr (Q8) {
-            const long long off = q8_chunk_offset(p, row8, base + ti.tile * kTileKeys + c * kChunk);
-            const uint32_t dst = sVr + st * C::kVSlot;
-            const uint8_t* src = static_cast<const uint8_t*>(p.v);
-            bulk_load(dst + kRawOff + c * kQ8QsChunk, src + off, kQ8QsChunk, fb);
-            bulk_load(dst + kKVBytes + c * kQ8DChunk,
-                      src + off + q8_scale_offset(p, base + ti.tile * kTileKeys + c * kChunk),
-                      kQ8DChunk, fb);
+          if constexpr (kQuant) {
+            const long long tb = quant_tile_bytes(KV, p.block_size);
+            const int slot0 = key0 % p.block_size;
+            const uint8_t* src = static_cast<const uint8_t*>(p.v) + (long long)row8 * tb;
+            const uint32_t dst = sV + st * C::kVSlot;
+            bulk_load(dst + c * kQsChunk, src + (long long)slot0 * kHeadDim, kQsChunk, fb);
+            bulk_load(dst + kRawScales + c * (kChunk * kScaleBytes),
+                      src + (long long)p.block_size * kHeadDim + (long long)slot0 * kScaleBytes,
+                      kChunk * kScaleBytes, fb);
           } else {
-            tma_load_4d(sVr + st * kKVBytes + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
+            tma_load_4d(sV + st * C::kVSlot + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
           }
         }
         __syncwarp();
         issued = t + 1;
       }
       __syncthreads();  // (A)
-      if (lane == 0) {  // drain copies that no MMA waited for (abort path only)
+      if (lane == 0) {  // drain copies that no consumer waited for (abort path only)
         volatile int no_abort = 0;
-        for (int t = misc->v_consumed; t < issued; ++t)
-          mbar_wait(bar(BAR_VFULL + t % VS), (t / VS) & 1, &no_abort);
+        for (int u = kQuant ? misc->v_conv : misc->npv; u < issued; ++u)
+          mbar_wait(bar(BAR_VFULL + u % VS), (u / VS) & 1, &no_abort);
       }
     } else if (warp == 1) {
       // ===================== MMA issuer ======================================
-      // One thread, in a fixed order: QK(0), QK(1), then PV(t), QK(t+2) for
-      // t = 0, 1, ...  A commit completes once every MMA this thread issued
-      // before it has finished, so S(t) in TMEM also means that O(t-2) is.
-      // The number of tiles is t_count (uniform), so the issuer reads no
-      // published tile information.
       if (lane == 0) {
+        constexpr int kSG = C::kSG;
         const uint32_t id_qk = idesc_f16_f32(128, NR, false, false);
         const uint32_t id_pv = idesc_f16_f32(128, C::kPN, true, true);
-        // Descriptors at offset 0; a byte offset o is added as o >> 4 (the
-        // start-address field is the low 14 bits, addresses stay < 256 KB).
-        // q8_0: K and V are the converted slots (exact fp16 images of the
-        // int8 values; V's rows also carry the power of two of their scales).
-        // S^T gets one accumulator per scale group g (head_dim 32g .. 32g+31,
-        // two steps of 16), which the softmax combines with K's scales; PV
-        // multiplies V with each group's P (the weights times V's scale
-        // mantissas) into that group's O^T accumulator.
-        const uint64_t dK = smem_desc(sKr, 16, kGroupBytes, kSwizzle128B);
+        const uint32_t id_pv_lo = idesc_f16_f32(128, NR, true, true);
+        // Descriptors at offset 0; a byte offset o is added as o >> 4.
+        const uint64_t dK = smem_desc(sK, 16, kGroupBytes, kSwizzle128B);
         const uint64_t dQ = smem_desc(sQ, 16, 1024, kSwizzle128B);
-        const uint64_t dV = smem_desc(sVr, kAtomBytes, kGroupBytes, kSwizzle128B);
+        const uint64_t dV = smem_desc(kQuant ? sVC : sV, kAtomBytes, kGroupBytes, kSwizzle128B);
         const uint64_t dP = smem_desc(sP, C::kPN * 16, 128, kSwizzleNone);
-        constexpr int kSG = C::kSG;
-        // QK(u) once K(u) is ready and the softmax took S(u-2) from its buffer.
-        auto issue_qk = [&](int u) -> bool {
-          const bool ready =
-              mbar_wait(bar((Q8 ? BAR_CKFULL : BAR_KFULL) + u % KS), (u / KS) & 1, abort);
-          if (!(ready && mbar_wait(bar(BAR_SEMPTY + u % 2), ((u / 2) & 1) ^ 1, abort)))
-            return false;
+        int t_end = 0x7fffffff, nqk = 0, npv = 0;
+        // QK(u) once tile u is described, K(u) is ready and the softmax took
+        // S(u-2) from its buffer; returns 0 ok, 1 end of stream, -1 abort.
+        auto issue_qk = [&](int u) -> int {
+          if (!wait(BAR_INFO + u % kInfoSlots, (u / kInfoSlots) & 1)) return -1;
+          const TileInfo& ti = info[u % kInfoSlots];
+          const int seg = ti.seg, flags = ti.flags;
+          if (seg < 0) return 1;
+          if ((flags & 1) && !wait(BAR_QFULL + seg % 2, (seg / 2) & 1)) return -1;
+          if (!wait((kQuant ? BAR_CKFULL : BAR_KFULL) + u % KS, (u / KS) & 1)) return -1;
+          if (!wait(BAR_SEMPTY + u % 2, ((u / 2) & 1) ^ 1)) return -1;
           tc_fence_after();
           const uint64_t so = (uint64_t)((u % KS) * C::kKSlot) >> 4;
+          const uint64_t qo0 = (uint64_t)((seg % 2) * C::kQBuf) >> 4;
           const uint32_t d = tmem + (u % 2) * kSG * NR;
           constexpr int kSteps = kHeadDim / 16 / kSG;  // steps of 16 per accumulator
 #pragma unroll
           for (int k = 0; k < kHeadDim / 16; ++k) {
             const uint64_t ko = ((k / 4) * kAtomBytes + (k % 4) * 32) >> 4;
             const uint64_t qo = ((k / 4) * C::kQHalf + (k % 4) * 32) >> 4;
-            tc_mma_f16_ss(d + (k / kSteps) * NR, dK + so + ko, dQ + qo, id_qk, k % kSteps != 0);
+            tc_mma_f16_ss(d + (k / kSteps) * NR, dK + so + ko, dQ + qo0 + qo, id_qk, k % kSteps != 0);
           }
           tc_commit(bar(BAR_SFULL + u % 2));
           tc_commit(bar(BAR_KEMPTY + u % KS));
-          return true;
+          if (flags & 2) tc_commit(bar(BAR_QEMPTY + seg % 2));
+          return 0;
         };
-        int nqk = 0, npv = 0;
         bool ok = true;
-        for (int u = 0; u < 2 && u < t_count && ok; ++u) {
-          ok = issue_qk(u);
+        for (int u = 0; u < 2 && ok; ++u) {
+          const int r = issue_qk(u);
+          if (r == 1) {
+            t_end = u;
+            break;
+          }
+          ok = r == 0;
           if (ok) nqk = u + 1;
         }
-        for (int t = 0; ok && t < t_count; ++t) {
-          // PV(t) once P(t), V(t) and the O buffer are ready, then QK(t+2).
-          ok = mbar_wait(bar(BAR_PFULL + t % PB), (t / PB) & 1, abort) &&
-               mbar_wait(bar((Q8 ? BAR_CVFULL : BAR_VFULL) + t % VS), (t / VS) & 1, abort);
+        for (int t = 0; ok && t < t_end; ++t) {
+          const TileInfo& ti = info[t % kInfoSlots];  // described before QK(t)
+          const int seg = ti.seg, flags = ti.flags, ob = seg % 2;
+          ok = wait(BAR_PFULL + t % PB, (t / PB) & 1) &&
+               (kQuant ? wait(BAR_CVFULL, t & 1) : wait(BAR_VFULL + t % VS, (t / VS) & 1)) &&
+               (!(flags & 1) || wait(BAR_OEMPTY + ob, ((seg / 2) & 1) ^ 1));
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = (uint64_t)((t % VS) * C::kVSlot) >> 4;
+          const uint64_t so = kQuant ? 0 : (uint64_t)((t % VS) * C::kVSlot) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
-          // O^T accumulates over all tiles; q8_0: the kSG group accumulators
-          // are the consecutive column ranges of one N = kPN product.
-          const uint32_t d = tmem + C::kTmemS;
+          const uint32_t d = tmem + C::kTmemS + ob * C::kTmemO;
 #pragma unroll
           for (int k = 0; k < kTileKeys / 16; ++k) {
             const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
             const uint64_t po = (k * 2 * C::kPN * 16) >> 4;
-            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, t > 0 || k > 0);
+            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, !(flags & 1) || k > 0);
+            if constexpr (kQuant)  // V_lo times the high parts of P (the first NR columns)
+              tc_mma_f16_ss(d, dV + (kKVBytes >> 4) + vo, dP + pb + po, id_pv_lo, 1);
           }
           tc_commit(bar(BAR_OFULL));
-          tc_commit(bar(BAR_VEMPTY + t % VS));
+          tc_commit(bar(kQuant ? BAR_CVEMPTY : BAR_VEMPTY + t % VS));
           npv = t + 1;
-          if (t + 2 < t_count) {
-            ok = issue_qk(t + 2);
-            if (ok) nqk = t + 3;
+          if (t_end == 0x7fffffff) {
+            const int r = issue_qk(t + 2);
+            if (r == 1) t_end = t + 2;
+            ok = r >= 0;
+            if (r == 0) nqk = t + 3;
           }
         }
-        misc->k_consumed = nqk;
-        misc->v_consumed = npv;
+        misc->nqk = nqk;
+        misc->npv = npv;
         tc_commit(bar(BAR_DONE));  // completes once every MMA above has finished
         volatile int no_abort = 0;
         mbar_wait(bar(BAR_DONE), 0, &no_abort);
       }
       __syncwarp();
       __syncthreads();  // (A)
-    } else if (Q8 && warp >= C::kConvWarp) {
-      // ===================== q8_0 converters =================================
-      // Raw tile t (int8 qs in the upper half of its slot; V: fp16 scales d
-      // per 32 elements after the tile) -> the fp16 operand in the same slot,
-      // exactly: K's operand is qs itself (every integer below 2048 is an
-      // fp16 value; K's scales are applied to the per-group scores in the
-      // softmax), V's is qs * 2^e with 2^e the power of two of the element's
-      // scale d = m * 2^e (exact for |d| < 1024: at most 7 significant bits
-      // above 2^-24); the mantissa m goes into that group's P.  The
-      // arithmetic is packed fp16 (two elements per instruction).  Layout as
-      // the fp16 TMA boxes: [key/8][half][key%8][64 dims], 128-byte swizzle.
-      // V rows of keys outside [lo_u, hi_u] (masked or never loaded) are
-      // written as zeros: they must not reach the PV product.
-      // The first kConvWarps converter warps convert K, the next kConvWarps
-      // V.  Thread ct of a stream's kCT takes the 16-byte column chunk
-      // c16 = ct % 8 (head_dim 16*c16 .. +15, half of one scale group) of keys
-      // r = ct / 8 + kRS*k: one 16-byte load and two 16-byte stores per key,
-      // the swizzled destination offset constant up to the key group, no bank
-      // conflicts on either side.  In place: keys 0 .. 63 land below the raw
-      // data; keys 64 .. 127 are stored only after every thread of the stream
-      // has read (and converted into registers) all its raw rows.
-      constexpr int kCT = 32 * C::kConvWarps;   // threads per stream
-      constexpr int kRS = kCT / 8;              // key stride between a thread's keys
-      constexpr int kKeysPer = kTileKeys / kRS; // keys per thread per tile
-      constexpr int kHalfKeys = kKeysPer / 2;   // per half tile
-      static_assert(kKeysPer % 2 == 0 && (kTileKeys / 2) * 256 <= kRawOff,
-                    "the lower half of the keys is stored below the raw tile");
+    } else if (kQuant && warp >= C::kConvWarp) {
+      // ===================== int8 converters =================================
+      // Layout of a converted tile as the fp16 TMA boxes: [key/8][half]
+      // [key%8][64 dims], 128-byte swizzle.  Thread ct of a stream's 128
+      // takes the 16-byte column chunk c16 = ct % 8 (head_dim 16 c16 .. +15,
+      // half of one q8_0 scale group) of keys r0 + 16 k, k = 0..7: one
+      // 16-byte load and two 16-byte stores per key and operand, no bank
+      // conflicts on either side.
+      // K: in place, the raw int8 tile in the upper half of its slot; keys
+      // 0..63 are written below it, keys 64..127 only after every thread of
+      // the stream has read its raw rows (named barrier); the operand is qs.
+      // V: raw slot -> the converted slot's hi and lo tiles (qs * d split
+      // into two fp16 parts); rows of keys no row of the part sees are
+      // written as zeros.
+      constexpr int kCT = 32 * C::kConvWarps;
+      constexpr int kRS = kCT / 8;               // key stride between a thread's keys (16)
+      constexpr int kKeysPer = kTileKeys / kRS;  // keys per thread per tile (8)
+      constexpr int kHalfKeys = kKeysPer / 2;
       const int kv = (warp - C::kConvWarp) / C::kConvWarps;  // 0: K, 1: V
-      const int ct = threadIdx.x - 32 * (C::kConvWarp + C::kConvWarps * kv);  // 0 .. kCT-1
-      const int c16 = ct & 7, r0 = ct >> 3;      // column chunk, first key
-      const int r08 = r0 & 7;                    // its row within a key group
-      // destination of the two 8-element halves: chunk cc = 2*c16 + e of the
-      // key's 256-byte row, i.e. half cc / 8, 16-byte slot (cc % 8) ^ (key % 8)
+      const int ct = threadIdx.x - 32 * (C::kConvWarp + C::kConvWarps * kv);
+      const int c16 = ct & 7, r0 = ct >> 3;
+      const int r08 = r0 & 7;
       const uint32_t dst_a = (r0 >> 3) * kGroupBytes + ((2 * c16) >> 3) * kAtomBytes + r08 * 128 +
                              ((((2 * c16) & 7) ^ r08) << 4);
       const uint32_t dst_b = (r0 >> 3) * kGroupBytes + ((2 * c16 + 1) >> 3) * kAtomBytes +
                              r08 * 128 + ((((2 * c16 + 1) & 7) ^ r08) << 4);
       const int NSl = kv == 0 ? KS : VS;
-      const uint32_t bar_full = kv == 0 ? BAR_KFULL : BAR_VFULL;
-      const uint32_t bar_conv = kv == 0 ? BAR_CKFULL : BAR_CVFULL;
-      const uint32_t ring = sbase + (kv == 0 ? C::kK : C::kV);
-      const uint32_t slot_bytes = kv == 0 ? C::kKSlot : C::kVSlot;
-      bool ok = true;
-      // Eight int8 -> eight fp16 values times the power of two p2 (1 for K).
-      auto convert = [&](uint32_t w0, uint32_t w1, __half2 p2) -> uint4 {
-        __half2 x[4];
-        q8_to_half8(make_uint2(w0, w1), x);
-        uint32_t h[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half2 y = kv == 0 ? x[e] : __hmul2(x[e], p2);
-          h[e] = *reinterpret_cast<const uint32_t*>(&y);
-        }
-        return make_uint4(h[0], h[1], h[2], h[3]);
-      };
-      for (int t = 0; t < t_count && ok; ++t) {
-        const int key_t = base + (t_first + t) * kTileKeys;  // first key of the tile
+      int t = 0;
+      for (;; ++t) {
+        // The tile's description (end of the stream, V's visible keys), then
+        // the data; the stream's threads decide together so that all of them
+        // reach the named barriers.
+        bool live = wait(BAR_INFO + t % kInfoSlots, (t / kInfoSlots) & 1);
+        const TileInfo& ti = info[t % kInfoSlots];
+        live = live && ti.seg >= 0;
         const int rs = t % NSl;
-        // The stream's threads decide together (one gave up: all stop), so
-        // that every one of them reaches the named barrier below.
-        ok = named_bar_and(kBarConv0 + kv, kCT,
-                           __all_sync(0xffffffffu, mbar_wait(bar(bar_full + rs), (t / NSl) & 1, abort)));
-        if (!ok) break;
-        const uint32_t slot = ring + rs * slot_bytes;
-        const uint32_t src = slot + kRawOff + r0 * kHeadDim + c16 * 16;       // key r0, chunk c16
-        const uint32_t srcd = slot + kKVBytes + r0 * 8 + (c16 >> 1) * 2;     // its scale (V)
+        if (live) live = wait((kv == 0 ? BAR_KFULL : BAR_VFULL) + rs, (t / NSl) & 1);
+        if (live && kv == 1) live = wait(BAR_CVEMPTY, (t & 1) ^ 1);
+        if (!named_bar_and(kBarConv0 + kv, kCT, __all_sync(0xffffffffu, live))) break;
+        const int key_t = ti.key0, vlo = ti.vis_lo, vhi = ti.vis_hi;
+        if (kv == 1) {
+          const uint32_t slot = sV + rs * C::kVSlot;
+          const uint32_t src = slot + r0 * kHeadDim + c16 * 16;
+#pragma unroll 2
+          for (int k = 0; k < kKeysPer; ++k) {
+            const int r = k * kRS + r0;
+            const uint4 qv = lds_v4(src + k * kRS * kHeadDim);
+            uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4 qv[kHalfKeys];
-          uint16_t dv[kHalfKeys];
+            for (int e = 0; e < 8; ++e) hi[e] = lo[e] = 0u;
+            if (key_t + r >= vlo && key_t + r <= vhi) {
+              __half2 x[8];
+              q8_to_half4(qv.x, x[0], x[1]);
+              q8_to_half4(qv.y, x[2], x[3]);
+              q8_to_half4(qv.z, x[4], x[5]);
+              q8_to_half4(qv.w, x[6], x[7]);
+              if constexpr (kQ8) {
+                // d: the fp16 scale of this 32-element group; qs * d split
+                // exactly into fp16(qs * d) and the (exact) residual.
+                const __half d = __ushort_as_half(
+                    lds_u16(slot + kRawScales + r * kScaleBytes + (c16 >> 1) * 2));
+                const __half2 d2 = __halves2half2(d, d);
 #pragma unroll
-          for (int i = 0; i < kHalfKeys; ++i) {
-            const int k = h * kHalfKeys + i;
-            qv[i] = lds_v4(src + k * kRS * kHeadDim);
-            dv[i] = kv == 0 ? (uint16_t)0 : lds_u16(srcd + k * kRS * 8);
+                for (int e = 0; e < 8; ++e) {
+                  const __half2 yh = __hmul2(x[e], d2);
+                  hi[e] = h2_bits(yh);
+                  lo[e] = h2_bits(__hfma2(x[e], d2, __hneg2(yh)));
+                }
+              } else {
+                // s: the fp32 scale of this row; qs * s in fp32, split into
+                // two fp16 parts.
+                const float sc = __uint_as_float(lds_u32(slot + kRawScales + r * kScaleBytes));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float2 f = __half22float2(x[e]);
+                  const float a = f.x * sc, b = f.y * sc;
+                  const __half2 yh = __floats2half2_rn(a, b);
+                  const float2 g2 = __half22float2(yh);
+                  hi[e] = h2_bits(yh);
+                  lo[e] = h2_bits(__floats2half2_rn(a - g2.x, b - g2.y));
+                }
+              }
+            }
+            const uint32_t g8 = k * (kRS / 8) * kGroupBytes;
+            sts_v4(sVC + g8 + dst_a, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+            sts_v4(sVC + g8 + dst_b, make_uint4(hi[4], hi[5], hi[6], hi[7]));
+            sts_v4(sVC + kKVBytes + g8 + dst_a, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+            sts_v4(sVC + kKVBytes + g8 + dst_b, make_uint4(lo[4], lo[5], lo[6], lo[7]));
           }
-          uint4 xa[kHalfKeys], xb[kHalfKeys];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar(BAR_CVFULL));
+            mbar_arrive(bar(BAR_VEMPTY + rs));  // the raw slot may be refilled
+          }
+        } else {
+          const uint32_t slot = sK + rs * C::kKSlot;
+          const uint32_t src = slot + kRawOff + r0 * kHeadDim + c16 * 16;
 #pragma unroll
-          for (int i = 0; i < kHalfKeys; ++i) {
-            const int r = (h * kHalfKeys + i) * kRS + r0;
-            xa[i] = make_uint4(0, 0, 0, 0);
-            xb[i] = xa[i];
-            if (kv == 0 || (key_t + r >= lo_u && key_t + r <= hi_u)) {
-              const __half p2 = __ushort_as_half(q8_scale_pow2_bits(dv[i]));
-              const __half2 p22 = __halves2half2(p2, p2);
-              xa[i] = convert(qv[i].x, qv[i].y, p22);
-              xb[i] = convert(qv[i].z, qv[i].w, p22);
+          for (int hh = 0; hh < 2; ++hh) {
+            uint4 xa[kHalfKeys], xb[kHalfKeys];
+#pragma unroll
+            for (int i = 0; i < kHalfKeys; ++i) {
+              const int k = hh * kHalfKeys + i;
+              const uint4 qv = lds_v4(src + k * kRS * kHeadDim);
+              __half2 a0, a1, a2, a3;
+              q8_to_half4(qv.x, a0, a1);
+              q8_to_half4(qv.y, a2, a3);
+              xa[i] = make_uint4(h2_bits(a0), h2_bits(a1), h2_bits(a2), h2_bits(a3));
+              q8_to_half4(qv.z, a0, a1);
+              q8_to_half4(qv.w, a2, a3);
+              xb[i] = make_uint4(h2_bits(a0), h2_bits(a1), h2_bits(a2), h2_bits(a3));
+            }
+            // The upper keys overwrite raw rows: every thread of the stream
+            // has read all of its rows once it is past this barrier.
+            if (hh == 1) named_bar_sync(kBarConv0 + kv, kCT);
+#pragma unroll
+            for (int i = 0; i < kHalfKeys; ++i) {
+              const uint32_t g8 = (hh * kHalfKeys + i) * (kRS / 8) * kGroupBytes;
+              sts_v4(slot + g8 + dst_a, xa[i]);
+              sts_v4(slot + g8 + dst_b, xb[i]);
             }
           }
-          // The upper half overwrites raw rows: every thread of the stream
-          // has read all of its rows once it is past this barrier.
-          if (h == 1) named_bar_sync(kBarConv0 + kv, kCT);
-#pragma unroll
-          for (int i = 0; i < kHalfKeys; ++i) {
-            const uint32_t g8 = (h * kHalfKeys + i) * (kRS / 8) * kGroupBytes;
-            sts_v4(slot + g8 + dst_a, xa[i]);
-            sts_v4(slot + g8 + dst_b, xb[i]);
-          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_CKFULL + rs));
         }
-        fence_proxy_async_smem();  // generic writes -> the tensor core's reads
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bar_conv + rs));
+        (void)key_t;
+      }
+      if (ct == 0) {
+        if (kv == 0) misc->k_conv = t; else misc->v_conv = t;
       }
       __syncthreads();  // (A)
     } else {
       // ===================== softmax + correction ============================
-      // Warpgroup g handles rows [g*RW, g*RW + RW); its warps cover the four
-      // TMEM lane quarters, i.e. keys (for S) and head_dim elements (for O).
+      // Warpgroup g handles rows [g*RW, g*RW + RW) of the part; its warps
+      // cover the four TMEM lane quarters: keys (for S), head_dim (for O).
       const int g = (warp - 2) / 4, widx = (warp - 2) % 4;
       const int row0 = g * RW;
       const int q4 = warp & 3;
-      const int j = q4 * 32 + lane;
+      const int j = q4 * 32 + lane;  // this thread's key within a tile / head_dim lane of O
       const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
       float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
       float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
-      float* bc = reinterpret_cast<float*>(smem + C::kBcast) + (warp - 2) * 64;  // [2][32]
       const uint32_t bar_id = kBarGroup0 + g;
       const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
-
-      // Per query token, the visible key range; keys inside every token's
-      // range see all rows: the fast path of interior tiles.
-      int tlo[kMaxQuery], thi[kMaxQuery];
-      int lo_all = lo_u, hi_all = hi_u;
-#pragma unroll
-      for (int i = 0; i < kMaxQuery; ++i) {
-        tlo[i] = 1;
-        thi[i] = 0;
-        if (i < nq) {
-          key_range(L, nq, i, p.causal, p.window, tlo[i], thi[i]);
-          lo_all = max(lo_all, tlo[i]);
-          hi_all = min(hi_all, thi[i]);
-        }
-      }
-      const uint32_t grp = G >= 32 ? 0xffffffffu : ((1u << G) - 1u);
-      const uint32_t all_rows = R >= 32 ? 0xffffffffu : ((1u << R) - 1u);
+      constexpr int kSG = C::kSG;
 
       float lpart[RW], bias[RW];
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         lpart[r] = 0.f;
-        bias[r] = INFINITY;  // no reference yet: the row's first key forces one
+        bias[r] = INFINITY;
       }
-      // Reference max (raw score) of row row0 + lane % RW; -inf until the
-      // row sees a key.  bias[r] = kPShift - cs * (row r's reference max).
-      float m_lane = -INFINITY;
+      float m_lane = -INFINITY;  // reference max (raw score) of row row0 + lane % RW
+      int seg_cur = -1, seg_rows = 0, seg_L = 0, seg_h = 0;
+      uint32_t all_rows = 0;
       bool ok = true;
-      const int end_t = t_count;  // tiles of this CTA (local t -> tile t_first + t)
-      // O^T accumulates in TMEM over every tile (from column kTmemS: the
-      // high parts of the rows, then their residuals).  When a row's
-      // reference rises at tile t, its O column is scaled by alpha in place,
-      // after PV(t-1) has finished and before P(t) is published.  fp16: S(t)
-      // in TMEM implies that PV(t-2) has finished (the issuer commits S(t)
-      // after issuing PV(t-2)), so P buffer t % 2 is free again; q8_0 (one P
-      // buffer) waits for PV(t-1) before storing P(t).
-      // q8_0: this thread's lanes of O^T are head_dim elements 32*q4 ..
-      // 32*q4 + 31, i.e. scale group q4: only that group's accumulator is
-      // read (and rescaled) here.
-      const uint32_t o_hi = tmem + lane_off + C::kTmemS + (Q8 ? q4 * 2 * NR : 0) + row0;
-      const uint32_t o_lo = o_hi + NR;
-      constexpr int kSG = C::kSG;
-      // q8_0: the K and V scales of this thread's key (4 fp16 each), read
-      // from the cache (an L2 hit: the tile's bulk copies brought them) one
-      // tile ahead; zeros for a key no row sees.
-      auto fetch_scales = [&](int u) -> uint4 {
-        uint4 sc = make_uint4(0, 0, 0, 0);
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_INFO + u % kInfoSlots),
-                                                     (u / kInfoSlots) & 1, abort));
-        if (ok) {
-          const int key = base + (t_first + u) * kTileKeys + j;
-          const int tix = info[u % kInfoSlots].row8[j / kChunk];  // (block, head) tile, -1: not loaded
-          if (tix >= 0 && key >= lo_u && key <= hi_u) {
-            const long long off = q8_key_scales_offset(p, tix, key % p.block_size);
-            const uint2 a = ldg_nc_v2(static_cast<const uint8_t*>(p.k) + off);
-            const uint2 b = ldg_nc_v2(static_cast<const uint8_t*>(p.v) + off);
-            sc = make_uint4(a.x, a.y, b.x, b.y);
+      int o_seen = 0;  // PV phases known to be complete
+      // Wait until PV(k) has finished: exact while phases < k are complete
+      // and phase k + 1 cannot be (P(k+1) not yet published).
+      auto wait_o_done = [&](int k) -> bool {
+        if (o_seen > k) return true;
+        if (!wait(BAR_OFULL, k & 1)) return false;
+        o_seen = k + 1;
+        return true;
+      };
+      // int8 caches: K's scales of this thread's key (q8_0: four fp16 group
+      // scales; int8 rows: the fp32 row scale), read from the cache (an L2
+      // hit: the K producer prefetched them) one tile ahead; zero for a key
+      // that is not copied.
+      auto fetch_scales = [&](int u) -> uint2 {
+        uint2 sc = make_uint2(0, 0);
+        if constexpr (kQuant) {
+          const TileInfo& ti = info[u % kInfoSlots];
+          const int key = ti.key0 + j;
+          const int tix = ti.row8[j / kChunk];
+          if (tix >= 0 && key >= ti.vis_lo && key <= ti.vis_hi) {
+            const long long off = (long long)tix * quant_tile_bytes(KV, p.block_size) +
+                                  (long long)p.block_size * kHeadDim +
+                                  (long long)(key % p.block_size) * kScaleBytes;
+            const uint8_t* src = static_cast<const uint8_t*>(p.k) + off;
+            if constexpr (kQ8) sc = ldg_nc_v2(src);
+            else sc.x = ldg_nc_u32(src);
           }
         }
         return sc;
       };
-      // Wait until PV(k) has finished.  A parity wait for phase k of the
-      // O barrier is exact only when phases < k have completed and phase k+1
-      // cannot have (P(k+1) not yet published): k = t-1 before P(t) goes
-      // out, where phases < t-1 are complete because S(t) implies PV(t-2).
-      // A wait after the last P went out would not be exact for PV(end_t-2),
-      // so that one is waited for before.  o_seen counts the phases known to
-      // be complete.
-      int o_seen = 0;
-      auto wait_o_done = [&](int k) -> bool {
-        if (o_seen > k) return true;
-        if (!mbar_wait(bar(BAR_OFULL), k & 1, abort)) return false;
-        o_seen = k + 1;
-        return true;
+      auto info_wait = [&](int u) -> bool {
+        int r = 1;
+        if (lane == 0) r = wait(BAR_INFO + u % kInfoSlots, (u / kInfoSlots) & 1);
+        r = __shfl_sync(0xffffffffu, r, 0);
+        __syncwarp();
+        return r != 0;
       };
-      uint4 sc_next = make_uint4(0, 0, 0, 0);
-      if constexpr (Q8) {
-        if (end_t > 0) sc_next = fetch_scales(0);
-      }
-      for (int t = 0; t < end_t; ++t) {
-        const int gt = t_first + t;  // tile number of local tile t
-        const int sb = t % 2, st = t % VS;
-        float mv[kSG];  // q8_0: V's scale mantissas of this key, per group
+      uint2 sc_next = make_uint2(0, 0);
+      bool next_known = false;  // INFO(t) already waited for (scale prefetch)
+      for (int t = 0;; ++t) {
+        // The warpgroup agrees to go on (every warp saw a live tile).
+        bool live = ok && (next_known || info_wait(t));
+        live = live && info[t % kInfoSlots].seg >= 0;
+        if (!named_bar_and(bar_id, kSoftmaxThreads, live)) break;
+        const TileInfo& ti = info[t % kInfoSlots];
+        const int seg = ti.seg, flags = ti.flags, key0 = ti.key0, vlo = ti.vis_lo, vhi = ti.vis_hi;
+        const int sb = t % 2, st = t % VS, ob = seg % 2;
+        if (seg != seg_cur) {
+          // A new segment: its rows, its context and a fresh softmax state.
+          const SegInfo& si = seginfo[seg % kSegSlots];
+          seg_cur = seg;
+          seg_rows = si.rows;
+          seg_L = si.L;
+          seg_h = si.h;
+          const int vr = min(RW, max(0, seg_rows - row0));
+          all_rows = vr >= 32 ? 0xffffffffu : ((1u << vr) - 1u);
+          m_lane = -INFINITY;
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            lpart[r] = 0.f;
+            bias[r] = INFINITY;  // no reference yet: the row's first key forces one
+          }
+        }
+        uint2 sc = make_uint2(0, 0);
+        if constexpr (kQuant) {
+          sc = next_known ? sc_next : fetch_scales(t);
+          next_known = false;
+          if (info_wait(t + 1)) {  // prefetch the next tile's scales
+            next_known = true;
+            if (info[(t + 1) % kInfoSlots].seg >= 0) sc_next = fetch_scales(t + 1);
+          } else {
+            ok = false;
+          }
+        }
         float sv[RW];
 #pragma unroll
         for (int r = 0; r < RW; ++r) sv[r] = 0.f;
-        if constexpr (Q8) {
-          const uint4 sc = sc_next;
-          if (t + 1 < end_t) sc_next = fetch_scales(t + 1);
-          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
-          // Score = sum over the scale groups of K's scale times the group's
-          // partial product (fp32, groups in order).
-          float sg[kSG][RW];
+        ok = __all_sync(0xffffffffu, ok && wait(BAR_SFULL + sb, (t / 2) & 1));
+        if (ok) {
+          tc_fence_after();
+          if constexpr (kQ8) {
+            // Score = sum over the scale groups of K's scale times the
+            // group's partial product (fp32, groups in order).
+            float sg[kSG][RW];
 #pragma unroll
-          for (int q = 0; q < kSG; ++q)
-#pragma unroll
-            for (int r = 0; r < RW; ++r) sg[q][r] = 0.f;
-          if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int q = 0; q < kSG; ++q)
-              tmem_ld<RW>(tmem + lane_off + sb * kSG * NR + q * NR + row0, sg[q]);
+            for (int q = 0; q < kSG; ++q) tmem_ld<RW>(tmem + lane_off + sb * kSG * NR + q * NR + row0, sg[q]);
             tmem_ld_wait();
-            tc_fence_before();
-          }
-          const uint32_t kw[2] = {sc.x, sc.y}, vw[2] = {sc.z, sc.w};
+            const uint32_t kw[2] = {sc.x, sc.y};
 #pragma unroll
-          for (int q = 0; q < kSG; ++q) {
-            const uint16_t kd = (uint16_t)(kw[q / 2] >> (16 * (q % 2)));
-            const uint16_t vd = (uint16_t)(vw[q / 2] >> (16 * (q % 2)));
-            const float dk = __half2float(__ushort_as_half(kd));
-            mv[q] = q8_scale_mantissa(vd);
+            for (int q = 0; q < kSG; ++q) {
+              const float dk = __half2float(__ushort_as_half((uint16_t)(kw[q / 2] >> (16 * (q % 2)))));
 #pragma unroll
-            for (int r = 0; r < RW; ++r) sv[r] = q == 0 ? dk * sg[0][r] : fmaf(dk, sg[q][r], sv[r]);
-          }
-        } else {
-          ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(BAR_SFULL + sb), (t / 2) & 1, abort));
-          mv[0] = 1.f;
-          if (ok) {
-            tc_fence_after();
+              for (int r = 0; r < RW; ++r) sv[r] = q == 0 ? dk * sg[0][r] : fmaf(dk, sg[q][r], sv[r]);
+            }
+          } else {
             tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
             tmem_ld_wait();
-            tc_fence_before();
+            if constexpr (kQuant) {  // int8 rows: K's row scale
+              const float dk = __uint_as_float(sc.x);
+#pragma unroll
+              for (int r = 0; r < RW; ++r) sv[r] *= dk;
+            }
           }
+          tc_fence_before();
         }
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(bar(BAR_SEMPTY + sb));
 
+        // Which rows of the part see this key: the tokens that see it form a
+        // contiguous run, whose rows are a contiguous run of bits.
+        const int key = key0 + j;
         uint32_t rmask = 0;
-        // Which rows see this key?  Chunks that were not loaded lie wholly
-        // outside [lo_u, hi_u], so their keys see none.
-        const int key = base + gt * kTileKeys + j;
-        if (ok && key >= lo_u && key <= hi_u) {
-          if (key >= lo_all && key <= hi_all) {
-            rmask = all_rows;
-          } else {
+        if (ok && key >= vlo && key <= vhi) {
+          int i_lo, i_hi;
+          tokens_seeing(seg_L, p.n_query, p.causal, p.window, key, i_lo, i_hi);
+          const int off = seg_h * p.rows_half;
+          const int b = min(max(i_lo * p.group - off, 0), seg_rows);
+          const int e = min(max((i_hi + 1) * p.group - off, 0), seg_rows);
+          if (e > b) rmask = (e >= 32 ? 0xffffffffu : ((1u << e) - 1u)) & ~((1u << b) - 1u);
+        }
+        const uint32_t rm_g = rmask >> row0;  // this warpgroup's rows
+        const bool all_vis = __all_sync(0xffffffffu, all_rows != 0 && (rm_g & all_rows) == all_rows);
+        if constexpr (TR) {
+          // Key-resolution record: every (row, key) pair this kernel scores,
+          // with the physical slot its K row was copied from.
+          if (ok && rm_g != 0) {
+            const int row8 = ti.row8[j / kChunk];
+            long long phys;
+            if constexpr (kQuant) {
+              phys = row8 / Hkv;
+            } else {
+              const long long row = (long long)row8 * 8 + (key % kChunk);
+              phys = row / p.block_size / Hkv;
+            }
+            const unsigned id = (unsigned)(phys * p.block_size + key % p.block_size);
+            const SegInfo& si = seginfo[seg % kSegSlots];
 #pragma unroll
-            for (int i = 0; i < kMaxQuery; ++i)
-              if (i < nq && key >= tlo[i] && key <= thi[i]) rmask |= grp << (i * G);
+            for (int r = 0; r < RW; ++r) {
+              if ((rm_g >> r) & 1u) {
+                int32_t* tr = p.trace + out_row(p, si.s, si.kvh, si.h, row0 + r) * 5;
+                atomicAdd(tr + 0, 1);
+                atomicMin(tr + 1, key);
+                atomicMax(tr + 2, key);
+                atomicXor(reinterpret_cast<unsigned*>(tr + 3), id);
+                atomicAdd(reinterpret_cast<unsigned*>(tr + 4), id);
+              }
+            }
           }
         }
-        // every key of this warp is seen by every row: the interior fast path
-        const bool all_vis = __all_sync(0xffffffffu, rmask == all_rows);
         // x = cs * s + bias, the log2 of the scaled weight; -inf for a row
         // that does not see this key: its weight is exactly 0 and it cannot
         // raise the row's reference.
         float x[RW];
         float xmax = -INFINITY;
-        if (all_vis) {
 #pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            x[r] = fmaf(sv[r], cs, bias[r]);
-            xmax = fmaxf(xmax, x[r]);
-          }
-        } else {
-          const uint32_t rm = rmask >> row0;
-#pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
-            xmax = fmaxf(xmax, x[r]);
-          }
+        for (int r = 0; r < RW; ++r) {
+          x[r] = (all_vis || ((rm_g >> r) & 1u)) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
+          xmax = fmaxf(xmax, x[r]);
         }
-        const bool exceed = xmax > (float)C::kPShift + kLazy;
-        // Reconverge before the group barrier: a warp that arrives diverged
-        // (after lane-predicated code) makes the barrier several times slower
-        // (measured: 61k verify 122 -> 67 us per call).
+        const bool exceed = xmax > (float)kPShift + kLazy;
+        // Reconverge before the group barrier (a diverged arrival makes the
+        // barrier several times slower).
         __syncwarp();
-        // One barrier per tile: orders the shared-memory traffic of the group
-        // and tells every thread whether any score passed its row's reference.
+        // One barrier per tile: orders the group's shared-memory traffic and
+        // tells every thread whether any score passed its row's reference.
         const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
         if (rescale) {
-          // New reference max per row: warp transpose-reduction, then
-          // across the group's four warps.
-          const uint32_t rm = all_vis ? 0xffffffffu : (rmask >> row0);
+          const uint32_t rm = all_vis ? 0xffffffffu : rm_g;
           float tmp[RW];
 #pragma unroll
           for (int r = 0; r < RW; ++r) tmp[r] = ((rm >> r) & 1u) ? sv[r] : -INFINITY;
@@ -1267,34 +1450,24 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           // alpha = 2^(cs (m_old - m_new)); bias makes 2^(cs s + bias) =
           // 2^(cs (s - m_new) + kPShift).
           const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(cs * (m_lane - m_new));
-          const float bias_l =
-              (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)C::kPShift);
+          const float bias_l = (m_new == -INFINITY) ? INFINITY : fmaf(-cs, m_new, (float)kPShift);
           m_lane = m_new;
-          if (lane < RW) {
-            bc[lane] = bias_l;
-            bc[32 + lane] = alpha;
-          }
-          __syncwarp();
           float av[RW];
 #pragma unroll
-          for (int r = 0; r < RW; r += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(bc + r);
-            const float4 b4 = *reinterpret_cast<const float4*>(bc + 32 + r);
-            bias[r] = a4.x; bias[r + 1] = a4.y; bias[r + 2] = a4.z; bias[r + 3] = a4.w;
-            av[r] = b4.x; av[r + 1] = b4.y; av[r + 2] = b4.z; av[r + 3] = b4.w;
-          }
-#pragma unroll
           for (int r = 0; r < RW; ++r) {
+            bias[r] = __shfl_sync(0xffffffffu, bias_l, r);
+            av[r] = __shfl_sync(0xffffffffu, alpha, r);
             x[r] = ((rm >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
             lpart[r] *= av[r];
           }
-          if (t > 0) {  // rescale the accumulated O columns of this group's rows
+          if (!(flags & 1)) {  // rescale this segment's accumulated O columns
             ok = __all_sync(0xffffffffu, ok && wait_o_done(t - 1));
             if (ok) {
               tc_fence_after();
+              const uint32_t o_hi = tmem + lane_off + C::kTmemS + ob * C::kTmemO + row0;
               float oh[RW], ol[RW];
               tmem_ld<RW>(o_hi, oh);
-              tmem_ld<RW>(o_lo, ol);
+              tmem_ld<RW>(o_hi + NR, ol);
               tmem_ld_wait();
 #pragma unroll
               for (int r = 0; r < RW; ++r) {
@@ -1302,7 +1475,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
                 ol[r] *= av[r];
               }
               tmem_st<RW>(o_hi, oh);
-              tmem_st<RW>(o_lo, ol);
+              tmem_st<RW>(o_hi + NR, ol);
               tmem_st_wait();
               tc_fence_before();  // ordered before the PFULL arrive below
             }
@@ -1317,119 +1490,121 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
           lpart[r] += pw[r];
         }
 
-        // A key no row can see must not reach the PV product: zero its V
-        // row (after its V tile has landed).  (q8_0: the converter does.)
-        if (!Q8 && g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
-          ok = __all_sync(0xffffffffu,
-                          ok && mbar_wait(bar(BAR_VFULL + st), (t / VS) & 1, abort));
+        // fp16 cache: a key no row of the part sees must not reach the PV
+        // product: zero its V row once the V tile has landed (the int8
+        // converters write such rows as zeros themselves).
+        if (!kQuant && g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
+          ok = __all_sync(0xffffffffu, ok && wait(BAR_VFULL + st, (t / VS) & 1));
           if (ok && rmask == 0) {
             const uint4 z = make_uint4(0, 0, 0, 0);
-            const uint32_t vrow = sVr + st * kKVBytes + (j / 8) * kGroupBytes + (j % 8) * 128;
+            const uint32_t vrow = sV + st * C::kVSlot + (j / 8) * kGroupBytes + (j % 8) * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              sts_v4(vrow + c * 16, z);
-              sts_v4(vrow + kAtomBytes + c * 16, z);
+            for (int cc = 0; cc < 8; ++cc) {
+              sts_v4(vrow + cc * 16, z);
+              sts_v4(vrow + kAtomBytes + cc * 16, z);
             }
           }
         }
-        // One P buffer: PV(t-1) must have read it before P(t) goes in.  The
-        // last tile waits for PV(t-1) in any case, so that the final wait
-        // below is for one phase only.
-        if ((PB == 1 || t == end_t - 1) && t > 0) {
+        // A segment's last P goes out only after PV(t-1), so that the wait
+        // for PV(t) below is for one phase only.
+        if ((flags & 2) && t > 0) {
           ok = __all_sync(0xffffffffu, ok && wait_o_done(t - 1));
           if (ok) tc_fence_after();
         }
         if (ok) {
-          // P^T as no-swizzle MN-major core matrices [key/8][n/8][key%8]
-          // [n%8], n = group * 2NR + row' with row' < NR the high parts and
-          // row' >= NR the residuals, in P buffer t % PB.  Each weight (times
-          // V's scale mantissa of the group, q8_0) is split into an fp16 high
-          // part (truncated to 11 significant bits: exact in fp16 over the
-          // weights' range) and an fp16 residual.
+          // P^T as no-swizzle MN-major core matrices [key/8][n/8][key%8][n%8]:
+          // n < NR the high parts of the rows, n >= NR their residuals.  Each
+          // weight is split into an fp16 high part (truncated to 11
+          // significant bits) and a residual.
           const uint32_t kb = (j >> 3) * (C::kPN / 8) * 128 + (j & 7) * 16;
           constexpr uint32_t lo_off = (NR / 8) * 128;
+          const uint32_t pbuf = sP + (t % PB) * C::kPBytes;
+          uint32_t phi[RW / 2], plo[RW / 2];
 #pragma unroll
-          for (int q = 0; q < kSG; ++q) {
-            const uint32_t pbuf = sP + (t % PB) * C::kPBytes + q * (2 * NR / 8) * 128;
-            uint32_t phi[RW / 2], plo[RW / 2];
+          for (int r = 0; r < RW; r += 2) {
+            const float h0 = __uint_as_float(__float_as_uint(pw[r]) & 0xffffe000u);
+            const float h1 = __uint_as_float(__float_as_uint(pw[r + 1]) & 0xffffe000u);
+            phi[r / 2] = h2_bits(__floats2half2_rn(h0, h1));
+            plo[r / 2] = h2_bits(__floats2half2_rn(pw[r] - h0, pw[r + 1] - h1));
+          }
+          if constexpr (RW >= 8) {
 #pragma unroll
-            for (int r = 0; r < RW; r += 2) {
-              const float p0 = Q8 ? pw[r] * mv[q] : pw[r];
-              const float p1 = Q8 ? pw[r + 1] * mv[q] : pw[r + 1];
-              const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-              const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-              const __half2 h = __floats2half2_rn(h0, h1);
-              const __half2 l2 = __floats2half2_rn(p0 - h0, p1 - h1);
-              phi[r / 2] = *reinterpret_cast<const uint32_t*>(&h);
-              plo[r / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+            for (int r8 = 0; r8 < RW / 8; ++r8) {
+              const uint32_t off = kb + ((row0 / 8) + r8) * 128;
+              sts_v4(pbuf + off, make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
+              sts_v4(pbuf + lo_off + off,
+                     make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
             }
-            if constexpr (RW >= 8) {
-#pragma unroll
-              for (int r8 = 0; r8 < RW / 8; ++r8) {
-                const uint32_t off = kb + ((row0 / 8) + r8) * 128;
-                sts_v4(pbuf + off,
-                       make_uint4(phi[r8 * 4], phi[r8 * 4 + 1], phi[r8 * 4 + 2], phi[r8 * 4 + 3]));
-                sts_v4(pbuf + lo_off + off,
-                       make_uint4(plo[r8 * 4], plo[r8 * 4 + 1], plo[r8 * 4 + 2], plo[r8 * 4 + 3]));
-              }
-            } else {  // four rows: half of one 16-byte core-matrix row
-              const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
-              sts_v2(pbuf + off, phi[0], phi[1]);
-              sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
-            }
+          } else {  // four rows: half of one 16-byte core-matrix row
+            const uint32_t off = kb + (row0 / 8) * 128 + (row0 % 8) * 2;
+            sts_v2(pbuf + off, phi[0], phi[1]);
+            sts_v2(pbuf + lo_off + off, plo[0], plo[1]);
           }
           fence_proxy_async_smem();
         }
         __syncwarp();
         if (ok && lane == 0) mbar_arrive(bar(BAR_PFULL + t % PB));
-      }
 
-      // The accumulated O^T once PV(end_t - 1) has finished: high + residual
-      // (PV(end_t - 2) was waited for before the last P went out).
-      float acc[RW];
+        if (flags & 2) {
+          // ---- the segment's partial: O once PV(t) has finished ------------
+          const SegInfo& si = seginfo[seg % kSegSlots];
+          float acc[RW];
 #pragma unroll
-      for (int r = 0; r < RW; ++r) acc[r] = 0.f;
-      if (end_t >= 1) ok = __all_sync(0xffffffffu, ok && wait_o_done(end_t - 1));
-      if (ok) {
-        tc_fence_after();
-        float oh[RW], ol[RW];
-        tmem_ld<RW>(o_hi, oh);
-        tmem_ld<RW>(o_lo, ol);
-        tmem_ld_wait();
+          for (int r = 0; r < RW; ++r) acc[r] = 0.f;
+          ok = __all_sync(0xffffffffu, ok && wait_o_done(t));
+          if (ok) {
+            tc_fence_after();
+            const uint32_t o_hi = tmem + lane_off + C::kTmemS + ob * C::kTmemO + row0;
+            float oh[RW], ol[RW];
+            tmem_ld<RW>(o_hi, oh);
+            tmem_ld<RW>(o_hi + NR, ol);
+            tmem_ld_wait();
 #pragma unroll
-        for (int r = 0; r < RW; ++r) acc[r] = oh[r] + ol[r];
-        tc_fence_before();
-      }
-
-      // Row sums: per-thread partials -> per-warp (lane r) -> across warps.
-      const float wl = warp_row_reduce<RW, false>(lpart, lane);
-      if (lane < RW) lsum[widx * 32 + lane] = wl;
-      __syncwarp();
-      named_bar_sync(bar_id, kSoftmaxThreads);
-      __syncthreads();  // (A): also makes the K producer's bad-block mark visible
-      const bool aborted = *abort != 0;
-      const bool bad = misc->bad != 0;
+            for (int r = 0; r < RW; ++r) acc[r] = oh[r] + ol[r];
+            tc_fence_before();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_OEMPTY + ob));  // the accumulator may be reused
+          // Row sums: per-thread partials -> per warp (lane r) -> across warps.
+          float lp[RW];
 #pragma unroll
-      for (int r = 0; r < RW; ++r) {
-        if (row0 + r < R) {
-          const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
-          const long long pr = part_base + row0 + r;
-          p.part_out[pr * kHeadDim + j] = (!aborted && !bad && l > 0.f) ? acc[r] / l : 0.f;
+          for (int r = 0; r < RW; ++r) lp[r] = lpart[r];
+          const float wsum = warp_row_reduce<RW, false>(lp, lane);
+          if (lane < RW) lsum[widx * 32 + lane] = wsum;
+          __syncwarp();
+          named_bar_sync(bar_id, kSoftmaxThreads);
+          const bool bad = si.bad != 0;
+          const long long pbase = (long long)si.slot * p.rows_half;
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            if (row0 + r < seg_rows) {
+              const float l = lsum[r] + lsum[32 + r] + lsum[64 + r] + lsum[96 + r];
+              p.part_out[(pbase + row0 + r) * kHeadDim + j] = (ok && !bad && l > 0.f) ? acc[r] / l : 0.f;
+            }
+          }
+          if (widx == 0 && lane < RW && row0 + lane < seg_rows) {
+            // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
+            // NaN marks a partial that must not be used (a stand-in block, a timeout).
+            const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
+            p.part_lse[pbase + row0 + lane] =
+                (bad || !ok) ? __uint_as_float(kInvalidLse)
+                : l > 0.f ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
+                          : -INFINITY;
+          }
+          __threadfence();  // the partial is visible before the group counts it in
+          named_bar_sync(bar_id, kSoftmaxThreads);
+          if (widx == 0 && lane == 0) {
+            if (arrive(p, si.group, si.expect, si.first && g == 0, 1)) {
+              const int i = atomicAdd(&misc->n_merge, 1);  // complete: merge it at the end
+              if (i < kMergeListLen) merge_list[i] = si.group;
+            }
+            misc->segs_done[g] = seg + 1;
+          }
         }
       }
-      if (widx == 0 && lane < RW && row0 + lane < R) {
-        // lse = ln sum_j e^{z_j}: log2 sum_j 2^{cs s_j} = log2 l' + cs m - kPShift.
-        // NaN marks a partial that read a stand-in for an out-of-range block.
-        const float l = lsum[lane] + lsum[32 + lane] + lsum[64 + lane] + lsum[96 + lane];
-        p.part_lse[part_base + row0 + lane] =
-            bad ? __int_as_float(0x7fc00000)
-            : (!aborted && l > 0.f)
-                ? (fmaf(cs, m_lane, -(float)C::kPShift) + log2f(l)) * 0.69314718055994531f
-                : -INFINITY;
-      }
+      __syncthreads();  // (A)
     }
     // ---- tear-down (every thread passed (A)) ---------------------------------
-    if (threadIdx.x == 32 && misc->abort) atomicOr(p.flags, kFlagTimeout);
     tc_fence_after();
     if (warp == 1) {
       __syncwarp();
@@ -1437,66 +1612,87 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     }
   }
 
-  // ---- arrival and merge --------------------------------------------------------
-  if (t_count == 0 && threadIdx.x == 0) misc->abort = 0;  // set by the K producer otherwise
+  // ---- unfinished segments, abort flag, merges ---------------------------------
   __syncthreads();  // (B) partials written, copies drained, TMEM freed
-  // Two counters per (sequence, KV head) group (cnt, above).  After (B), one
-  // thread counts the CTA in with release semantics, which publish the
-  // CTA's partials (the barrier ordered their stores before it).
-  if (p.coop) {
-    // Every CTA of the grid is resident: a barrier over the group's S CTAs,
-    // then each merges its share of the group.  The barrier needs no reset:
-    // the group's first CTA adds 2^31 - (S - 1) and the others 1, so the top
-    // bit of counter 0 flips once all S have arrived and its low bits return
-    // to their value (zero).  The arrival does not wait for a reply; the
-    // wait (acquire loads) is bounded.
+  if (threadIdx.x == 0) {
+    if (misc->abort) atomicOr(p.flags, kFlagTimeout);
+    // Segments published but not counted in by a softmax warpgroup (abort
+    // path): an invalid partial, counted in for that warpgroup.
+    for (int g = 0; g < NG; ++g) {
+      for (int sg = misc->segs_done[g]; sg < misc->segs_published; ++sg) {
+        const SegInfo& si = seginfo[sg % kSegSlots];
+        for (int r = 0; r < si.rows; ++r)
+          p.part_lse[(long long)si.slot * p.rows_half + r] = __uint_as_float(kInvalidLse);
+        __threadfence();
+        if (arrive(p, si.group, si.expect, si.first && g == 0, 1)) {
+          const int i = atomicAdd(&misc->n_merge, 1);
+          if (i < kMergeListLen) merge_list[i] = si.group;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (p.mode == 0) {
+    // The CTAs whose range ends in a KV head merge its partials, each a
+    // share, once all of the head's partials are in (a bounded wait on the
+    // group's barrier: every CTA of the grid is resident).
+    if (misc->own_group < 0) return;
     if (threadIdx.x == 0) {
-      const unsigned int add = split == 0 ? 0x80000000u - (unsigned int)(S - 1) : 1u;
-      red_release_add_gpu(cnt, add);
+      const int grp = (misc->own_s * Hkv + misc->own_group) * H + misc->own_h;
+      const int* cnt = group_counter(p, grp);
+      const unsigned phase = (unsigned)misc->own_phase;
       const unsigned long long t0 = globaltimer();
       int ok = 1;
-      while (((unsigned int)ld_acquire_gpu(cnt) & 0x80000000u) == bar_phase) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
+      while (((unsigned)ld_acquire_gpu(cnt) & 0x80000000u) == phase) {
+        if (globaltimer() - t0 > p.wait_limit_ns) {
           ok = 0;
           break;
         }
-        __nanosleep(20);
       }
       misc->last = ok;
+      if (!ok) atomicOr(p.flags, kFlagTimeout);
     }
     __syncthreads();
-    if (misc->last) {
-      merge_slice<RW, NG, Q8>(p, s, kvh, split, S, first, smem, sbase);
-    } else if (threadIdx.x == 0) {
-      atomicOr(p.flags, kFlagTimeout);
+    if (!misc->last) return;
+    const int P = misc->own_rows * (kHeadDim / 4);
+    const int sl = misc->own_slice, ns = misc->own_slices;
+    const int pa = (int)((long long)sl * P / ns), pb = (int)((long long)(sl + 1) * P / ns);
+    const long long slot0 = (long long)(misc->own_s * H + misc->own_h) * (p.ctas_per_set + Hkv) +
+                            misc->own_first + misc->own_group;
+    merge_pairs<kThreads>(p, slot0, misc->own_count, misc->own_rows, misc->own_s, misc->own_group,
+                          misc->own_h, pa, pb, smem, sbase, C::kRed);
+  } else {
+    // Groups this CTA completed: merge each, whole.
+    const int n = min(misc->n_merge, kMergeListLen);
+    if (n > 0) __threadfence();  // the other CTAs' partials, published before their counts
+    for (int i = 0; i < n; ++i) {
+      const int grp = merge_list[i];
+      const int h = grp % H, kvh = (grp / H) % Hkv, s = grp / (H * Hkv);
+      const int L = ld_nc_s32(p.context_lens + s);
+      int nb, ns;
+      seq_items(seq_vis(p, s, L).nch, p.item_tiles, nb, ns);
+      const int rows = part_rows(p, h);
+      merge_pairs<kThreads>(p, (long long)grp * p.slots_per_group, nb + ns, rows, s, kvh, h, 0,
+                            rows * (kHeadDim / 4), smem, sbase, C::kRed);
     }
-    return;
   }
-  // Otherwise the last CTA of the group to arrive (counter 1) merges all of
-  // it and sets the counter back to zero.
-  if (threadIdx.x == 0) {
-    __threadfence();
-    misc->last = (atomicAdd(cnt + 1, 1) == S - 1);
-  }
-  __syncthreads();
-  if (!misc->last) return;
-  __threadfence();  // the other CTAs' partials, published before their counts
-  merge_group<RW, NG, Q8>(p, s, kvh, S, first, smem, sbase);
-  if (threadIdx.x == 0) cnt[1] = 0;
 }
 
 // ---- host side ----------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* f = nullptr;
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        q == cudaDriverEntryPointSuccess) {
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      fn.store(f, std::memory_order_release);
+    }
   }
-  return fn;
+  return f;
 }
 
 // The fp16 cache viewed as a 4-D tensor {64 columns, 8 rows, 2 halves,
@@ -1516,37 +1712,43 @@ bool encode_cache_map(CUtensorMap* m, const void* cache, long long rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int RW, int NG, bool Q8>
-cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& mv,
-                      cudaStream_t stream) {
-  const size_t smem = Cfg<RW, NG, Q8>::kTotal + 1024;
-  static int resident[64] = {};  // CTAs of this kernel the device holds at once (0: unknown)
+constexpr int kMaxDevices = 64;
+
+template <int RW, int NG, int KV, bool TR>
+cudaError_t launch_cfg(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& mv,
+                       cudaStream_t stream) {
+  using Cf = Cfg<RW, NG, KV>;
+  auto kern = decode_tc_kernel<RW, NG, KV, TR>;
+  const size_t smem = Cf::kTotal + 1024;
+  // CTAs of this kernel the device holds at once (0: not yet known).
+  static std::atomic<int> resident[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || resident[dev] == 0) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<RW, NG, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int res = resident[dev].load(std::memory_order_acquire);
+  if (res == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_tc_kernel<RW, NG, Q8>, Cfg<RW, NG, Q8>::kThreads,
-                                                      smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cf::kThreads, smem);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) resident[dev] = per_sm * sms;
+    res = per_sm * sms;
+    if (res <= 0) return cudaErrorInvalidConfiguration;
+    resident[dev].store(res, std::memory_order_release);
   }
-  const long long ctas = p.num_ctas;
-  // A cooperative launch guarantees that every CTA is resident at once, which
-  // the group-wide merge waits rely on; larger grids merge in their last CTA.
-  p.coop = (dev >= 0 && dev < 64 && ctas <= resident[dev]) ? 1 : 0;
+  // Mode 0 waits on other CTAs: every CTA must be resident at once, which a
+  // cooperative launch guarantees; the plan never asks for more CTAs than
+  // the device holds.
+  if (p.num_ctas > res) return cudaErrorCooperativeLaunchTooLarge;
+  p.coop = p.mode == 0 ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.num_ctas);
-  cfg.blockDim = dim3(Cfg<RW, NG, Q8>::kThreads);
+  cfg.blockDim = dim3(Cf::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  // Programmatic stream serialization lets this grid's CTAs be scheduled
-  // while the previous kernel drains (they wait in griddepcontrol.wait).
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1554,36 +1756,37 @@ cudaError_t launch_rw(DecodeParams p, const CUtensorMap& mk, const CUtensorMap& 
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.coop ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<RW, NG, Q8>, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
 }
 
-}  // namespace
-
-bool decode_tc_supported(int kv_dtype, int rows, int num_blocks, int num_kv_heads, int block_size) {
-  // fp16: up to 32 rows per KV head; q8_0: up to 16 (the converted K and V
-  // tiles leave no shared memory for the 32-row P buffers).
-  const int max_rows = kv_dtype == kKvFp16 ? 2 * 16 : kv_dtype == kKvQ8_0 ? 16 : 0;
-  return rows >= 1 && rows <= max_rows && block_size % kChunk == 0 &&
-         (long long)num_blocks * num_kv_heads * block_size <= INT32_MAX;
-}
-
-cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream) {
-  if (p.kv_dtype == kKvQ8_0) {
-    // Raw q8_0 tiles arrive by untiled bulk copies: no tensor maps.
+template <bool TR>
+cudaError_t launch_any(const DecodeParams& p, cudaStream_t stream) {
+  if (p.kv_dtype != kKvFp16) {
+    // Raw int8 tiles arrive by untiled bulk copies: no tensor maps.
     CUtensorMap none;
     memset(&none, 0, sizeof(none));
-    if (p.rows <= 8) return launch_rw<4, 2, true>(p, none, none, stream);
-    return launch_rw<8, 2, true>(p, none, none, stream);
+    if (p.kv_dtype == kKvQ8_0) {
+      if (p.rows_half <= 8) return launch_cfg<4, 2, kKvQ8_0, TR>(p, none, none, stream);
+      return launch_cfg<8, 2, kKvQ8_0, TR>(p, none, none, stream);
+    }
+    if (p.rows_half <= 8) return launch_cfg<4, 2, kKvInt8Row, TR>(p, none, none, stream);
+    return launch_cfg<8, 2, kKvInt8Row, TR>(p, none, none, stream);
   }
   CUtensorMap mk, mv;
   const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
   if (!encode_cache_map(&mk, p.k, rows) || !encode_cache_map(&mv, p.v, rows))
     return cudaErrorInvalidValue;
-  // Two softmax warpgroups (measured: four groups of 8 rows at 32 rows are
-  // slower than two of 16).
-  if (p.rows <= 8) return launch_rw<4, 2, false>(p, mk, mv, stream);
-  if (p.rows <= 16) return launch_rw<8, 2, false>(p, mk, mv, stream);
-  return launch_rw<16, 2, false>(p, mk, mv, stream);
+  if (p.rows_half <= 8) return launch_cfg<4, 2, kKvFp16, TR>(p, mk, mv, stream);
+  if (p.rows_half <= 16) return launch_cfg<8, 2, kKvFp16, TR>(p, mk, mv, stream);
+  return launch_cfg<16, 2, kKvFp16, TR>(p, mk, mv, stream);
+}
+
+}  // namespace
+
+int max_rows_per_part(int kv_dtype) { return kv_dtype == kKvFp16 ? 32 : 16; }
+
+cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream) {
+  return p.trace != nullptr ? launch_any<true>(p, stream) : launch_any<false>(p, stream);
 }
 
 }  // namespace pa

@@ -11,20 +11,26 @@
 
 namespace pa {
 
-// Which kernel a call uses, and how the context is split.
+// How one call's work is cut (the work decomposition is described with
+// DecodeParams in common.cuh).
 struct Plan {
-  bool tensor_cores;
-  int splits, blocks_per_split;
-  int ctas;  // tensor-core kernel: CTAs of the grid (the device shares them out
-             // among the (sequence, KV head) groups); splits = ceil(ctas / groups)
-  int tiles_per_item;  // tensor-core kernel: 0, or the item size of a batched grid
+  int mode;             // 0: static partition (few groups), 1: work queue (a batch)
+  int halves;           // row parts per KV head
+  int rows_half;        // rows per part
+  int ctas;             // CTAs per launch
+  int ctas_per_set;     // mode 0: CTAs per (sequence, part)
+  int item_tiles;       // mode 1: 128-key tiles per big item
+  int slots_per_group;  // mode 1: partial slots per group
+  int launches;         // kernel launches of the call
+  long long slots;      // partial slots of the whole call
 };
 
-// Workspace: status header | arrival counters | split partial outputs |
-// split partial log-sum-exps.  Header and counters (the zero prefix) must be
-// zero before the first call; every call leaves the counters at zero.
+// Workspace: status header | arrival counters (two per group) | queue
+// counters (one per launch) | split partial outputs | split partial
+// log-sum-exps.  The header and the counters (the zero prefix) must be zero
+// before the first call; every call leaves the counters at zero.
 struct WsLayout {
-  size_t part_out, part_lse, total;
+  size_t arrivals, queue, part_out, part_lse, total;
 };
 
 int check_dims(const pa_dims* d, int n_query);
@@ -32,17 +38,31 @@ int check_decode_args(const void* q, const void* k, const void* v, const int32_t
                       const int32_t* cl, int causal, int window, float scale, int kv_dtype,
                       const void* out);
 Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms);
-// The largest plan any device can choose (sizes workspaces without a device).
-Plan max_plan(const pa_dims* d);
-WsLayout ws_layout(const pa_dims* d, int n_query, int splits);
 size_t ws_zero_prefix(const pa_dims* d);
+WsLayout ws_layout(const pa_dims* d, int n_query, const Plan& plan);
+// Bytes a workspace needs for any cache type on any device.
+size_t ws_size_any_device(const pa_dims* d, int n_query);
 int device_sm_count();
+// Wait limit of device-side pipeline waits for calls enqueued from now on.
+unsigned long long wait_limit_ns();
+unsigned long long set_wait_limit_ns(unsigned long long ns);
+
+// Partial mode (context-parallel decode): every pointer null, or the key
+// range of each sequence and the fp32 outputs (see DecodeParams).
+struct PartialArgs {
+  const int32_t* key_begin = nullptr;
+  const int32_t* key_count = nullptr;
+  float* out = nullptr;
+  float* out_lse = nullptr;
+};
 
 // Enqueue one decode with a prepared plan on `ws` (>= ws_layout(...).total
-// bytes, 256-byte aligned, zero prefix).  Returns a pa_status.
+// bytes, 256-byte aligned, zero prefix).  trace: null, or the key-resolution
+// record (set up by the caller).  Returns a pa_status.
 int enqueue_decode(const pa_dims* d, const Plan& plan, const void* q, const void* k_cache,
                    const void* v_cache, const int32_t* block_table, const int32_t* context_lens,
                    int n_query, int causal, int window, float scale, int kv_dtype, void* out,
-                   void* ws, cudaStream_t stream);
+                   void* ws, int32_t* trace, cudaStream_t stream,
+                   const PartialArgs& partial = PartialArgs());
 
 }  // namespace pa

@@ -7,20 +7,33 @@
 
 namespace pa {
 
-// Plain split-KV decode on CUDA cores (any block_size % 16 == 0, fp16/q8_0).
-size_t decode_simt_smem_bytes(int rows);
-cudaError_t launch_decode_simt(const DecodeParams& p, cudaStream_t stream);
-
-// Split-KV decode on the tensor cores (tcgen05/TMEM, TMA-staged fp16 tiles).
-// One CTA per SM; fp16 cache, rows = n_query * group <= 32.  Also merges the
-// split partials into p.out (the last CTA of each (sequence, KV head)).
-bool decode_tc_supported(int kv_dtype, int rows, int num_blocks, int num_kv_heads, int block_size);
+// Split-KV paged decode on the tensor cores (tcgen05/TMEM, TMA / bulk-copy
+// staged KV tiles), merge included: one launch per call (per kMaxQueueSeqs
+// sequences in work-queue mode).  Records the key-resolution trace when
+// p.trace is set.
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream);
+// Most query rows one CTA handles per KV head for a cache type.
+int max_rows_per_part(int kv_dtype);
 
 // Log-sum-exp merge of split partials into fp16 rows.
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
-// Per-row key-resolution record (debug / tests).
-cudaError_t launch_trace(const DecodeParams& p, int32_t* trace, cudaStream_t stream);
+// Key-resolution record: set every row to {0, INT32_MAX, -1, 0, 0} before
+// a traced decode, and rows no key reached to {0, -1, -1, 0, 0} after it.
+cudaError_t launch_trace_init(int32_t* trace, long long rows, cudaStream_t stream);
+cudaError_t launch_trace_finish(int32_t* trace, long long rows, cudaStream_t stream);
+
+// Quantise new keys/values and write them into the paged cache.
+struct CacheWriteParams {
+  const __half* k_new;         // [B][n_new][Hkv][D]
+  const __half* v_new;
+  void* k_cache;
+  void* v_cache;
+  const int32_t* block_table;  // [B][mbps]
+  const int32_t* context_lens; // [B]: the new tokens are the last n_new positions
+  int num_seqs, num_kv_heads, block_size, max_blocks_per_seq, num_blocks, n_new, kv_dtype;
+  unsigned* flags;             // data-error flags (a workspace status word)
+};
+cudaError_t launch_cache_write(const CacheWriteParams& p, cudaStream_t stream);
 
 }  // namespace pa

@@ -80,18 +80,20 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Returns false
-// (and sets *abort) once the time limit passes, or if another role already
+// (and sets *abort) once `limit_ns` has passed, or if another role already
 // gave up (*abort set): the caller then stops issuing work.  Between checks
 // the thread is suspended in try_wait (woken when the phase completes)
 // instead of spinning, so that waiting warps leave their issue slots to the
 // warps that compute.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
+  const uint32_t hint = limit_ns < 20000ull ? (uint32_t)limit_ns : 20000u;
   for (;;) {
-    if (mbar_try_wait_ns(bar, parity, 20000)) return true;
+    if (mbar_try_wait_ns(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
       return false;
     }

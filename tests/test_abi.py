@@ -58,7 +58,7 @@ def test_workspace_size_host_only(L):
     for bad in (dims(num_q_heads=30), dims(block_size=8), dims(head_dim=64), dims(num_seqs=0)):
         assert L.paged_attn_workspace_size(ctypes.byref(bad), 8) == 0
     assert L.paged_attn_workspace_size(ctypes.byref(d), 0) == 0
-    assert L.paged_attn_workspace_size(ctypes.byref(d), 9) == 0
+    assert L.paged_attn_workspace_size(ctypes.byref(d), 17) == 0
     assert L.paged_attn_workspace_size(None, 1) == 0
 
 
@@ -77,7 +77,7 @@ def test_decode_rejects_bad_arguments_on_host(L):
     assert call(None, args()) == b.PA_ERR_INVALID_ARG
     assert call(d, args(q=None)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(nq=0)) == b.PA_ERR_INVALID_ARG
-    assert call(d, args(nq=9)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(nq=17)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(causal=2)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(window=-1)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(dt=7)) == b.PA_ERR_INVALID_ARG
@@ -122,46 +122,47 @@ def _align(x):
     return (x + 255) & ~255
 
 
-def _plan_splits(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
-    """The splits paged_attn_decode plans on a device with `sms` SMs (the
-    planner in csrc/dispatch.cu, restated): the tensor-core kernel for up to
-    32 (fp16) or 16 (q8_0) rows per KV head, the CUDA-core kernel beyond."""
-    rows = nq * (Hq // Hkv)
-    groups = B * Hkv
-    if rows <= (32 if kv_dtype == 0 else 16):
-        max_split = _ceil(mbps * bs, 128)
-        if groups * 4 > sms:
-            T = max(16, _ceil(max_split * groups, 4 * sms))
-            return _ceil(max_split, T)
-        ctas = max(groups, min(sms, groups * max_split))
-        return _ceil(ctas, groups)
-    min_blocks = _ceil(128, bs)
-    max_splits = max(1, _ceil(mbps, min_blocks))
-    splits = max(1, min(_ceil(2 * sms, groups), max_splits))
-    bps = _ceil(mbps, splits)
-    return _ceil(mbps, bps)
+def _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
+    """(partial slots, rows per part) of the plan paged_attn_decode makes on
+    a device with `sms` SMs (the planner in csrc/dispatch.cu, restated): the
+    rows of a KV head in parts of at most 32 (fp16) or 16 (int8 caches);
+    few groups: an equal share of the SMs per (sequence, part), at least one
+    CTA per KV head, at most one per tile of a full table, plus one slot per
+    KV head; a batch: items of up to 16 tiles, the last cut into up to 4."""
+    R = nq * (Hq // Hkv)
+    H = _ceil(R, 32 if kv_dtype == 0 else 16)
+    RH = _ceil(R, H)
+    groups = B * Hkv * H
+    max_chunks = mbps * bs // 16
+    max_tiles = _ceil(max_chunks, 8)
+    if groups * 4 <= sms:
+        ch = max(Hkv, min(sms // (B * H), Hkv * max_tiles))
+        return B * H * (ch + Hkv), RH
+    T = min(16, max_tiles)
+    return groups * (_ceil(max_chunks, 8 * T) - 1 + 4), RH
 
 
-def _ws_needed(B, Hq, Hkv, nq, splits):
-    rows = B * splits * nq * Hq
-    prefix = 256 + _align(B * Hkv * 2 * 4)
-    return prefix + _align(rows * 128 * 4) + _align(rows * 4)
+def _ws_needed(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
+    slots, RH = _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms)
+    prefix = 256 + _align(B * Hkv * 4 * 2 * 4) + _align(_ceil(B, 256) * 4)
+    return prefix + _align(slots * RH * 128 * 4) + _align(slots * RH * 4)
 
 
 def test_workspace_size_covers_every_plan(L):
     """paged_attn_workspace_size needs no device, so it must cover the plan
-    of any device: every SM count up to 1024, both kernels, every block size
-    (a multiple of 16 up to 128; those that do not divide 128 let the
-    tensor-core kernel cut more splits than whole blocks would)."""
+    of any device and any cache type: every SM count up to 1024, every
+    block size (a multiple of 16 up to 128), row counts that need one, two,
+    three or four row parts."""
     import numpy as np
     rng = np.random.default_rng(7)
     shapes = [(1, 32, 8, 16, 3841, 8), (1, 32, 4, 16, 12288, 1), (8, 32, 8, 16, 4096, 4),
-              (1, 8, 1, 48, 100, 4), (1, 8, 1, 112, 100, 4), (64, 64, 8, 16, 4096, 8)]
+              (1, 8, 1, 48, 100, 4), (1, 8, 1, 112, 100, 4), (64, 64, 8, 16, 4096, 8),
+              (300, 32, 8, 16, 64, 16), (2, 48, 8, 16, 500, 8)]
     for _ in range(60):
         Hkv = int(rng.choice([1, 2, 4, 8]))
         shapes.append((int(rng.integers(1, 40)), Hkv * int(rng.choice([1, 2, 4, 8])), Hkv,
                        16 * int(rng.integers(1, 9)), int(rng.integers(1, 5000)),
-                       int(rng.integers(1, 9))))
+                       int(rng.integers(1, 17))))
     for B, Hq, Hkv, bs, mbps, nq in shapes:
         if nq * (Hq // Hkv) > 64:
             continue
@@ -169,10 +170,34 @@ def test_workspace_size_covers_every_plan(L):
                  max_blocks_per_seq=mbps, num_blocks=mbps * B + 1)
         have = L.paged_attn_workspace_size(ctypes.byref(d), nq)
         assert have > 0
-        for kv_dtype in (0, 1):
+        for kv_dtype in (0, 1, 2):
             for sms in list(range(1, 300)) + [512, 1024]:
-                need = _ws_needed(B, Hq, Hkv, nq, _plan_splits(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms))
+                need = _ws_needed(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms)
                 assert have >= need, (B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms, have, need)
+
+
+def test_wait_limit_setter(L):
+    """paged_attn_set_wait_limit returns the previous limit; 0 restores the
+    default of one second (host state only)."""
+    first = L.paged_attn_set_wait_limit(12345)
+    assert first == 10 ** 9
+    assert L.paged_attn_set_wait_limit(0) == 12345
+    assert L.paged_attn_set_wait_limit(0) == 10 ** 9
+
+
+def test_mode0_partition_formulas():
+    """The static partition's closed forms (csrc/decode_tc.cu: cta_holding,
+    cta_ending_from) against brute force over the CTA ranges
+    [k W / Ce, (k+1) W / Ce): the CTA holding each chunk, the first CTA whose
+    range ends at or after each chunk."""
+    for W in range(1, 80):
+        for Ce in range(1, min(W, 30) + 1):
+            b = [k * W // Ce for k in range(Ce + 1)]
+            for x in range(W):
+                k = next(k for k in range(Ce) if b[k] <= x < b[k + 1])
+                assert ((x + 1) * Ce - 1) // W == k
+                first_end = next(k for k in range(Ce) if b[k + 1] - 1 >= x)
+                assert ((x + 1) * Ce + W - 1) // W - 1 == first_end
 
 
 def test_binding_refuses_tensors_the_kernel_would_read_out_of_bounds():
