@@ -104,20 +104,25 @@ enum : int {
   BAR_VFULL = 6,     // [3] V chunks landed (int8: in a raw slot)
   BAR_VEMPTY = 9,    // [3] V slot free again
   BAR_CKFULL = 12,   // [3] int8: K slot converted
-  BAR_CVFULL = 15,   // int8: converted V (hi | lo) ready
-  BAR_CVEMPTY = 16,  // int8: converted V read by PV
-  BAR_SFULL = 17,    // [2] S^T in TMEM
-  BAR_SEMPTY = 19,   // [2] S^T read by the softmax
-  BAR_PFULL = 21,    // [2] P of a tile in shared memory
-  BAR_OFULL = 23,    // PV of one more tile accumulated
-  BAR_OEMPTY = 24,   // [2] a segment's O accumulator read out
-  BAR_QFULL = 26,    // [2] a segment's Q staged
-  BAR_QEMPTY = 28,   // [2] Q buffer free
-  BAR_DONE = 30,     // every MMA finished
-  BAR_INFO = 31,     // [8] a tile's description published
-  BAR_COUNT = 39
+  BAR_CVFULL = 15,   // [3] int8: a converted half-tile of V (hi | lo) ready
+  BAR_CVEMPTY = 18,  // [3] int8: a converted half-tile read by PV
+  BAR_SFULL = 21,    // [2] S^T in TMEM
+  BAR_SEMPTY = 23,   // [2] S^T read by the softmax
+  BAR_PFULL = 25,    // [2] P of a tile in shared memory
+  BAR_OFULL = 27,    // PV of one more tile accumulated
+  BAR_OEMPTY = 28,   // [2] a segment's O accumulator read out
+  BAR_QFULL = 30,    // [2] a segment's Q staged
+  BAR_QEMPTY = 32,   // [2] Q buffer free
+  BAR_DONE = 34,     // every MMA finished
+  BAR_INFO = 35,     // [8] a tile's description published
+  BAR_COUNT = 43
 };
-constexpr int kBarSlots = 40;
+constexpr int kBarSlots = 44;
+// int8: converted V lives in a ring of three half-tile slots (64 keys: the hi
+// tile, then the lo tile), so that the converters run ahead of PV.
+constexpr int kVCSlots = 3;
+constexpr uint32_t kVCSlot = kKVBytes;           // 64 keys x (hi + lo)
+constexpr uint32_t kVCLo = kKVBytes / 2;         // offset of the lo half-tile
 
 // A tile as the K producer publishes it.
 struct TileInfo {
@@ -143,6 +148,11 @@ struct SegInfo {
   int pad[6];
 };
 static_assert(sizeof(SegInfo) == 64, "SegInfo layout");
+
+// Finished partials a softmax warpgroup has yet to count in (group, expected
+// arrivals, designated first): counted in at the end of its loop, or when
+// the list is full.
+constexpr int kPendLen = 8;
 
 struct Misc {
   uint32_t tmem_base;
@@ -173,15 +183,15 @@ struct Cfg {
   static constexpr int NR = (NG * RW < 16) ? 16 : NG * RW;  // MMA N of QK^T
   static constexpr int kSG = kQ8 ? kHeadDim / 32 : 1;      // S^T accumulators per tile
   static constexpr int KS = kQuant ? 2 : 3;
-  static constexpr int VS = kQuant ? 3 : (NR > 16 ? 2 : 3);
+  static constexpr int VS = kQuant ? 2 : (NR > 16 ? 2 : 3);
   static constexpr uint32_t kKSlot = kKVBytes;
-  // int8: raw V slots (16 KB of qs, then the tile's scales); the converted V
-  // (hi tile | lo tile) has one slot of its own.
+  // int8: raw V slots (16 KB of qs, then the tile's scales) feeding a ring of
+  // kVCSlots converted half-tiles.
   static constexpr uint32_t kVSlot = kQuant ? kRawScales + 1024 : kKVBytes;
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = KS * kKSlot;
   static constexpr uint32_t kVC = kV + VS * kVSlot;
-  static constexpr uint32_t kVCBytes = kQuant ? 2 * kKVBytes : 0;
+  static constexpr uint32_t kVCBytes = kQuant ? kVCSlots * kVCSlot : 0;
   static constexpr uint32_t kQ = kVC + kVCBytes;
   static constexpr uint32_t kQHalf = NR * 128;       // one 64-column half of Q
   static constexpr uint32_t kQBuf = 2 * kQHalf;      // Q of one segment
@@ -197,7 +207,8 @@ struct Cfg {
   static constexpr uint32_t kMisc = kSeg + kSegSlots * sizeof(SegInfo);
   static constexpr uint32_t kQueueArr = kMisc + 128;   // mode 1: int [3][kMaxQueueSeqs + 1]
   static constexpr uint32_t kMergeList = kQueueArr + 3 * (kMaxQueueSeqs + 1) * 4;
-  static constexpr uint32_t kTotal = kMergeList + kMergeListLen * 4;
+  static constexpr uint32_t kPend = kMergeList + kMergeListLen * 4;  // int [NG][kPendLen][3]
+  static constexpr uint32_t kTotal = kPend + NG * kPendLen * 3 * 4;
   // TMEM: S^T[2] (kSG accumulators of NR columns), then O^T[2] (2 NR: the
   // high parts' products, then the residuals').
   static constexpr uint32_t kTmemS = 2 * kSG * NR;
@@ -217,13 +228,6 @@ struct Cfg {
 __device__ __forceinline__ int ld_nc_s32(const int* p) {
   int r;
   asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
   return r;
 }
 __device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
@@ -348,13 +352,20 @@ __device__ __forceinline__ void part_range(const DecodeParams& p, int L, int h, 
   lo = min(lo0, lo1);
   hi = max(hi0, hi1);
 }
+// a / b for a >= 0, b > 0, with 32-bit division when both fit (the usual
+// case: far cheaper than the 64-bit sequence).
+__device__ __forceinline__ long long div64(long long a, long long b) {
+  if (((unsigned long long)a | (unsigned long long)b) <= 0xffffffffull)
+    return (long long)((unsigned)a / (unsigned)b);
+  return a / b;
+}
 // Mode 0: the CTA of Ce whose chunk range [k W / Ce, (k+1) W / Ce) holds
 // chunk x, and the first CTA whose range ends at or after chunk y.
 __device__ __forceinline__ int cta_holding(long long x, int Ce, long long W) {
-  return (int)(((x + 1) * Ce - 1) / W);
+  return (int)div64((x + 1) * Ce - 1, W);
 }
 __device__ __forceinline__ int cta_ending_from(long long y, int Ce, long long W) {
-  return (int)(((y + 1) * Ce + W - 1) / W) - 1;
+  return (int)div64((y + 1) * Ce + W - 1, W) - 1;
 }
 // Mode 1: a group's chunks are items of 8T chunks, the last of which is cut
 // into up to four sub-items (processed after every big item).
@@ -581,15 +592,15 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         // int8 raw V slots are freed by the converter warps, fp16 ones by a commit
         mbar_init(bar(BAR_VEMPTY + i), kQuant ? C::kConvWarps : 1);
         mbar_init(bar(BAR_CKFULL + i), C::kConvWarps);
+        mbar_init(bar(BAR_CVFULL + i), C::kConvWarps);
+        mbar_init(bar(BAR_CVEMPTY + i), 1);
       }
-      mbar_init(bar(BAR_CVFULL), C::kConvWarps);
-      mbar_init(bar(BAR_CVEMPTY), 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(bar(BAR_SFULL + i), 1);
         mbar_init(bar(BAR_SEMPTY + i), 4 * NG);
         mbar_init(bar(BAR_PFULL + i), 4 * NG);
         mbar_init(bar(BAR_OEMPTY + i), 4 * NG);
-        mbar_init(bar(BAR_QFULL + i), 1);
+        mbar_init(bar(BAR_QFULL + i), 32);  // one per lane of the K producer
         mbar_init(bar(BAR_QEMPTY + i), 1);
       }
       mbar_init(bar(BAR_OFULL), 1);
@@ -608,6 +619,8 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
 
     const int c = lane;  // lane c < 8 owns chunk c of every tile
     const int cta = blockIdx.x, Cgrid = gridDim.x;
+    // The cache is streamed once: its lines go first when L2 needs room.
+    const uint64_t pol = l2_evict_first_policy();
     int* qarr = reinterpret_cast<int*>(smem + C::kQueueArr);  // mode 1: Ls, P1, P2
     int* Ls = qarr;
     int* P1 = Ls + (kMaxQueueSeqs + 1);
@@ -617,15 +630,37 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     int next_q = 0;  // mode 1: the next item index, taken one segment ahead
 
     // -- mode 0: this CTA's chunk range of its (sequence, part) set ---------
+    constexpr long long kNone = -(1LL << 40);
     int m0_s = 0, m0_h = 0, m0_k = 0, m0_L = 0, m0_Ce = 0, m0_nseg = 0, m0_next = 0;
-    SeqVis m0_v{0, -1, 0, 0};
+    SeqVis m0_v{0, -1, 0, 0, 0, false};
     long long m0_a = 0, m0_b = 0, m0_W = 0;
+    int own_g = -1, own_phase_raw = 0;
+    // Speculation (mode 0, no window, every key of the context): the range
+    // this CTA gets if the sequence fills its whole table, whose first
+    // tile's table entries are read while the context length is in flight;
+    // they are used when the real range starts at the same chunk.
+    long long spec_raw = kNone;
+    int spec_kvh = -1, spec_c0 = -1;
     if (p.mode == 0) {
       const int sigma = cta / p.ctas_per_set;
       m0_k = cta % p.ctas_per_set;
       m0_s = sigma / H;
       m0_h = sigma % H;
       m0_L = ld_nc_s32(p.context_lens + m0_s);
+      if (p.window == 0 && p.key_begin == nullptr) {
+        const long long nch_s = (long long)p.max_blocks_per_seq * p.block_size / kChunk;
+        const long long Ws = (long long)Hkv * nch_s;
+        const int Ces = (int)(Ws < (long long)p.ctas_per_set ? Ws : (long long)p.ctas_per_set);
+        if (m0_k < Ces) {
+          const long long a = div64((long long)m0_k * Ws, Ces);
+          spec_kvh = (int)div64(a, nch_s);
+          spec_c0 = (int)(a - (long long)spec_kvh * nch_s);
+          const long long ch = spec_c0 + c;
+          if (c < kChunksPerTile && ch < nch_s)
+            spec_raw = ld_nc_s32(p.block_table + (long long)m0_s * p.max_blocks_per_seq +
+                                 ch * kChunk / p.block_size);
+        }
+      }
       m0_v = seq_vis(p, m0_s, m0_L);
       m0_W = (long long)Hkv * m0_v.nch;
       m0_Ce = (int)(m0_W < (long long)p.ctas_per_set ? m0_W : (long long)p.ctas_per_set);
@@ -637,33 +672,19 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
           if (lane == 0 && m0_h == 0 && m0_v.bad) atomicOr(p.flags, kFlagBadLen);
         }
       } else if (m0_k < m0_Ce) {
-        m0_a = (long long)m0_k * m0_W / m0_Ce;
-        m0_b = (long long)(m0_k + 1) * m0_W / m0_Ce;
-        const int kvh0 = (int)(m0_a / m0_v.nch);
+        m0_a = div64((long long)m0_k * m0_W, m0_Ce);
+        m0_b = div64((long long)(m0_k + 1) * m0_W, m0_Ce);
+        const int kvh0 = (int)div64(m0_a, m0_v.nch);
         m0_nseg = (m0_b > (long long)(kvh0 + 1) * m0_v.nch) ? 2 : 1;
         // Merge duty: the KV head of this CTA's last chunk, shared with the
-        // other CTAs whose range ends in it.
-        const int g = (int)((m0_b - 1) / m0_v.nch);
-        const long long g0 = (long long)g * m0_v.nch;
-        const int ko_lo = cta_ending_from(g0, m0_Ce, m0_W);
-        const int ko_hi =
-            g + 1 < Hkv ? cta_ending_from(g0 + m0_v.nch, m0_Ce, m0_W) - 1 : m0_Ce - 1;
-        const int kf = cta_holding(g0, m0_Ce, m0_W);
-        const int kl = cta_holding(g0 + m0_v.nch - 1, m0_Ce, m0_W);
-        if (lane == 0) {
-          const int grp = (m0_s * Hkv + g) * H + m0_h;
-          misc->own_phase = (int)((unsigned)ld_acquire_gpu(group_counter(p, grp)) & 0x80000000u);
-          misc->own_group = g;
-          misc->own_first = kf;
-          misc->own_count = kl - kf + 1;
-          misc->own_slice = m0_k - ko_lo;
-          misc->own_slices = ko_hi - ko_lo + 1;
-          misc->own_s = m0_s;
-          misc->own_h = m0_h;
-          misc->own_rows = part_rows(p, m0_h);
-        }
+        // other CTAs whose range ends in it.  Its barrier phase is read now,
+        // before this CTA can arrive (relaxed: the load stays in flight).
+        own_g = (int)div64(m0_b - 1, m0_v.nch);
+        if (lane == 0)
+          own_phase_raw = ld_relaxed_gpu(group_counter(p, (m0_s * Hkv + own_g) * H + m0_h));
       }
     } else {
+      // -- mode 1: per-sequence item counts and their prefix sums ----------    } else {
       // -- mode 1: per-sequence item counts and their prefix sums ----------
       const int GH = Hkv * H;
       int run1 = 0, run2 = 0;
@@ -708,7 +729,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     auto next_segment = [&](SegDesc& d) -> bool {
       if (p.mode == 0) {
         if (m0_next >= m0_nseg) return false;
-        d.kvh = (int)(m0_a / m0_v.nch) + m0_next;
+        d.kvh = (int)div64(m0_a, m0_v.nch) + m0_next;
         const long long g0 = (long long)d.kvh * m0_v.nch;
         d.c0 = (int)max(0LL, m0_a - g0);
         d.c1 = (int)min((long long)m0_v.nch, m0_b - g0);
@@ -785,40 +806,29 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       return true;
     };
 
-    // Q rows of a segment -> registers (lane-strided 16-byte pieces), later
-    // -> shared memory, K-major with the 128-byte swizzle: row n, piece cc of
-    // half cc / 8 at half * kQHalf + n * 128 + ((cc % 8) ^ (n % 8)) * 16.
-    // Rows past the part's valid rows are zero.  A negative scale is moved
-    // into Q (an exact sign flip), so scores are only multiplied by cs >= 0.
+    // Q rows of a segment -> shared memory by asynchronous 16-byte copies
+    // (lane-strided pieces), K-major with the 128-byte swizzle: row n, piece
+    // cc of half cc / 8 at half * kQHalf + n * 128 + ((cc % 8) ^ (n % 8)) * 16.
+    // Rows past the part's valid rows are zero-filled.  Each lane's copies
+    // count one arrival on QFULL when they have landed; the MMA issuer makes
+    // them visible to the tensor cores with a proxy fence.
     constexpr int kQPer = NR * 16 / 32;  // 16-byte pieces per lane
-    uint4 qreg[kQPer];
-    const uint32_t flip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-    auto load_q = [&](const SegDesc& d) {
+    auto stage_q = [&](const SegDesc& d, int qb) {
       const int rows = part_rows(p, d.h);
-#pragma unroll
-      for (int k = 0; k < kQPer; ++k) {
-        const int e = k * 32 + lane, n = e / 16, cc = e % 16;
-        qreg[k] = make_uint4(0, 0, 0, 0);
-        if (n < rows) qreg[k] = ldg_nc_v4(p.q + out_row(p, d.s, d.kvh, d.h, n) * kHeadDim + cc * 8);
-      }
-    };
-    auto store_q = [&](int qb) {
       const uint32_t dst = sQ + qb * C::kQBuf;
 #pragma unroll
       for (int k = 0; k < kQPer; ++k) {
         const int e = k * 32 + lane, n = e / 16, cc = e % 16;
-        uint4 v = qreg[k];
-        v.x ^= flip; v.y ^= flip; v.z ^= flip; v.w ^= flip;
-        sts_v4(dst + (cc / 8) * C::kQHalf + n * 128 + (((cc % 8) ^ (n & 7)) * 16), v);
+        const bool in = n < rows;
+        const __half* src = in ? p.q + out_row(p, d.s, d.kvh, d.h, n) * kHeadDim + cc * 8 : p.q;
+        cp_async_16_zfill(dst + (cc / 8) * C::kQHalf + n * 128 + (((cc % 8) ^ (n & 7)) * 16), src,
+                          in ? 16u : 0u);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_QFULL + qb));
+      cp_async_mbar_arrive_noinc(bar(BAR_QFULL + qb));
     };
 
     // Block-table entry of chunk c of the tile that starts at chunk tc0
     // (kNone: not copied).
-    constexpr long long kNone = -(1LL << 40);
     auto lookup = [&](const SegDesc& d, int tc0) -> long long {
       const int ci = tc0 + c;
       if (c >= kChunksPerTile || ci >= d.c1) return kNone;
@@ -854,10 +864,24 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     };
 
     int t = 0, seg_n = 0, seg_written = 0;
-    SegDesc cur{};
+    SegDesc cur{}, nxt{};
     bool have = next_segment(cur);
-    if (have) load_q(cur);
-    long long raw_cur = have ? lookup(cur, cur.c0) : kNone;
+    // The segment after the current one is taken at the current one's first
+    // tile, so that its first block-table entries are in flight for a whole
+    // segment (a load issued behind the stream takes microseconds).
+    bool have_nxt = false, planned = false;
+    long long raw_first_nxt = kNone;
+    long long raw_cur = kNone;
+    if (have) {
+      if (cur.kvh == spec_kvh && cur.c0 == spec_c0 && cur.base == 0) {
+        // the speculated entries, for the chunks the real range keeps
+        const int ci = cur.c0 + c, key0 = cur.base + ci * kChunk;
+        raw_cur = (c < kChunksPerTile && ci < cur.c1 && key0 <= cur.vis_hi &&
+                   key0 + kChunk - 1 >= cur.vis_lo) ? spec_raw : kNone;
+      } else {
+        raw_cur = lookup(cur, cur.c0);
+      }
+    }
     bool ok = true;
     while (have && ok) {
       const int segslot = seg_n % kSegSlots, qb = seg_n % 2;
@@ -875,8 +899,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       if (lane == 0) w = wait(BAR_QEMPTY + qb, ((seg_n / 2) & 1) ^ 1);
       ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       if (!ok) break;
+      stage_q(cur, qb);
       const int ntile = (cur.c1 - cur.c0 + kChunksPerTile - 1) / kChunksPerTile;
-      SegDesc nxt{};
+      planned = false;
       for (int tau = 0; tau < ntile; ++tau) {
         const int tc0 = cur.c0 + tau * kChunksPerTile;
         const int row_cur = to_row8(raw_cur, cur, tc0, segslot);
@@ -912,30 +937,32 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
                                    (long long)slot0 * kScaleBytes;
             const uint8_t* kc = static_cast<const uint8_t*>(p.k);
             const uint8_t* vc = static_cast<const uint8_t*>(p.v);
-            bulk_load(sK + st * C::kKSlot + kRawOff + c * kQsChunk, kc + off, kQsChunk, fb);
-            bulk_prefetch_l2(kc + soff, kChunk * kScaleBytes);  // K scales: the softmax reads them
-            bulk_prefetch_l2(vc + off, kQsChunk);
-            bulk_prefetch_l2(vc + soff, kChunk * kScaleBytes);
+            bulk_load_hint(sK + st * C::kKSlot + kRawOff + c * kQsChunk, kc + off, kQsChunk, fb, pol);
+            // K scales (the softmax reads them) and the V tile, into L2
+            bulk_prefetch_l2_hint(kc + soff, kChunk * kScaleBytes, pol);
+            bulk_prefetch_l2_hint(vc + off, kQsChunk, pol);
+            bulk_prefetch_l2_hint(vc + soff, kChunk * kScaleBytes, pol);
           } else {
-            tma_load_4d(sK + st * C::kKSlot + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb);
-            tma_prefetch_4d(&tmap_v, 0, 0, 0, row_cur);
+            tma_load_4d_hint(sK + st * C::kKSlot + c * kChunkBytes, &tmap_k, 0, 0, 0, row_cur, fb, pol);
+            tma_prefetch_4d_hint(&tmap_v, 0, 0, 0, row_cur, pol);
           }
         }
         __syncwarp();
-        if (tau == 0) store_q(qb);
+        if (tau == 0) {
+          have_nxt = next_segment(nxt);
+          planned = true;
+          if (have_nxt) raw_first_nxt = lookup(nxt, nxt.c0);
+        }
         ++t;
         if (!more) {
-          // Next segment: its descriptor, Q rows and first block-table entries.
           ++seg_n;
-          have = next_segment(nxt);
-          if (have) {
-            load_q(nxt);
-            raw_nxt = lookup(nxt, nxt.c0);
-          }
+          raw_nxt = raw_first_nxt;
         }
         raw_cur = raw_nxt;
       }
+      if (!ok) break;
       cur = nxt;
+      have = have_nxt;
     }
     if (ok) {  // end of the stream
       if (lane == 0) {
@@ -946,11 +973,35 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       }
     } else {
       // Abort: count in every segment this CTA owns but did not publish, and
-      // (mode 1) take the remaining items off the queue the same way.
-      SegDesc d{};
-      while (next_segment(d)) give_up(d);
+      // (mode 1) take the remaining items off the queue the same way (the
+      // queue is taken from until it first reports its end, never after).
+      if (planned && have_nxt) give_up(nxt);
+      if (!planned || have_nxt) {
+        SegDesc d{};
+        while (next_segment(d)) give_up(d);
+      }
     }
+    cp_async_wait_all();  // no Q copy outlives the producer
     if (lane == 0) misc->segs_published = seg_written;
+    if (own_g >= 0 && lane == 0) {
+      // mode 0 merge duty (see above): the KV head's partials are CTAs
+      // [kf, kl] of the set, its owners [ko_lo, ko_hi]
+      const long long g0 = (long long)own_g * m0_v.nch;
+      const int ko_lo = cta_ending_from(g0, m0_Ce, m0_W);
+      const int ko_hi =
+          own_g + 1 < Hkv ? cta_ending_from(g0 + m0_v.nch, m0_Ce, m0_W) - 1 : m0_Ce - 1;
+      const int kf = cta_holding(g0, m0_Ce, m0_W);
+      const int kl = cta_holding(g0 + m0_v.nch - 1, m0_Ce, m0_W);
+      misc->own_phase = (int)((unsigned)own_phase_raw & 0x80000000u);
+      misc->own_group = own_g;
+      misc->own_first = kf;
+      misc->own_count = kl - kf + 1;
+      misc->own_slice = m0_k - ko_lo;
+      misc->own_slices = ko_hi - ko_lo + 1;
+      misc->own_s = m0_s;
+      misc->own_h = m0_h;
+      misc->own_rows = part_rows(p, m0_h);
+    }
     __syncwarp();
     __syncthreads();  // (A) every role finished its loop
     if (lane == 0) {  // drain copies that no consumer waited for (abort path only)
@@ -978,6 +1029,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     if (warp == kVWarp) {
       // ===================== V producer ======================================
       const int c = lane;
+      const uint64_t pol = l2_evict_first_policy();
       int issued = 0;
       for (int t = 0;; ++t) {
         int w = 1;
@@ -1005,12 +1057,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
             const int slot0 = key0 % p.block_size;
             const uint8_t* src = static_cast<const uint8_t*>(p.v) + (long long)row8 * tb;
             const uint32_t dst = sV + st * C::kVSlot;
-            bulk_load(dst + c * kQsChunk, src + (long long)slot0 * kHeadDim, kQsChunk, fb);
-            bulk_load(dst + kRawScales + c * (kChunk * kScaleBytes),
-                      src + (long long)p.block_size * kHeadDim + (long long)slot0 * kScaleBytes,
-                      kChunk * kScaleBytes, fb);
+            bulk_load_hint(dst + c * kQsChunk, src + (long long)slot0 * kHeadDim, kQsChunk, fb, pol);
+            bulk_load_hint(dst + kRawScales + c * (kChunk * kScaleBytes),
+                           src + (long long)p.block_size * kHeadDim + (long long)slot0 * kScaleBytes,
+                           kChunk * kScaleBytes, fb, pol);
           } else {
-            tma_load_4d(sV + st * C::kVSlot + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb);
+            tma_load_4d_hint(sV + st * C::kVSlot + c * kChunkBytes, &tmap_v, 0, 0, 0, row8, fb, pol);
           }
         }
         __syncwarp();
@@ -1042,7 +1094,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
           const TileInfo& ti = info[u % kInfoSlots];
           const int seg = ti.seg, flags = ti.flags;
           if (seg < 0) return 1;
-          if ((flags & 1) && !wait(BAR_QFULL + seg % 2, (seg / 2) & 1)) return -1;
+          if (flags & 1) {
+            if (!wait(BAR_QFULL + seg % 2, (seg / 2) & 1)) return -1;
+            fence_proxy_async_smem();  // Q arrived by cp.async (generic proxy)
+          }
           if (!wait((kQuant ? BAR_CKFULL : BAR_KFULL) + u % KS, (u / KS) & 1)) return -1;
           if (!wait(BAR_SEMPTY + u % 2, ((u / 2) & 1) ^ 1)) return -1;
           tc_fence_after();
@@ -1075,23 +1130,46 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
           const TileInfo& ti = info[t % kInfoSlots];  // described before QK(t)
           const int seg = ti.seg, flags = ti.flags, ob = seg % 2;
           ok = wait(BAR_PFULL + t % PB, (t / PB) & 1) &&
-               (kQuant ? wait(BAR_CVFULL, t & 1) : wait(BAR_VFULL + t % VS, (t / VS) & 1)) &&
+               (kQuant || wait(BAR_VFULL + t % VS, (t / VS) & 1)) &&
                (!(flags & 1) || wait(BAR_OEMPTY + ob, ((seg / 2) & 1) ^ 1));
           if (!ok) break;
           tc_fence_after();
-          const uint64_t so = kQuant ? 0 : (uint64_t)((t % VS) * C::kVSlot) >> 4;
           const uint64_t pb = (uint64_t)((t % PB) * C::kPBytes) >> 4;
           const uint32_t d = tmem + C::kTmemS + ob * C::kTmemO;
+          if constexpr (kQuant) {
+            // Two half-tiles of 64 keys, each from its converted slot:
+            // V_hi [P_hi | P_lo], then V_lo times the high parts of P (the
+            // first NR columns).
 #pragma unroll
-          for (int k = 0; k < kTileKeys / 16; ++k) {
-            const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
-            const uint64_t po = (k * 2 * C::kPN * 16) >> 4;
-            tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, !(flags & 1) || k > 0);
-            if constexpr (kQuant)  // V_lo times the high parts of P (the first NR columns)
-              tc_mma_f16_ss(d, dV + (kKVBytes >> 4) + vo, dP + pb + po, id_pv_lo, 1);
+            for (int hf = 0; hf < 2; ++hf) {
+              const int hx = 2 * t + hf;
+              if (!wait(BAR_CVFULL + hx % kVCSlots, (hx / kVCSlots) & 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t so = (uint32_t)(hx % kVCSlots) * kVCSlot;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t vo = (so + k * 2 * kGroupBytes) >> 4;
+                const uint64_t po = ((hf * 4 + k) * 2 * C::kPN * 16) >> 4;
+                tc_mma_f16_ss(d, dV + vo, dP + pb + po, id_pv, !(flags & 1) || hf > 0 || k > 0);
+                tc_mma_f16_ss(d, dV + vo + (kVCLo >> 4), dP + pb + po, id_pv_lo, 1);
+              }
+              tc_commit(bar(BAR_CVEMPTY + hx % kVCSlots));
+            }
+            if (!ok) break;
+          } else {
+            const uint64_t so = (uint64_t)((t % VS) * C::kVSlot) >> 4;
+#pragma unroll
+            for (int k = 0; k < kTileKeys / 16; ++k) {
+              const uint64_t vo = (k * 2 * kGroupBytes) >> 4;
+              const uint64_t po = (k * 2 * C::kPN * 16) >> 4;
+              tc_mma_f16_ss(d, dV + so + vo, dP + pb + po, id_pv, !(flags & 1) || k > 0);
+            }
+            tc_commit(bar(BAR_VEMPTY + t % VS));
           }
           tc_commit(bar(BAR_OFULL));
-          tc_commit(bar(kQuant ? BAR_CVEMPTY : BAR_VEMPTY + t % VS));
           npv = t + 1;
           if (t_end == 0x7fffffff) {
             const int r = issue_qk(t + 2);
@@ -1145,15 +1223,22 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         live = live && ti.seg >= 0;
         const int rs = t % NSl;
         if (live) live = wait((kv == 0 ? BAR_KFULL : BAR_VFULL) + rs, (t / NSl) & 1);
-        if (live && kv == 1) live = wait(BAR_CVEMPTY, (t & 1) ^ 1);
         if (!named_bar_and(kBarConv0 + kv, kCT, __all_sync(0xffffffffu, live))) break;
         const int key_t = ti.key0, vlo = ti.vis_lo, vhi = ti.vis_hi;
         if (kv == 1) {
-          const uint32_t slot = sV + rs * C::kVSlot;
-          const uint32_t src = slot + r0 * kHeadDim + c16 * 16;
+         const uint32_t slot = sV + rs * C::kVSlot;
+         bool vok = true;
+#pragma unroll 1
+         for (int hf = 0; hf < 2; ++hf) {
+          // half-tile hx = keys 64 hf .. 64 hf + 63 of tile t, into converted
+          // slot hx % kVCSlots once PV has read that slot's previous half-tile
+          const int hx = 2 * t + hf;
+          vok = __all_sync(0xffffffffu, vok && wait(BAR_CVEMPTY + hx % kVCSlots, ((hx / kVCSlots) & 1) ^ 1));
+          const uint32_t dslot = sVC + (uint32_t)(hx % kVCSlots) * kVCSlot;
+          const uint32_t src = slot + (hf * 64 + r0) * kHeadDim + c16 * 16;
 #pragma unroll 2
-          for (int k = 0; k < kKeysPer; ++k) {
-            const int r = k * kRS + r0;
+          for (int k = 0; k < kKeysPer / 2; ++k) {
+            const int r = hf * 64 + k * kRS + r0;
             const uint4 qv = lds_v4(src + k * kRS * kHeadDim);
             uint32_t hi[8], lo[8];
 #pragma unroll
@@ -1192,17 +1277,19 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
               }
             }
             const uint32_t g8 = k * (kRS / 8) * kGroupBytes;
-            sts_v4(sVC + g8 + dst_a, make_uint4(hi[0], hi[1], hi[2], hi[3]));
-            sts_v4(sVC + g8 + dst_b, make_uint4(hi[4], hi[5], hi[6], hi[7]));
-            sts_v4(sVC + kKVBytes + g8 + dst_a, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-            sts_v4(sVC + kKVBytes + g8 + dst_b, make_uint4(lo[4], lo[5], lo[6], lo[7]));
+            if (vok) {
+              sts_v4(dslot + g8 + dst_a, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+              sts_v4(dslot + g8 + dst_b, make_uint4(hi[4], hi[5], hi[6], hi[7]));
+              sts_v4(dslot + kVCLo + g8 + dst_a, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+              sts_v4(dslot + kVCLo + g8 + dst_b, make_uint4(lo[4], lo[5], lo[6], lo[7]));
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(bar(BAR_CVFULL));
-            mbar_arrive(bar(BAR_VEMPTY + rs));  // the raw slot may be refilled
-          }
+          if (lane == 0 && vok) mbar_arrive(bar(BAR_CVFULL + hx % kVCSlots));
+         }
+         __syncwarp();
+         if (lane == 0) mbar_arrive(bar(BAR_VEMPTY + rs));  // the raw slot may be refilled
         } else {
           const uint32_t slot = sK + rs * C::kKSlot;
           const uint32_t src = slot + kRawOff + r0 * kHeadDim + c16 * 16;
@@ -1253,7 +1340,10 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       float* red = reinterpret_cast<float*>(smem + C::kRed) + g * 2 * 4 * 32;  // [2][4][32]
       float* lsum = reinterpret_cast<float*>(smem + C::kLsum) + g * 4 * 32;    // [4][32]
       const uint32_t bar_id = kBarGroup0 + g;
-      const float cs = fabsf(p.scale_log2);  // scores are scaled by cs >= 0 (log2 domain)
+      // Scores are scaled by cs >= 0 (log2 domain); a negative scale is an
+      // exact sign flip of every score, taken as the score is read.
+      const float cs = fabsf(p.scale_log2);
+      const float sgn = p.scale_log2 < 0.f ? -1.f : 1.f;
       constexpr int kSG = C::kSG;
 
       float lpart[RW], bias[RW];
@@ -1303,17 +1393,38 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         __syncwarp();
         return r != 0;
       };
+      int* pend = reinterpret_cast<int*>(smem + C::kPend) + g * kPendLen * 3;
+      int npend = 0, pend_last = -1;
+      // Count the listed partials in (the warpgroup's leader, after a barrier
+      // that follows every thread's stores): one fence, then the arrivals.
+      auto flush = [&]() {
+        if (widx == 0 && lane == 0 && npend > 0) {
+          __threadfence();
+          for (int i = 0; i < npend; ++i) {
+            const int* pe = pend + i * 3;
+            if (arrive(p, pe[0], pe[1], pe[2] != 0, 1)) {
+              const int k = atomicAdd(&misc->n_merge, 1);  // complete: merge it at the end
+              if (k < kMergeListLen) merge_list[k] = pe[0];
+            }
+          }
+          misc->segs_done[g] = pend_last + 1;
+        }
+        npend = 0;
+      };
       uint2 sc_next = make_uint2(0, 0);
       bool next_known = false;  // INFO(t) already waited for (scale prefetch)
       for (int t = 0;; ++t) {
-        // The warpgroup agrees to go on (every warp saw a live tile).
+        // This warp's view of tile t: live unless the stream ended or a wait
+        // gave up.  The warpgroup learns at its one barrier per tile (below)
+        // whether any warp is not live, and then stops together.
         bool live = ok && (next_known || info_wait(t));
-        live = live && info[t % kInfoSlots].seg >= 0;
-        if (!named_bar_and(bar_id, kSoftmaxThreads, live)) break;
         const TileInfo& ti = info[t % kInfoSlots];
-        const int seg = ti.seg, flags = ti.flags, key0 = ti.key0, vlo = ti.vis_lo, vhi = ti.vis_hi;
+        live = live && ti.seg >= 0;
+        ok = ok && live;
+        const int seg = live ? ti.seg : 0, flags = live ? ti.flags : 0;
+        const int key0 = ti.key0, vlo = live ? ti.vis_lo : 1, vhi = live ? ti.vis_hi : 0;
         const int sb = t % 2, st = t % VS, ob = seg % 2;
-        if (seg != seg_cur) {
+        if (live && seg != seg_cur) {
           // A new segment: its rows, its context and a fresh softmax state.
           const SegInfo& si = seginfo[seg % kSegSlots];
           seg_cur = seg;
@@ -1331,13 +1442,15 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         }
         uint2 sc = make_uint2(0, 0);
         if constexpr (kQuant) {
-          sc = next_known ? sc_next : fetch_scales(t);
-          next_known = false;
-          if (info_wait(t + 1)) {  // prefetch the next tile's scales
-            next_known = true;
-            if (info[(t + 1) % kInfoSlots].seg >= 0) sc_next = fetch_scales(t + 1);
-          } else {
-            ok = false;
+          if (live) {
+            sc = next_known ? sc_next : fetch_scales(t);
+            next_known = false;
+            if (info_wait(t + 1)) {  // prefetch the next tile's scales
+              next_known = true;
+              if (info[(t + 1) % kInfoSlots].seg >= 0) sc_next = fetch_scales(t + 1);
+            } else {
+              ok = false;
+            }
           }
         }
         float sv[RW];
@@ -1356,7 +1469,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
             const uint32_t kw[2] = {sc.x, sc.y};
 #pragma unroll
             for (int q = 0; q < kSG; ++q) {
-              const float dk = __half2float(__ushort_as_half((uint16_t)(kw[q / 2] >> (16 * (q % 2)))));
+              const float dk = sgn * __half2float(__ushort_as_half((uint16_t)(kw[q / 2] >> (16 * (q % 2)))));
 #pragma unroll
               for (int r = 0; r < RW; ++r) sv[r] = q == 0 ? dk * sg[0][r] : fmaf(dk, sg[q][r], sv[r]);
             }
@@ -1364,9 +1477,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
             tmem_ld<RW>(tmem + lane_off + sb * NR + row0, sv);
             tmem_ld_wait();
             if constexpr (kQuant) {  // int8 rows: K's row scale
-              const float dk = __uint_as_float(sc.x);
+              const float dk = sgn * __uint_as_float(sc.x);
 #pragma unroll
               for (int r = 0; r < RW; ++r) sv[r] *= dk;
+            } else if (sgn < 0.f) {
+#pragma unroll
+              for (int r = 0; r < RW; ++r) sv[r] = -sv[r];
             }
           }
           tc_fence_before();
@@ -1430,8 +1546,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         // barrier several times slower).
         __syncwarp();
         // One barrier per tile: orders the group's shared-memory traffic and
-        // tells every thread whether any score passed its row's reference.
-        const bool rescale = named_bar_or(bar_id, kSoftmaxThreads, exceed);
+        // counts the threads that are not live or saw a score pass their
+        // row's reference; only then (rarely) a second one tells the two
+        // apart, so that the whole warpgroup leaves the loop together.
+        const uint32_t flagged = named_bar_popc(bar_id, kSoftmaxThreads, !live || exceed);
+        if (flagged != 0 && named_bar_or(bar_id, kSoftmaxThreads, !live)) break;
+        const bool rescale = flagged != 0;
         if (rescale) {
           const uint32_t rm = all_vis ? 0xffffffffu : rm_g;
           float tmp[RW];
@@ -1591,17 +1711,24 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
                 : l > 0.f ? (fmaf(cs, m_lane, -(float)kPShift) + log2f(l)) * 0.69314718055994531f
                           : -INFINITY;
           }
-          __threadfence();  // the partial is visible before the group counts it in
-          named_bar_sync(bar_id, kSoftmaxThreads);
+          // Counted in later: a fence here would wait for these stores to
+          // drain behind the stream.  The warpgroup's barriers order every
+          // thread's stores before the leader's fence at the flush.
           if (widx == 0 && lane == 0) {
-            if (arrive(p, si.group, si.expect, si.first && g == 0, 1)) {
-              const int i = atomicAdd(&misc->n_merge, 1);  // complete: merge it at the end
-              if (i < kMergeListLen) merge_list[i] = si.group;
-            }
-            misc->segs_done[g] = seg + 1;
+            int* pe = pend + npend * 3;
+            pe[0] = si.group;
+            pe[1] = si.expect;
+            pe[2] = (si.first && g == 0) ? 1 : 0;
+          }
+          ++npend;
+          pend_last = seg;
+          if (npend == kPendLen) {
+            named_bar_sync(bar_id, kSoftmaxThreads);
+            flush();
           }
         }
       }
+      flush();          // the loop's exit barrier ordered the last stores
       __syncthreads();  // (A)
     }
     // ---- tear-down (every thread passed (A)) ---------------------------------

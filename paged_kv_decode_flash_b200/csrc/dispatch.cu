@@ -87,13 +87,15 @@ Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
   const long long groups = (long long)d->num_seqs * d->num_kv_heads * pl.halves;
   const long long max_tiles = ceil_div(max_chunks(d), kChunksPerTile);
   if (groups * 4 <= sms) {
-    // Few groups: each (sequence, part) gets an equal share of the SMs, at
-    // least one CTA per KV head (so that a CTA's range spans at most two of
-    // them) and at most one per tile of a full table.
+    // Few groups: each (sequence, part) gets an equal share of the SMs, the
+    // same number of CTAs for every KV head (so that a full table's cut
+    // falls on head boundaries and no CTA switches heads mid-stream), at
+    // least one and at most one per tile of a full table.
     const long long share = sms / ((long long)d->num_seqs * pl.halves);
+    const long long per_head =
+        std::max<long long>(1, std::min<long long>(share / d->num_kv_heads, max_tiles));
     pl.mode = 0;
-    pl.ctas_per_set = (int)std::max<long long>(
-        d->num_kv_heads, std::min<long long>(share, d->num_kv_heads * max_tiles));
+    pl.ctas_per_set = (int)(d->num_kv_heads * per_head);
     pl.ctas = (int)((long long)d->num_seqs * pl.halves * pl.ctas_per_set);
     pl.launches = 1;
     pl.slots = (long long)d->num_seqs * pl.halves * (pl.ctas_per_set + d->num_kv_heads);

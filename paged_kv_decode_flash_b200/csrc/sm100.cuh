@@ -108,6 +108,13 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   return v;
 }
 
+// Load at GPU scope without ordering (coherent, not cached in L1).
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Atomic add at GPU scope with release semantics, no value returned.
 __device__ __forceinline__ void red_release_add_gpu(int* p, unsigned int v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -148,6 +155,20 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t threads, bool
       : "r"(id), "r"(threads), "r"(static_cast<uint32_t>(v))
       : "memory");
   return r != 0;
+}
+
+// Named barrier that also counts the participating threads whose predicate
+// is true.
+__device__ __forceinline__ uint32_t named_bar_popc(uint32_t id, uint32_t threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi;\n\t"
+      "setp.ne.u32 pi, %3, 0;\n\t"
+      "bar.red.popc.u32 %0, %1, %2, pi;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(threads), "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r;
 }
 
 // Named barrier that also ANDs a predicate over the participating threads.
@@ -210,12 +231,63 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
                : "memory");
 }
 
+// An L2 policy that marks lines evict-first: streamed data that is read once
+// leaves the rest of L2 (code, tables, queries, partials) in place.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// The loads and prefetches above with an L2 cache policy.
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const void* tmap, int c0, int c1,
+                                                 int c2, int c3, uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d_hint(const void* tmap, int c0, int c1, int c2,
+                                                     int c3, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.4d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3, %4}], %5;" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2_hint(const void* src, uint32_t bytes, uint64_t pol) {
+  asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(src)),
+               "r"(bytes), "l"(pol)
+               : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared, L2 only (generic proxy: no
 // proxy fence is needed against data other threads wrote with plain stores).
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
                "l"(reinterpret_cast<uint64_t>(src))
                : "memory");
+}
+// The same with a source size: bytes past src_bytes (0 or 16) are zero.
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
+               : "memory");
+}
+// One arrival on an mbarrier once every cp.async this thread issued so far
+// has landed (the arrival is not counted in advance: the barrier's count
+// includes it).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 // Wait until every cp.async this thread issued has landed.
 __device__ __forceinline__ void cp_async_wait_all() {

@@ -126,9 +126,10 @@ def _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
     """(partial slots, rows per part) of the plan paged_attn_decode makes on
     a device with `sms` SMs (the planner in csrc/dispatch.cu, restated): the
     rows of a KV head in parts of at most 32 (fp16) or 16 (int8 caches);
-    few groups: an equal share of the SMs per (sequence, part), at least one
-    CTA per KV head, at most one per tile of a full table, plus one slot per
-    KV head; a batch: items of up to 16 tiles, the last cut into up to 4."""
+    few groups: an equal share of the SMs per (sequence, part), the same
+    number of CTAs for every KV head (at least one, at most one per tile of a
+    full table), plus one slot per KV head; a batch: items of up to 16
+    tiles, the last cut into up to 4."""
     R = nq * (Hq // Hkv)
     H = _ceil(R, 32 if kv_dtype == 0 else 16)
     RH = _ceil(R, H)
@@ -136,7 +137,7 @@ def _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
     max_chunks = mbps * bs // 16
     max_tiles = _ceil(max_chunks, 8)
     if groups * 4 <= sms:
-        ch = max(Hkv, min(sms // (B * H), Hkv * max_tiles))
+        ch = Hkv * max(1, min(sms // (B * H) // Hkv, max_tiles))
         return B * H * (ch + Hkv), RH
     T = min(16, max_tiles)
     return groups * (_ceil(max_chunks, 8 * T) - 1 + 4), RH
