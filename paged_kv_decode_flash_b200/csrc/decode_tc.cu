@@ -816,13 +816,25 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     auto stage_q = [&](const SegDesc& d, int qb) {
       const int rows = part_rows(p, d.h);
       const uint32_t dst = sQ + qb * C::kQBuf;
+      // Row n = 2k + lane / 16 of the part is token qi, head qg of the KV
+      // head's group (as out_row), stepped by two rows per piece.
+      const int cc = lane % 16, gr0 = d.h * p.rows_half + lane / 16;
+      int qi = gr0 / p.group, qg = gr0 - qi * p.group;
+      const __half* base =
+          p.q + ((long long)d.s * p.n_query * p.num_q_heads + (long long)d.kvh * p.group) * kHeadDim +
+          cc * 8;
 #pragma unroll
       for (int k = 0; k < kQPer; ++k) {
-        const int e = k * 32 + lane, n = e / 16, cc = e % 16;
+        const int n = 2 * k + lane / 16;
         const bool in = n < rows;
-        const __half* src = in ? p.q + out_row(p, d.s, d.kvh, d.h, n) * kHeadDim + cc * 8 : p.q;
+        const __half* src = in ? base + ((long long)qi * p.num_q_heads + qg) * kHeadDim : p.q;
         cp_async_16_zfill(dst + (cc / 8) * C::kQHalf + n * 128 + (((cc % 8) ^ (n & 7)) * 16), src,
                           in ? 16u : 0u);
+        qg += 2;
+        while (qg >= p.group) {
+          qg -= p.group;
+          ++qi;
+        }
       }
       cp_async_mbar_arrive_noinc(bar(BAR_QFULL + qb));
     };
@@ -1783,7 +1795,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
     if (!misc->last) return;
     const int P = misc->own_rows * (kHeadDim / 4);
     const int sl = misc->own_slice, ns = misc->own_slices;
-    const int pa = (int)((long long)sl * P / ns), pb = (int)((long long)(sl + 1) * P / ns);
+    const int pa = sl * P / ns, pb = (sl + 1) * P / ns;  // P <= 64 * 32, sl < 4096: no overflow
     const long long slot0 = (long long)(misc->own_s * H + misc->own_h) * (p.ctas_per_set + Hkv) +
                             misc->own_first + misc->own_group;
     merge_pairs<kThreads>(p, slot0, misc->own_count, misc->own_rows, misc->own_s, misc->own_group,
