@@ -50,6 +50,10 @@ int32_t paged_attn_num_splits(const pa_dims* dims, int32_t n_query, int32_t kv_d
   if (sms <= 0) return PA_ERR_CUDA;
   const Plan pl = make_plan(dims, n_query, kv_dtype, sms);
   if (pl.mode == 1) return pl.slots_per_group;
+  if (pl.split_ctas > 0) {  // the per-head split kernel: CTAs per (sequence, KV head)
+    const int groups = dims->num_seqs * dims->num_kv_heads;
+    return (pl.split_ctas + groups - 1) / groups;
+  }
   // A KV head's chunks span ceil(Ce / Hkv) ranges, plus one where they start
   // inside a range.
   return (pl.ctas_per_set + dims->num_kv_heads - 1) / dims->num_kv_heads + 1;

@@ -145,7 +145,10 @@ struct SegInfo {
   int first;            // this segment makes the group's designated first arrival
   int expect;           // arrivals the group expects (segments x softmax warpgroups)
   int bad;              // a block index out of range was replaced by block 0
-  int pad[6];
+  int key_first;        // key of the segment's first tile
+  int ntile;            // the segment's tiles
+  int vis_lo, vis_hi;   // the keys of the segment that some row sees
+  int pad[2];
 };
 static_assert(sizeof(SegInfo) == 64, "SegInfo layout");
 
@@ -903,6 +906,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         si.L = cur.L; si.rows = part_rows(p, cur.h);
         si.group = (cur.s * Hkv + cur.kvh) * H + cur.h;
         si.first = cur.first; si.expect = cur.expect; si.bad = 0;
+        si.key_first = cur.base + cur.c0 * kChunk;
+        si.ntile = (cur.c1 - cur.c0 + kChunksPerTile - 1) / kChunksPerTile;
+        si.vis_lo = cur.vis_lo; si.vis_hi = cur.vis_hi;
       }
       seg_written = seg_n + 1;
       __syncwarp();
@@ -911,7 +917,6 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       if (lane == 0) w = wait(BAR_QEMPTY + qb, ((seg_n / 2) & 1) ^ 1);
       ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       if (!ok) break;
-      stage_q(cur, qb);
       const int ntile = (cur.c1 - cur.c0 + kChunksPerTile - 1) / kChunksPerTile;
       planned = false;
       for (int tau = 0; tau < ntile; ++tau) {
@@ -961,6 +966,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         }
         __syncwarp();
         if (tau == 0) {
+          // The segment's Q rows, behind its first K copies (QK(first) waits
+          // for both).
+          stage_q(cur, qb);
           have_nxt = next_segment(nxt);
           planned = true;
           if (have_nxt) raw_first_nxt = lookup(nxt, nxt.c0);
@@ -1365,8 +1373,8 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         bias[r] = INFINITY;
       }
       float m_lane = -INFINITY;  // reference max (raw score) of row row0 + lane % RW
-      int seg_cur = -1, seg_rows = 0, seg_L = 0, seg_h = 0;
-      uint32_t all_rows = 0;
+      int seg_cur = -1, seg_rows = 0, seg_L = 0, seg_h = 0, lo_all = 0, hi_all = -1;
+      uint32_t all_rows = 0, part_rows_mask = 0;
       bool ok = true;
       int o_seen = 0;  // PV phases known to be complete
       // Wait until PV(k) has finished: exact while phases < k are complete
@@ -1408,10 +1416,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       int* pend = reinterpret_cast<int*>(smem + C::kPend) + g * kPendLen * 3;
       int npend = 0, pend_last = -1;
       // Count the listed partials in (the warpgroup's leader, after a barrier
-      // that follows every thread's stores): one fence, then the arrivals.
+      // that follows every thread's stores).  Mode 0 arrives with a release
+      // reduction, which publishes the warpgroup's stores (ordered before it
+      // by the barrier); mode 1's arrivals return a value: a fence first.
       auto flush = [&]() {
         if (widx == 0 && lane == 0 && npend > 0) {
-          __threadfence();
+          if (p.mode != 0) __threadfence();
           for (int i = 0; i < npend; ++i) {
             const int* pe = pend + i * 3;
             if (arrive(p, pe[0], pe[1], pe[2] != 0, 1)) {
@@ -1425,16 +1435,34 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
       };
       uint2 sc_next = make_uint2(0, 0);
       bool next_known = false;  // INFO(t) already waited for (scale prefetch)
+      // fp16 without the trace: a tile's description is read only at the
+      // first tile of a segment; the others follow from the segment's.
+      constexpr bool kSegDriven = !kQuant && !TR;
+      int seg_left = 0, seg_key = 0, seg_vlo = 1, seg_vhi = 0;
       for (int t = 0;; ++t) {
         // This warp's view of tile t: live unless the stream ended or a wait
         // gave up.  The warpgroup learns at its one barrier per tile (below)
         // whether any warp is not live, and then stops together.
-        bool live = ok && (next_known || info_wait(t));
         const TileInfo& ti = info[t % kInfoSlots];
-        live = live && ti.seg >= 0;
+        bool live;
+        int seg, flags, key0, vlo, vhi;
+        if (kSegDriven && seg_left > 0) {
+          live = ok;
+          seg = seg_cur;
+          flags = seg_left == 1 ? 2 : 0;
+          key0 = seg_key;
+          vlo = seg_vlo;
+          vhi = seg_vhi;
+        } else {
+          live = ok && (next_known || info_wait(t));
+          live = live && ti.seg >= 0;
+          seg = live ? ti.seg : 0;
+          flags = live ? ti.flags : 0;
+          key0 = ti.key0;
+          vlo = live ? ti.vis_lo : 1;
+          vhi = live ? ti.vis_hi : 0;
+        }
         ok = ok && live;
-        const int seg = live ? ti.seg : 0, flags = live ? ti.flags : 0;
-        const int key0 = ti.key0, vlo = live ? ti.vis_lo : 1, vhi = live ? ti.vis_hi : 0;
         const int sb = t % 2, st = t % VS, ob = seg % 2;
         if (live && seg != seg_cur) {
           // A new segment: its rows, its context and a fresh softmax state.
@@ -1443,8 +1471,27 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
           seg_rows = si.rows;
           seg_L = si.L;
           seg_h = si.h;
+          seg_left = si.ntile;
+          seg_key = si.key_first;
+          seg_vlo = si.vis_lo;
+          seg_vhi = si.vis_hi;
           const int vr = min(RW, max(0, seg_rows - row0));
           all_rows = vr >= 32 ? 0xffffffffu : ((1u << vr) - 1u);
+          part_rows_mask = seg_rows >= 32 ? 0xffffffffu : ((1u << seg_rows) - 1u);
+          // The keys every row of the part sees (tokens i_first .. i_last):
+          // [lo_all, hi_all], where the row mask is the whole part.
+          {
+            const int off = seg_h * p.rows_half;
+            const int i_first = off / p.group, i_last = (off + seg_rows - 1) / p.group;
+            const int p0 = seg_L - p.n_query;
+            if (p.causal) {
+              lo_all = p.window > 0 ? max(0, p0 + i_last - p.window + 1) : 0;
+              hi_all = min(seg_L - 1, p0 + i_first);
+            } else {
+              lo_all = p.window > 0 ? max(0, seg_L - p.window) : 0;
+              hi_all = seg_L - 1;
+            }
+          }
           m_lane = -INFINITY;
 #pragma unroll
           for (int r = 0; r < RW; ++r) {
@@ -1506,7 +1553,9 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         // contiguous run, whose rows are a contiguous run of bits.
         const int key = key0 + j;
         uint32_t rmask = 0;
-        if (ok && key >= vlo && key <= vhi) {
+        if (ok && key >= vlo && key <= vhi && key >= lo_all && key <= hi_all) {
+          rmask = part_rows_mask;  // the interior: every row of the part
+        } else if (ok && key >= vlo && key <= vhi) {
           int i_lo, i_hi;
           tokens_seeing(seg_L, p.n_query, p.causal, p.window, key, i_lo, i_hi);
           const int off = seg_h * p.rows_half;
@@ -1548,10 +1597,18 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         // raise the row's reference.
         float x[RW];
         float xmax = -INFINITY;
+        if (all_vis) {
 #pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          x[r] = (all_vis || ((rm_g >> r) & 1u)) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
-          xmax = fmaxf(xmax, x[r]);
+          for (int r = 0; r < RW; ++r) {
+            x[r] = fmaf(sv[r], cs, bias[r]);
+            xmax = fmaxf(xmax, x[r]);
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            x[r] = ((rm_g >> r) & 1u) ? fmaf(sv[r], cs, bias[r]) : -INFINITY;
+            xmax = fmaxf(xmax, x[r]);
+          }
         }
         const bool exceed = xmax > (float)kPShift + kLazy;
         // Reconverge before the group barrier (a diverged arrival makes the
@@ -1625,7 +1682,7 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
         // fp16 cache: a key no row of the part sees must not reach the PV
         // product: zero its V row once the V tile has landed (the int8
         // converters write such rows as zeros themselves).
-        if (!kQuant && g == 0 && __any_sync(0xffffffffu, ok && rmask == 0)) {
+        if (!kQuant && g == 0 && !all_vis && __any_sync(0xffffffffu, ok && rmask == 0)) {
           ok = __all_sync(0xffffffffu, ok && wait(BAR_VFULL + st, (t / VS) & 1));
           if (ok && rmask == 0) {
             const uint4 z = make_uint4(0, 0, 0, 0);
@@ -1739,6 +1796,8 @@ __global__ void __launch_bounds__(Cfg<RW, NG, KV>::kThreads, 1)
             flush();
           }
         }
+        --seg_left;
+        seg_key += kTileKeys;
       }
       flush();          // the loop's exit barrier ordered the last stores
       __syncthreads();  // (A)

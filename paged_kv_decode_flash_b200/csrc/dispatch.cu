@@ -99,6 +99,16 @@ Plan make_plan(const pa_dims* d, int n_query, int kv_dtype, int sms) {
     pl.ctas = (int)((long long)d->num_seqs * pl.halves * pl.ctas_per_set);
     pl.launches = 1;
     pl.slots = (long long)d->num_seqs * pl.halves * (pl.ctas_per_set + d->num_kv_heads);
+    // fp16, at most 8 tokens and 32 rows (one part): the per-head split
+    // kernel, one CTA per SM shared out among the (sequence, KV head) groups
+    // (at least one each, no more than a full table's tiles).  Its CTA-
+    // indexed partials fit in the slots above: groups x (SMs / groups + 1)
+    // >= its CTAs.
+    const long long kv_groups = (long long)d->num_seqs * d->num_kv_heads;
+    if (pl.halves == 1 &&
+        split_decode_supported(kv_dtype, n_query, n_query * (d->num_q_heads / d->num_kv_heads),
+                               d->num_blocks, d->num_kv_heads, d->block_size))
+      pl.split_ctas = (int)std::max(kv_groups, std::min<long long>(sms, kv_groups * max_tiles));
   } else {
     // A batch: items of T tiles (the last one of a group in up to four
     // pieces) from a queue, one CTA per SM; one launch per kMaxQueueSeqs
@@ -214,7 +224,13 @@ int enqueue_decode(const pa_dims* d, const Plan& plan, const void* q, const void
   p.key_count = partial.key_count;
   p.out_f32 = partial.out;
   p.out_lse = partial.out_lse;
-  if (plan.mode == 0) return launch_decode_tc(p, st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  if (plan.mode == 0) {
+    // Every key of the context (no context-parallel key range): the per-head
+    // split kernel where the plan chose it.
+    if (plan.split_ctas > 0 && partial.key_begin == nullptr)
+      return launch_split_decode(p, plan.split_ctas, st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_decode_tc(p, st) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  }
   // Mode 1: one launch per kMaxQueueSeqs sequences, each with its own
   // counters and partial slots.
   const long long rows_per_seq = (long long)n_query * d->num_q_heads;

@@ -23,6 +23,7 @@ struct Plan {
   int slots_per_group;  // mode 1: partial slots per group
   int launches;         // kernel launches of the call
   long long slots;      // partial slots of the whole call
+  int split_ctas;       // > 0: the call runs the per-head split kernel on this many CTAs
 };
 
 // Workspace: status header | arrival counters (two per group) | queue

@@ -15,6 +15,16 @@ cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream);
 // Most query rows one CTA handles per KV head for a cache type.
 int max_rows_per_part(int kv_dtype);
 
+// The per-head split kernel (decode_split.cu): fp16 cache, few (sequence,
+// KV head) groups, up to 8 query tokens and 32 rows per KV head, every key
+// of the context.  Each group's 128-key tiles are cut into contiguous runs
+// over its share of `ctas` CTAs; partial slots are CTA-indexed (rows
+// [cta * rows, cta * rows + rows)); merge included; records the trace when
+// p.trace is set.  Only p's fields of a mode-0 plan are read.
+bool split_decode_supported(int kv_dtype, int n_query, int rows, int num_blocks,
+                            int num_kv_heads, int block_size);
+cudaError_t launch_split_decode(const DecodeParams& p, int ctas, cudaStream_t stream);
+
 // Log-sum-exp merge of split partials into fp16 rows.
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
