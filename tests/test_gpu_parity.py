@@ -392,9 +392,11 @@ def test_decode_kernel_trace_is_bit_exact(B, orc):
     """The decode kernel's own record of every (row, key) pair it scored and
     the physical slot it copied that key's K row from -- count, first and
     last key, xor and sum of the slot ids -- equals the oracle's, bit for
-    bit, over every kernel configuration (fp16 / q8_0 / int8 rows, few
-    groups / work queue, one or several row parts).  The traced call's
-    output is bit-identical to the plain call's."""
+    bit, over both kernels (the per-head split kernel: fp16, few groups, up
+    to 8 tokens and 32 rows; the segment kernel: the rest) and every
+    configuration (fp16 / q8_0 / int8 rows, few groups / work queue, one or
+    several row parts).  The traced call's output is bit-identical to the
+    plain call's."""
     for case in _trace_cases():
         dev, args, kw = _args(B, case)
         dec = B.PagedDecode.for_case(case)
