@@ -262,9 +262,12 @@ def bench_ours(args, rank, world, dist):
         case = make_workload(name, seed=rank)
         kv_bytes = gen.visible_kv_bytes(case)
         pool_bytes = case.k_cache.nbytes + case.v_cache.nbytes
-        # Inputs larger than L2: enough copies of the pool that the VISIBLE
-        # bytes the rotated calls read add up to 3x L2 (at most 48 GB of copies).
-        copies = max(2, math.ceil(3 * l2_bytes / kv_bytes))
+        # Inputs larger than L2: at least four copies of the pool, and enough
+        # that the VISIBLE bytes the rotated calls read add up to 3x L2 (at
+        # most 48 GB of copies).  With two copies of a 252 MB pool, lines of
+        # the call before last measurably survived in L2 (0.5 us at 61k, 2.8
+        # us with every cache line marked evict-first); with four, none do.
+        copies = max(4, math.ceil(3 * l2_bytes / kv_bytes))
         copies = max(2, min(copies, int(48e9 // pool_bytes)))
         base = B.case_to_device(case, device)
         pools = [(base["k_cache"], base["v_cache"])]
