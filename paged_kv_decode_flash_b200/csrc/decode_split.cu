@@ -52,19 +52,13 @@
 // zero-filled in shared memory before the PV product (the NaN-poisoned
 // out-of-window blocks of the pages' regression test must not leak).
 //
-// q8_0 cache (int8 qs with one fp16 scale d per 32 head_dim elements): the
-// scale stays out of the operands, so that they remain exact without a
-// high/residual split.  K's operand is qs; S^T gets one TMEM accumulator per
-// scale group, and the softmax forms each score as the sum over the groups of
-// K's scale times the group's partial product, in fp32.  V's operand is
-// qs * 2^e, with d = m * 2^e split into its power of two and its mantissa m;
-// P gets one copy per scale group with the weights multiplied by that
-// group's m (then split into fp16 parts as above), and each group has its
-// own O^T accumulator, of which a head_dim lane reads only its own group's.
-// The softmax reads the scales of its keys from the cache (L2) a tile ahead.
-// Batches with many (sequence, KV head) groups cut every group's tiles into
-// fixed-size items, one CTA each, over several waves; the size depends on
-// the shapes only, so a sequence's output does not depend on the others.
+// The template keeps a q8_0 variant (scales kept out of the operands: K's
+// applied to the per-group scores, V's power of two folded into the operand
+// and its mantissa into one P copy per scale group), which the library does
+// not instantiate: int8 caches run the segment kernel (decode_tc.cu).
+// (The kernel can also cut every group's tiles into fixed-size items, one CTA
+// each, over several waves; the library uses it only with few groups, one
+// wave, where each group's CTAs take contiguous runs of its tiles.)
 //
 // Merge: every CTA writes its fp32 partial (O, lse).  With a cooperative
 // launch (every CTA resident) the CTAs of one (sequence, KV head) meet at a
