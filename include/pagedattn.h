@@ -54,8 +54,12 @@
  *   context_lens  int32 [num_seqs]
  * Supported: head_dim 128; block_size a multiple of 16 (the kernels work in
  * 16-key chunks; sizes 16 to 112 are exercised by the tests); n_query
- * 1..16; num_q_heads a multiple of num_kv_heads with
- * n_query * num_q_heads / num_kv_heads <= 64.
+ * 1..128; num_q_heads a multiple of num_kv_heads with
+ * n_query * num_q_heads / num_kv_heads <= 1024.  A KV head's rows are cut
+ * into parts of at most 32 (fp16) or 16 (int8 caches) rows, each of which
+ * reads the keys its tokens see: a chunk of many tokens (a long verify, a
+ * prefill chunk appended to the cache) costs one pass over its visible KV
+ * per part.
  *
  * Ownership and synchronisation: the caller owns every buffer, including the
  * workspace.  Calls allocate nothing, never synchronise the host with the
@@ -122,7 +126,7 @@ int paged_attn_workspace_init(const pa_dims* dims, void* stream);
 
 /* Decode attention (see the header comment for the exact definition).
  * q, k_cache, v_cache, block_table, context_lens, out: device pointers,
- * 16-byte aligned.  n_query in 1..16; causal 0 or 1; window >= 0 (0 = no
+ * 16-byte aligned.  n_query in 1..128; causal 0 or 1; window >= 0 (0 = no
  * window); scale multiplies q.k (usually 1/sqrt(head_dim)); kv_dtype a
  * pa_kv_dtype.  Enqueues the split-KV kernel, whose CTAs also merge the
  * split partials, on `stream` (see paged_attn_launches_per_call).  Calls

@@ -14,8 +14,8 @@
 namespace pa {
 
 constexpr int kHeadDim = 128;          // the only head_dim the decode kernels take
-constexpr int kMaxRows = 64;           // n_query * (Hq / Hkv) rows per KV head
-constexpr int kMaxQuery = 16;
+constexpr int kMaxRows = 1024;         // n_query * (Hq / Hkv) rows per KV head
+constexpr int kMaxQuery = 128;        // new tokens per call (chunked verify / prefill)
 constexpr size_t kWsHeader = 256;      // status header at the start of the workspace
 constexpr int kChunk = 16;             // keys per gather unit (block_size % 16 == 0)
 constexpr int kTileKeys = 128;         // keys per pipeline tile

@@ -58,7 +58,7 @@ def test_workspace_size_host_only(L):
     for bad in (dims(num_q_heads=30), dims(block_size=8), dims(head_dim=64), dims(num_seqs=0)):
         assert L.paged_attn_workspace_size(ctypes.byref(bad), 8) == 0
     assert L.paged_attn_workspace_size(ctypes.byref(d), 0) == 0
-    assert L.paged_attn_workspace_size(ctypes.byref(d), 17) == 0
+    assert L.paged_attn_workspace_size(ctypes.byref(d), 129) == 0
     assert L.paged_attn_workspace_size(None, 1) == 0
 
 
@@ -77,15 +77,15 @@ def test_decode_rejects_bad_arguments_on_host(L):
     assert call(None, args()) == b.PA_ERR_INVALID_ARG
     assert call(d, args(q=None)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(nq=0)) == b.PA_ERR_INVALID_ARG
-    assert call(d, args(nq=17)) == b.PA_ERR_INVALID_ARG
+    assert call(d, args(nq=129)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(causal=2)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(window=-1)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(dt=7)) == b.PA_ERR_INVALID_ARG
     assert call(d, args(scale=float("nan"))) == b.PA_ERR_INVALID_ARG
     assert call(d, args(q=ctypes.c_void_p((1 << 20) + 2))) == b.PA_ERR_INVALID_ARG  # misaligned
     assert call(dims(head_dim=64, workspace=4096, workspace_bytes=1 << 30), args()) == b.PA_ERR_UNSUPPORTED
-    assert call(dims(num_q_heads=128, num_kv_heads=8, workspace=4096, workspace_bytes=1 << 30),
-                args()) == b.PA_ERR_UNSUPPORTED  # 8 tokens x 16 heads per KV head > 64 rows
+    assert call(dims(num_q_heads=8 * 129, num_kv_heads=8, workspace=4096, workspace_bytes=1 << 30),
+                args()) == b.PA_ERR_UNSUPPORTED  # 8 tokens x 129 heads per KV head > 1024 rows
     assert call(dims(workspace=None), args()) == b.PA_ERR_WORKSPACE
     assert call(dims(workspace=4100, workspace_bytes=1 << 30), args()) == b.PA_ERR_WORKSPACE
 
@@ -122,6 +122,9 @@ def _align(x):
     return (x + 255) & ~255
 
 
+MAX_PARTS = 1024 // 16  # counters cover the most row parts any call uses (1024 rows in parts of 16)
+
+
 def _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
     """(partial slots, rows per part) of the plan paged_attn_decode makes on
     a device with `sms` SMs (the planner in csrc/dispatch.cu, restated): the
@@ -145,15 +148,15 @@ def _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
 
 def _ws_needed(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms):
     slots, RH = _plan(B, Hq, Hkv, bs, mbps, nq, kv_dtype, sms)
-    prefix = 256 + _align(B * Hkv * 4 * 2 * 4) + _align(_ceil(B, 256) * 4)
+    prefix = 256 + _align(B * Hkv * MAX_PARTS * 2 * 4) + _align(_ceil(B, 256) * 4)
     return prefix + _align(slots * RH * 128 * 4) + _align(slots * RH * 4)
 
 
 def test_workspace_size_covers_every_plan(L):
     """paged_attn_workspace_size needs no device, so it must cover the plan
     of any device and any cache type: every SM count up to 1024, every
-    block size (a multiple of 16 up to 128), row counts that need one, two,
-    three or four row parts."""
+    block size (a multiple of 16 up to 128), 1 to 128 query tokens: row
+    counts that need one to 64 row parts."""
     import numpy as np
     rng = np.random.default_rng(7)
     shapes = [(1, 32, 8, 16, 3841, 8), (1, 32, 4, 16, 12288, 1), (8, 32, 8, 16, 4096, 4),
@@ -163,9 +166,9 @@ def test_workspace_size_covers_every_plan(L):
         Hkv = int(rng.choice([1, 2, 4, 8]))
         shapes.append((int(rng.integers(1, 40)), Hkv * int(rng.choice([1, 2, 4, 8])), Hkv,
                        16 * int(rng.integers(1, 9)), int(rng.integers(1, 5000)),
-                       int(rng.integers(1, 17))))
+                       int(rng.choice([1, 2, 4, 8, 16, 33, 64, 128]))))
     for B, Hq, Hkv, bs, mbps, nq in shapes:
-        if nq * (Hq // Hkv) > 64:
+        if nq * (Hq // Hkv) > 1024:
             continue
         d = dims(num_seqs=B, num_q_heads=Hq, num_kv_heads=Hkv, block_size=bs,
                  max_blocks_per_seq=mbps, num_blocks=mbps * B + 1)

@@ -152,6 +152,23 @@ def test_sixteen_token_verify(B, orc):
             assert_parity(out, ref, f"nq 16 window {window} dt {dt}")
 
 
+@pytest.mark.parametrize("dt", DTYPES)
+def test_chunked_prefill_of_many_tokens(B, orc, dt):
+    """A chunk of 64 new tokens appended to the cache (chunked prefill),
+    GQA 4: 256 rows per KV head in 8 (fp16) or 16 (int8) row parts, each
+    over the keys its tokens see, causal, with and without a window; and
+    128 tokens x 8 query heads per KV head (1024 rows, the most) on a short
+    context.  Every row against the oracle."""
+    for nq, Hq, Hkv, lens, window in ((64, 16, 4, (2500, 300), 0), (64, 16, 4, (2500, 300), 700),
+                                      (128, 8, 1, (400,), 0)):
+        case = gen.make_case(seed=170 + nq + window, context_lens=lens, n_query=nq,
+                             num_q_heads=Hq, num_kv_heads=Hkv, causal=1, window=window,
+                             kv_dtype=dt)
+        out, _ = run(B, case)
+        ref, _ = orc.attend(case)
+        assert_parity(out, ref, f"nq {nq} rows {nq * Hq // Hkv} window {window} dt {dt}")
+
+
 @pytest.mark.parametrize("bs,dt", [(48, gen.KV_FP16), (80, gen.KV_Q8_0), (112, gen.KV_FP16),
                                    (96, gen.KV_INT8_ROW)])
 def test_block_sizes_that_do_not_divide_a_tile(B, orc, bs, dt):
@@ -386,6 +403,9 @@ def _trace_cases():
                         num_kv_heads=4, causal=1, window=2500, kv_dtype=gen.KV_INT8_ROW)
     yield gen.make_case(seed=132, context_lens=(6000, 333), n_query=16, num_q_heads=16,
                         num_kv_heads=4, causal=0, window=1000, nan_keys_below=[5000, 0])
+    # a prefill chunk: 40 tokens x 4 heads = 160 rows in five parts
+    yield gen.make_case(seed=133, context_lens=(1500,), n_query=40, num_q_heads=8,
+                        num_kv_heads=2, causal=1, window=600)
 
 
 def test_decode_kernel_trace_is_bit_exact(B, orc):
