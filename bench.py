@@ -62,9 +62,12 @@ WORKLOAD_TEXT = {
     "mtp_int8_row_61k": "the same shape over an int8 cache with fp32 row scales",
     "verify_64rows_61k": "8-token verify at GQA 8 (64 rows per KV head): B=1, Hq/Hkv=64/8, "
                          "L=61448, fp16",
+    "prefill_chunk_16k": "a chunk of 64 new tokens appended to a 16320-token cache (L=16384, "
+                         "causal): B=1, Hq/Hkv=32/8 (256 rows per KV head, eight row parts "
+                         "of 32), fp16",
 }
 OTHER_CONFIGS = ("tiny", "sliding_window", "mixed_q8_0", "mtp_q8_0_61k", "mtp_int8_row_61k",
-                 "verify_64rows_61k")
+                 "verify_64rows_61k", "prefill_chunk_16k")
 
 
 def make_workload(name, seed=0):
@@ -77,6 +80,9 @@ def make_workload(name, seed=0):
     if name == "verify_64rows_61k":
         return gen.make_case(name=name, seed=seed, context_lens=(61448,), n_query=8,
                              num_q_heads=64, num_kv_heads=8, causal=1)
+    if name == "prefill_chunk_16k":
+        return gen.make_case(name=name, seed=seed, context_lens=(16384,), n_query=64,
+                             num_q_heads=32, num_kv_heads=8, causal=1)
     raise KeyError(name)
 
 
