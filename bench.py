@@ -185,7 +185,7 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (FileNotFoundError, OSError):
             self.proc = None
-        time.sleep(0.15)
+        time.sleep(0.5)  # nvidia-smi's start-up (driver queries) is over before timing
         return self
 
     def __exit__(self, *a):
@@ -317,6 +317,9 @@ def bench_ours(args, rank, world, dist):
         # first is the reported one, all `reps` give the spread.
         times = []
         with ClockSampler(dev_index) as clk:
+            with torch.cuda.stream(gstream):  # one more untimed replay, under the sampler
+                graph.replay()
+            torch.cuda.synchronize()
             for _ in range(reps):
                 t0 = torch.cuda.Event(enable_timing=True)
                 t1 = torch.cuda.Event(enable_timing=True)

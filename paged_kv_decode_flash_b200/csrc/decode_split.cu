@@ -639,10 +639,12 @@ __global__ void __launch_bounds__(Cfg<RW, NG, Q8>::kThreads, 1)
     }
   }
   // Group barrier of the cooperative merge (below): its phase bit, read
-  // before this CTA arrives (it cannot flip before then).
+  // before this CTA arrives (it cannot flip before then).  A relaxed load:
+  // it stays in flight while this thread (the K producer's lane 0) goes on;
+  // an acquire would hold back its every later access until it returns.
   int* cnt = p.arrivals + ((long long)s * p.num_kv_heads + kvh) * 2;
   unsigned int bar_phase = 0;
-  if (p.coop && threadIdx.x == 0) bar_phase = (unsigned int)ld_acquire_gpu(cnt) & 0x80000000u;
+  if (p.coop && threadIdx.x == 0) bar_phase = (unsigned int)ld_relaxed_gpu(cnt) & 0x80000000u;
   // Partials: CTA c owns rows [c*R, c*R + R) of the partial outputs and
   // log-sum-exps; the CTAs of one group are consecutive.
   const long long part_base = (long long)cta * R;
