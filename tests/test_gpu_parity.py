@@ -494,6 +494,27 @@ def test_cuda_graph_replay_matches_eager(B):
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
 
 
+def test_split_kernel_gives_every_kv_head_the_same_ctas(B):
+    """fp16 calls with few (sequence, KV head) groups run the per-head split
+    kernel with the same number of CTAs for every group -- SMs // groups,
+    at least one, at most one per 128-key tile of a full table -- so that no
+    head with one CTA fewer finishes last while the others idle."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # (B, Hq, Hkv, max_blocks_per_seq, n_query) at block size 16: the 61k
+    # verify, the 200k decode, the tiny and sliding-window calls, two
+    # sequences with short tables
+    for nseq, hq, hkv, mbps, nq in ((1, 32, 8, 3841, 8), (1, 32, 4, 12288, 1), (1, 8, 2, 64, 1),
+                                    (1, 32, 8, 1536, 8), (2, 16, 4, 100, 4)):
+        groups = nseq * hkv
+        dec = B.PagedDecode(num_seqs=nseq, num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+                            block_size=16, max_blocks_per_seq=mbps, num_blocks=nseq * mbps,
+                            n_query=nq)
+        max_tiles = -(-mbps // 8)
+        assert dec.num_splits(B.KV_FP16) == max(1, min(sms // groups, max_tiles)), \
+            (nseq, hq, hkv, mbps, nq)
+
+
 @pytest.mark.parametrize("name", ["spec_verify_61k", "mixed_q8_0"])
 def test_waits_that_time_out_leave_the_workspace_usable(B, orc, name):
     """A wait limit the pipeline cannot meet (1 ns): every kernel gives up
